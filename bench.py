@@ -1,0 +1,430 @@
+"""Benchmark of the sigmoid-routed MoE block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = route + permute + expert up-projection + down-projection + combine
+over one batch of synthetic tokens (the whole hot path), inputs resident in HBM.
+Default workload: the GLM-5-shaped prefill block (16384 tokens, H 6144, 256
+experts top-8 + 1 shared, I 2048).  Prints ONE JSON line on rank 0.
+
+N > 1 runs independent replicas, one per GPU (the layer has no cross-token
+term, so each rank processes its own batch; no data-path collective): weak
+scaling, value = tokens of all ranks / max over ranks of the device time.
+
+--impl reference times the CPU oracle (the slow, plain statement of the
+method, double precision, OpenMP) on the host cores, each step a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sigmoid_routed_mixture_b200 import workloads as W  # noqa: E402
+
+METRIC = "MoE-block tokens/s (GLM-5 shape, bf16, 1 B200)"
+UNIT = "tokens/s"
+KERNELS_PER_STEP = 7  # route 1 + permute 3 + up 1 + down 1 + combine 1
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return dict(hbm=float(p["hbm_gbs"]), tflops=float(p["bf16_tflops"]),
+                    tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, tflops=1590.0, tflops_sustained=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.tmp = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        self.proc = None
+        self.dev = device_index
+
+    def start(self):
+        try:
+            ids = os.environ.get("CUDA_VISIBLE_DEVICES")
+            gpu = ids.split(",")[self.dev] if ids else str(self.dev)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + CLOCK_FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", gpu], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = [r.split(",") for r in open(self.tmp.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.tmp.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle sample
+
+def oracle_sample_tokens(w, counts_of_token_experts, n_tokens, max_experts=48):
+    """Token sample for the CPU oracle: tokens whose K experts all lie among the
+    `max_experts` most loaded ones (bounds the weights the host must hold; the
+    oracle's cost per token does not depend on which experts it uses)."""
+    idx = counts_of_token_experts
+    load = np.bincount(idx.reshape(-1), minlength=w.E)
+    top = set(np.argsort(-load)[:max_experts].tolist())
+    cand = [t for t in range(idx.shape[0]) if set(idx[t].tolist()) <= top]
+    if len(cand) < n_tokens:
+        cand = list(range(min(n_tokens, idx.shape[0])))
+    return np.array(cand[:n_tokens], dtype=np.int64)
+
+
+def run_oracle_steps(w, x, w_r, b, tokens, expert_tables, shared, steps):
+    """Time route + permute + forward of the oracle on `tokens`, `steps` times."""
+    from oracle import oracle as O
+
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        idx, gate, margin, z = O.route(x[tokens], w_r, b, w.K, w.scale)
+        O.permute(idx, w.E, w.has_shared)
+        O.forward(x[tokens], expert_tables[0], expert_tables[1], expert_tables[2], shared[0], shared[1],
+                  shared[2], idx, gate, has_shared=w.has_shared)
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def host_expert_tables(w, experts, getter):
+    t1 = [getter("w1", e) if e in experts else None for e in range(w.E)]
+    t3 = [getter("w3", e) if e in experts else None for e in range(w.E)]
+    t2 = [getter("w2", e) if e in experts else None for e in range(w.E)]
+    return t1, t3, t2
+
+
+def cores():
+    return len(os.sched_getaffinity(0))
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores()))
+    from oracle import oracle as O
+
+    O.build()
+    w = W.WORKLOADS[args.workload]
+    x, w_r, b = W.router_inputs(w)
+    idx, _, _, _ = O.route(x[: min(w.T, 4096)], w_r, b, w.K, w.scale)
+    n = max(1, min(args.ref_tokens or 2 * cores(), w.T))
+    tokens = oracle_sample_tokens(w, idx, n)
+    sel, _, _, _ = O.route(x[tokens], w_r, b, w.K, w.scale)
+    experts = set(np.unique(sel).tolist())
+    rng_cache = {}
+
+    def getter(name, e):  # host-generated bf16 weights of the sampled experts (N(0, 0.02))
+        key = (name, e)
+        if key not in rng_cache:
+            rng = np.random.default_rng([w.seed, ("w1", "w3", "w2").index(name), e])
+            shape = (w.I, w.H) if name != "w2" else (w.H, w.I)
+            rng_cache[key] = W.f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32) * np.float32(0.02))
+        return rng_cache[key]
+
+    tables = host_expert_tables(w, experts, getter)
+    rng = np.random.default_rng([w.seed, 9])
+    shared = [W.f32_to_bf16_bits(rng.standard_normal(s, dtype=np.float32) * np.float32(0.02))
+              for s in ((w.I, w.H), (w.I, w.H), (w.H, w.I))]
+    run_oracle_steps(w, x, w_r, b, tokens, tables, shared, args.warmup)
+    times = run_oracle_steps(w, x, w_r, b, tokens, tables, shared, args.steps)
+    total = sum(times)
+    value = len(tokens) * args.steps / total
+    sample = ("route+permute+forward of %d of the %d tokens per step (double-precision C oracle, "
+              "OpenMP), %d distinct experts" % (len(tokens), w.T, len(experts)))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": workload_config(w, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(os.environ["OMP_NUM_THREADS"]),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, args):
+    return {"workload": w.name, "tokens": w.T, "hidden": w.H, "expert_intermediate": w.I,
+            "routed_experts": w.E, "top_k": w.K, "shared_experts": int(w.has_shared),
+            "routed_scale": w.scale, "skewed_routing": w.skew, "global_batch": w.T * args.gpus,
+            "parallelism": "replicas x%d" % args.gpus,
+            "l2": "inputs larger than L2 (packed expert weights %.1f GB)" % (
+                (w.E + 1) * 3 * w.H * w.I * 2 / 1e9)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="glm5_prefill", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-tokens", type=int, default=0)
+    ap.add_argument("--cpu-tokens", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    from sigmoid_routed_mixture_b200 import moe
+
+    w = W.WORKLOADS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    # each replica draws its own token batch; weights are the workload's
+    x, w_r, b = W.router_inputs(w)
+    if rank > 0:
+        rng = np.random.default_rng([w.seed, rank])
+        x = W.f32_to_bf16_bits(rng.standard_normal(x.shape, dtype=np.float32))
+        if w.skew:
+            x[:, 0] = W.f32_to_bf16_bits(np.ones((w.T,), dtype=np.float32))
+    weights = W.expert_weights(w, dev)
+    cfg = moe.Config.of(w)
+    blk = moe.MoeBlock(cfg, torch.from_numpy(w_r).to(dev), torch.from_numpy(b).to(dev), **weights)
+    del weights["w1"], weights["w3"], weights["w2"]
+    torch.cuda.empty_cache()
+    x_dev = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        moe.route(cfg, x_dev, blk.w_router, blk.bias, out=(blk.idx, blk.gate, blk.margin))
+        if ev is not None:
+            ev[1].record(stream)
+        moe.permute(cfg, blk.idx, blk.ws, out=(blk.counts, blk.offsets, blk.sorted))
+        if ev is not None:
+            ev[2].record(stream)
+        moe.expert_up(cfg, blk.weights, x_dev, blk.offsets, blk.sorted, blk.ws)
+        if ev is not None:
+            ev[3].record(stream)
+        moe.expert_down(cfg, blk.weights, blk.gate, blk.offsets, blk.sorted, blk.ws)
+        if ev is not None:
+            ev[4].record(stream)
+        moe.combine(cfg, blk.ws, blk.y)
+        if ev is not None:
+            ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if moe.device_error(blk.ws) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(torch.cuda.current_device())
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    e_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dist is not None:
+        dist.barrier()
+    total_ms = e_start.elapsed_time(e_end)
+    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)]
+                         for i in range(args.steps)])
+    t_max = total_ms
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+    value = w.T * world * args.steps / (t_max / 1e3)
+
+    # ---- end to end: pinned host x in, result out, every step
+    x_host = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory()
+    x_in = torch.empty_like(x_dev)
+
+    def e2e_step():
+        x_in.copy_(x_host, non_blocking=True)
+        blk(x_in)
+        y_host.copy_(blk.y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    z = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    z.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(z)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = w.T * world * args.e2e_steps / (e2e_ms / 1e3)
+    if moe.device_error(blk.ws) != 0:
+        raise RuntimeError("device error during the timed steps")
+
+    # ---- algorithmic work and the roofline of the dominant kernel
+    counts = blk.counts.cpu().numpy()
+    touched = int((counts[: w.E] > 0).sum()) + int(w.has_shared)
+    rows = cfg.rows
+    H, I = w.H, w.I
+    f_router = 2.0 * w.T * H * w.E
+    f_up = 2.0 * rows * H * 2 * I
+    f_down = 2.0 * rows * I * H
+    b_up = touched * 2 * I * H * 2 + w.T * H * 2
+    b_down = touched * H * I * 2 + w.T * H * 2
+    pk = peaks()
+    mean_stage = stage_ms.mean(axis=0)
+    names = ["route", "permute", "expert_up", "expert_down", "combine"]
+    dom = int(np.argmax(mean_stage))
+    ridge = pk["tflops"] * 1e12 / (pk["hbm"] * 1e9)
+    work = {"expert_up": (f_up, b_up), "expert_down": (f_down, b_down),
+            "route": (f_router, w.T * H * 2 + w.E * H * 4 + w.T * w.K * 8),
+            "permute": (0.0, w.T * w.K * 4 * 3 + rows * 4),
+            "combine": (0.0, rows * H * 2 + w.T * H * 2)}
+    f, by = work[names[dom]]
+    dur_s = mean_stage[dom] / 1e3
+    if f > 0 and f / by > ridge:
+        roof = {"kernel": names[dom], "bound": "tensor", "achieved": f / dur_s / 1e12,
+                "peak": pk["tflops"], "unit": "TFLOP/s", "peak_kind": "burst bf16 (cuBLAS), " + pk["source"]}
+    else:
+        roof = {"kernel": names[dom], "bound": "hbm", "achieved": by / dur_s / 1e9, "peak": pk["hbm"],
+                "unit": "GB/s", "peak_kind": "copy bandwidth, " + pk["source"]}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["algorithmic_per_launch"] = f if roof["bound"] == "tensor" else by
+    f_alg = f_router + f_up + f_down
+    b_alg = touched * 3 * H * I * 2 + w.E * H * 4 + w.E * 4 + 2 * w.T * H * 2
+    step_s = t_max / 1e3 / args.steps
+    t_roof = max(f_alg / (pk["tflops"] * 1e12), b_alg / (pk["hbm"] * 1e9))
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init weights of the GLM-5 MoE block shapes)",
+        "config": workload_config(w, argparse.Namespace(gpus=world)),
+        "roofline": roof,
+        "block_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof / step_s,
+                           "f_alg_tflop": f_alg / 1e12, "b_alg_gb": b_alg / 1e9},
+        "stage_ms": {n: float(v) for n, v in zip(names, mean_stage)},
+        "routing": {"touched_groups": touched, "zero_count_experts": int((counts[: w.E] == 0).sum()),
+                    "max_count": int(counts[: w.E].max()), "min_count": int(counts[: w.E].min()),
+                    "near_ties": int((blk.margin <= 1e-4).sum().item())},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(w.T * H * 2),
+                "d2h_bytes_per_step": int(w.T * H * 2), "steps": args.e2e_steps},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+
+    # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N = 1 only
+    if world == 1 and not args.no_cpu_baseline:
+        os.environ.setdefault("OMP_NUM_THREADS", str(cores()))
+        from oracle import oracle as O
+
+        O.build()
+        idx = blk.idx.cpu().numpy()
+        n = args.cpu_tokens or max(8, min(2 * cores(), w.T))
+        tokens = oracle_sample_tokens(w, idx, n)
+        experts = set(np.unique(idx[tokens]).tolist())
+        w13, w2p = blk.weights
+
+        def getter(name, e):
+            if name == "w1":
+                rows_ = [w13[(e * 2 * I + j * 256): (e * 2 * I + j * 256 + 128)] for j in range(2 * I // 256)]
+                return W.torch_bf16_to_bits(torch.cat(rows_))
+            if name == "w3":
+                rows_ = [w13[(e * 2 * I + j * 256 + 128): (e * 2 * I + (j + 1) * 256)] for j in range(2 * I // 256)]
+                return W.torch_bf16_to_bits(torch.cat(rows_))
+            return W.torch_bf16_to_bits(w2p[e * H:(e + 1) * H])
+
+        tables = host_expert_tables(w, experts, getter)
+        shared = [getter("w1", w.E), getter("w3", w.E), getter("w2", w.E)]
+        times = run_oracle_steps(w, x, w_r, b, tokens, tables, shared, 1)
+        line["cpu_baseline"] = {
+            "value": len(tokens) / times[0], "unit": UNIT, "cores": int(os.environ["OMP_NUM_THREADS"]),
+            "kind": "oracle",
+            "sample": "route+permute+forward of %d of the %d tokens (double-precision C oracle, OpenMP), "
+                      "%.1f s" % (len(tokens), w.T, times[0])}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,171 @@
+/*
+ * srm_moe.h -- C ABI of the sigmoid-routed mixture-of-experts FFN for NVIDIA
+ * B200 (sm_100a).  Library: libsrm_moe.so.
+ *
+ * The layer (GLM-4.7-Flash / GLM-5 decoder blocks) computes, per token row x:
+ *     z = x W_r,  s = sigmoid(z),  selection = top_K(s + b),
+ *     G_i = scale * s_i / sum over the selection of s_j   (un-biased s),
+ *     y = sum over the selection of G_i * W2_i (silu(W1_i x) (.) W3_i x)
+ *         + the shared expert's SwiGLU at weight 1.
+ * Definition: "GLM-5 . MoE transformer block" (open model atlas), section
+ * "All 43 steps", the Mixture-of-experts equations; selection-bias and
+ * renormalisation rules: nnterp encyclopedia pages GLM-4.7-Flash and GLM-5,
+ * section 03, note "The mixture: sigmoid scores, a selection bias,
+ * renormalized weights".
+ *
+ * Conventions for every call:
+ *   - All array arguments are DEVICE pointers unless stated otherwise, owned by
+ *     the caller; the library never allocates, frees or keeps them.
+ *   - Matrices are row-major and stored [out, in] (the module's weight layout,
+ *     "GLM-5 . Vocabulary projection" page: weight held output by input), so the
+ *     reduction dimension is contiguous.
+ *   - bf16 means IEEE bfloat16 bit patterns (2 bytes).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*,
+ *     NULL = legacy default stream) and stream-ordered; nothing synchronises
+ *     except moe_get_device_error.
+ *   - Host-side validation happens before any launch and returns a status;
+ *     on a non-OK status nothing was launched.  Problems only the device can
+ *     see (a corrupt expert id, a pipeline wait that ran out) are recorded in
+ *     the workspace's error word and read by moe_get_device_error; outputs of
+ *     such a call are unspecified.  No kernel traps or asserts.
+ *   - Supported shapes: 1 <= K <= E <= 256, K <= 16, H % 256 == 0,
+ *     I % 128 == 0, T >= 0 (T == 0 is a no-op), T * (K + 1) < 2^31.
+ *     Pointers that feed the tensor-memory-access engine (x, packed weights,
+ *     workspace) must be 16-byte aligned; every pointer must be 4-byte aligned.
+ */
+#ifndef SRM_MOE_H
+#define SRM_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_ARG = 1,          /* NULL pointer where one is required, negative size, K > E */
+    MOE_ERR_UNSUPPORTED = 2,  /* shape outside the supported set listed above */
+    MOE_ERR_ALIGN = 3,        /* pointer misaligned (see above) */
+    MOE_ERR_WORKSPACE = 4,    /* ws_bytes < moe_workspace_size(cfg) */
+    MOE_ERR_BAD_INDEX = 5,    /* device: an expert id outside [0, E) in topk_idx */
+    MOE_ERR_TIMEOUT = 6,      /* device: a pipeline wait exceeded its time limit */
+    MOE_ERR_CUDA = 7          /* a CUDA runtime or driver call failed */
+} moe_status_t;
+
+/* Shape and constants of one MoE block.
+ *   T  tokens in this call, H hidden size, I expert intermediate size (the
+ *   shared expert has the same width), E routed experts, K experts per token,
+ *   routed_scale = routed_scaling_factor (2.5 on GLM-5, 1.8 on GLM-4.7-Flash;
+ *   nnterp Config sections), has_shared = 1 to add the always-on shared
+ *   expert (n_shared_experts = 1), 0 to leave it out. */
+typedef struct {
+    int64_t T;
+    int32_t H, I, E, K;
+    float routed_scale;
+    int32_t has_shared;
+} moe_cfg_t;
+
+/* Expert weights after moe_pack_weights (device, bf16):
+ *   w13: [(E+1) * 2I][H]  per group g (g = E is the shared expert), rows in
+ *        blocks of 256: block j holds rows 128j..128j+127 of W1_g (gate
+ *        projection) followed by rows 128j..128j+127 of W3_g (up projection);
+ *        the gate-then-up order is the fused gate_up_proj order of the nnterp
+ *        GLM-4 page (section 03, "The MLP is GLM's fused one").
+ *   w2:  [(E+1) * H][I]  W2_g (down projection) for g = 0..E, shared last. */
+typedef struct {
+    const void *w13;
+    const void *w2;
+} moe_weights_t;
+
+/* Bytes of device workspace moe_permute and moe_forward need for `cfg`
+ * (one buffer serves both).  Returns 0 for an invalid cfg. */
+size_t moe_workspace_size(const moe_cfg_t *cfg);
+
+/* Pack per-expert weights into the moe_weights_t layout.
+ *   w1, w3: bf16 [E][I][H];  w2: bf16 [E][H][I];
+ *   ws1, ws3: bf16 [I][H];  ws2: bf16 [H][I] (shared expert; ignored and may
+ *   be NULL when has_shared == 0, in which case group E is zero-filled);
+ *   w13_out: bf16 [(E+1)*2I][H];  w2_out: bf16 [(E+1)*H][I].
+ * Pure data movement (no arithmetic).  cfg->T is not used. */
+moe_status_t moe_pack_weights(const moe_cfg_t *cfg, const void *w1, const void *w3, const void *w2,
+                              const void *ws1, const void *ws3, const void *ws2, void *w13_out,
+                              void *w2_out, void *stream);
+
+/* Router ("Mixture of experts" equations z = x W_r, s = sigmoid(z),
+ * E_sel = top_K(s + b), G = scale * s E_sel / sum s E_sel).
+ *   x:         bf16 [T][H]
+ *   w_router:  fp32 [E][H]   (W_r stored [out, in])
+ *   bias:      fp32 [E]      (e_score_correction_bias; used only to choose)
+ *   topk_idx:  int32 [T][K]  out: selected experts, slot order = descending
+ *              s + b, equal keys in ascending expert index
+ *   topk_gate: fp32 [T][K]   out: G per slot (sums to routed_scale)
+ *   margin:    fp32 [T] or NULL; out: (K-th key) - ((K+1)-th key) in the
+ *              same order, +inf when K == E.  z accumulates in fp32. */
+moe_status_t moe_route(const moe_cfg_t *cfg, const void *x, const float *w_router, const float *bias,
+                       int32_t *topk_idx, float *topk_gate, float *margin, void *stream);
+
+/* Expert-sorted permutation of the T*K assignments (deterministic).
+ *   topk_idx: int32 [T][K] (as written by moe_route, or by the caller)
+ *   counts:   int32 [E+1]  out: rows per group; counts[E] = T if has_shared
+ *   offsets:  int32 [E+2]  out: exclusive prefix sum of counts
+ *   sorted:   int32 [T*K + T*has_shared] out: sorted[offsets[g] + r] = row id
+ *             of the r-th row of group g in ascending token order; a routed
+ *             row id is t*K + slot, a shared row id is T*K + t.
+ *   ws, ws_bytes: workspace of at least moe_workspace_size(cfg) bytes.
+ * An id outside [0, E) is skipped and flagged MOE_ERR_BAD_INDEX on the device. */
+moe_status_t moe_permute(const moe_cfg_t *cfg, const int32_t *topk_idx, int32_t *counts,
+                         int32_t *offsets, int32_t *sorted, void *ws, size_t ws_bytes, void *stream);
+
+/* Expert FFNs and combine:
+ *   y[t] = sum over slots k = 0..K-1 (in order) of topk_gate[t][k] * E_{idx}(x_t)
+ *          + shared(x_t)   (fp32 sums of bf16 per-slot outputs, one final
+ *          rounding to bf16).
+ * Gates are used AS GIVEN (no renormalisation), so a caller may zero or edit
+ * them (expert ablation).  Inputs: x bf16 [T][H]; topk_gate fp32 [T][K];
+ * offsets, sorted from moe_permute.  Output y: bf16 [T][H].
+ * The intermediate activations live in the workspace. */
+moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *weights, const void *x,
+                         const float *topk_gate, const int32_t *offsets, const int32_t *sorted,
+                         void *y, void *ws, size_t ws_bytes, void *stream);
+
+/* The three stages moe_forward runs, in this order, exposed separately so a
+ * caller can time or overlap them.  They communicate through the workspace
+ * (intermediate h and the per-slot outputs), so the same ws, cfg, offsets and
+ * sorted must be used for all three.
+ *
+ * moe_expert_up: for every group g and its rows (expert-sorted, the token row
+ *   x_t gathered per row id), h = silu(x W1_g) (.) (x W3_g)  ("GLM-5 . MoE
+ *   transformer block", Mixture of experts: g = x W1, u = x W3,
+ *   a = g sigmoid(g), h = a (.) u); h is kept in bf16 in the workspace. */
+moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights, const void *x,
+                           const int32_t *offsets, const int32_t *sorted, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/* moe_expert_down: per row, E_g = h W2_g multiplied by that row's gate
+ *   (topk_gate[t][slot]; 1 for the shared expert), written in bf16 to the
+ *   row's (token, slot) position in the workspace ("expert_outputs: each
+ *   routing slot's weighted expert output", nnterp GLM-5 page, The API). */
+moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
+                             const float *topk_gate, const int32_t *offsets, const int32_t *sorted,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/* moe_combine: y[t] = (sum of the K slot outputs of token t, slots in order)
+ *   + the shared expert's output, in fp32, rounded once to bf16 [T][H]
+ *   (Delta_ffn = y_routed + y_shared). */
+moe_status_t moe_combine(const moe_cfg_t *cfg, void *y, void *ws, size_t ws_bytes, void *stream);
+
+/* Read (and clear) the device error word of a workspace.  Synchronises
+ * `stream`.  *device_status receives MOE_OK or the first device-side error
+ * recorded since the last read.  Returns MOE_ERR_CUDA if the copy fails. */
+moe_status_t moe_get_device_error(void *ws, moe_status_t *device_status, void *stream);
+
+/* Static English description of a status code (never NULL). */
+const char *moe_status_string(moe_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SRM_MOE_H */

@@ -1,0 +1,322 @@
+// api.cu -- host side of the C ABI declared in include/srm_moe.h: argument
+// validation, workspace layout, tensor-map (TMA descriptor) encoding and the
+// kernel launches, all asynchronous on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/srm_moe.h"
+#include "kernels.h"
+
+namespace {
+
+using srm::GemmArgs;
+
+constexpr int kMaxDevices = 64;
+
+struct WsLayout {
+  size_t err, scratch, h, ybuf, total;
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int64_t rows_y(const moe_cfg_t &c) { return c.T * c.K + (c.has_shared ? c.T : 0); }
+
+moe_status_t check_cfg(const moe_cfg_t *c) {
+  if (!c) return MOE_ERR_ARG;
+  if (c->T < 0 || c->H <= 0 || c->I <= 0 || c->E <= 0 || c->K <= 0 || c->K > c->E)
+    return MOE_ERR_ARG;
+  if (!isfinite(c->routed_scale)) return MOE_ERR_ARG;
+  if (c->has_shared != 0 && c->has_shared != 1) return MOE_ERR_ARG;
+  if (c->E > 256 || c->K > 16) return MOE_ERR_UNSUPPORTED;
+  if (c->H % 256 != 0 || c->I % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->H > (1 << 20) || c->I > (1 << 20)) return MOE_ERR_UNSUPPORTED;
+  if (c->T * static_cast<int64_t>(c->K + 1) >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(c->E + 1) * 2 * c->I >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(c->E + 1) * c->H >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+WsLayout layout(const moe_cfg_t &c) {
+  WsLayout L;
+  size_t off = 0;
+  L.err = off;
+  off += 256;
+  L.scratch = off;
+  off = align_up(off + sizeof(int32_t) * static_cast<size_t>(c.E) *
+                           static_cast<size_t>(srm::permute_num_chunks(c.T * c.K)),
+                 1024);
+  L.h = off;
+  off = align_up(off + 2ull * static_cast<size_t>(rows_y(c)) * static_cast<size_t>(c.I), 1024);
+  L.ybuf = off;
+  off = align_up(off + 2ull * static_cast<size_t>(rows_y(c)) * static_cast<size_t>(c.H), 1024);
+  L.total = off;
+  return L;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+int num_sms() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 row-major matrix [rows][inner] -> tensor map with a box of
+// box_rows x box_inner elements and 128-byte swizzling.
+bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, uint32_t box_inner,
+               uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_cfg_t *cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return layout(*cfg).total;
+}
+
+const char *moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_ALIGN: return "misaligned pointer";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_BAD_INDEX: return "expert index out of range (device)";
+    case MOE_ERR_TIMEOUT: return "pipeline wait timed out (device)";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+  }
+  return "unknown status";
+}
+
+moe_status_t moe_pack_weights(const moe_cfg_t *cfg, const void *w1, const void *w3, const void *w2,
+                              const void *ws1, const void *ws3, const void *ws2, void *w13_out,
+                              void *w2_out, void *stream) {
+  moe_status_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!w1 || !w3 || !w2 || !w13_out || !w2_out) return MOE_ERR_ARG;
+  if (cfg->has_shared && (!ws1 || !ws3 || !ws2)) return MOE_ERR_ARG;
+  const void *ptrs[] = {w1, w3, w2, w13_out, w2_out};
+  for (const void *p : ptrs)
+    if (!aligned(p, 16)) return MOE_ERR_ALIGN;
+  if (cfg->has_shared && (!aligned(ws1, 16) || !aligned(ws3, 16) || !aligned(ws2, 16)))
+    return MOE_ERR_ALIGN;
+  return cuda_status(srm::launch_pack(
+      static_cast<const uint16_t *>(w1), static_cast<const uint16_t *>(w3),
+      static_cast<const uint16_t *>(w2), static_cast<const uint16_t *>(ws1),
+      static_cast<const uint16_t *>(ws3), static_cast<const uint16_t *>(ws2), cfg->H, cfg->I,
+      cfg->E, cfg->has_shared, static_cast<uint16_t *>(w13_out), static_cast<uint16_t *>(w2_out),
+      num_sms(), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_route(const moe_cfg_t *cfg, const void *x, const float *w_router, const float *bias,
+                       int32_t *topk_idx, float *topk_gate, float *margin, void *stream) {
+  moe_status_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !w_router || !bias || !topk_idx || !topk_gate) return MOE_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(bias, 4) || !aligned(topk_idx, 4) ||
+      !aligned(topk_gate, 4) || (margin && !aligned(margin, 4)))
+    return MOE_ERR_ALIGN;
+  return cuda_status(srm::launch_route(static_cast<const uint16_t *>(x), w_router, bias,
+                                       static_cast<int>(cfg->T), cfg->H, cfg->E, cfg->K,
+                                       cfg->routed_scale, topk_idx, topk_gate, margin,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_permute(const moe_cfg_t *cfg, const int32_t *topk_idx, int32_t *counts,
+                         int32_t *offsets, int32_t *sorted, void *ws, size_t ws_bytes, void *stream) {
+  moe_status_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !offsets || !ws) return MOE_ERR_ARG;
+  if (cfg->T > 0 && (!topk_idx || !sorted)) return MOE_ERR_ARG;
+  if (!aligned(ws, 256) || !aligned(counts, 4) || !aligned(offsets, 4) ||
+      (topk_idx && !aligned(topk_idx, 4)) || (sorted && !aligned(sorted, 4)))
+    return MOE_ERR_ALIGN;
+  const WsLayout L = layout(*cfg);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  if (cudaMemsetAsync(wsb + L.err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cfg->T == 0) {
+    if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * (cfg->E + 1), s) != cudaSuccess ||
+        cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (cfg->E + 2), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  return cuda_status(srm::launch_permute(
+      topk_idx, static_cast<int>(cfg->T), cfg->E, cfg->K, cfg->has_shared, counts, offsets, sorted,
+      reinterpret_cast<int32_t *>(wsb + L.scratch), reinterpret_cast<int *>(wsb + L.err), s));
+}
+
+namespace {
+
+// Validation shared by the three expert stages; fills the workspace layout.
+moe_status_t check_stage(const moe_cfg_t *cfg, const void *ws, size_t ws_bytes, WsLayout *L) {
+  moe_status_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!ws) return MOE_ERR_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGN;
+  *L = layout(*cfg);
+  if (ws_bytes < L->total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+GemmArgs gemm_args(const moe_cfg_t &c, const int32_t *offsets, const int32_t *sorted,
+                   const float *gate, uint8_t *wsb, const WsLayout &L) {
+  GemmArgs p;
+  p.offsets = offsets;
+  p.sorted = sorted;
+  p.gate = gate;
+  p.err = reinterpret_cast<int *>(wsb + L.err);
+  p.T = static_cast<int>(c.T);
+  p.K = c.K;
+  p.tk = static_cast<int>(c.T * c.K);
+  p.n_rows_y = static_cast<int>(rows_y(c));
+  p.groups = c.E + c.has_shared;
+  return p;
+}
+
+}  // namespace
+
+moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights, const void *x,
+                           const int32_t *offsets, const int32_t *sorted, void *ws, size_t ws_bytes,
+                           void *stream) {
+  WsLayout L;
+  moe_status_t st = check_stage(cfg, ws, ws_bytes, &L);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!weights || !weights->w13 || !x || !offsets || !sorted) return MOE_ERR_ARG;
+  if (!aligned(weights->w13, 16) || !aligned(x, 16) || !aligned(offsets, 4) || !aligned(sorted, 4))
+    return MOE_ERR_ALIGN;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  const int H = cfg->H, I = cfg->I, E = cfg->E;
+  CUtensorMap tm_x, tm_w13;
+  if (!make_tmap(&tm_x, x, H, static_cast<uint64_t>(cfg->T), 64, 1) ||
+      !make_tmap(&tm_w13, weights->w13, H, static_cast<uint64_t>(E + 1) * 2 * I, 64, 256))
+    return MOE_ERR_CUDA;
+  GemmArgs p = gemm_args(*cfg, offsets, sorted, nullptr, wsb, L);
+  p.out = wsb + L.h;
+  p.n_total = 2 * I;
+  p.k_total = H;
+  p.out_ld = I;
+  return cuda_status(srm::launch_grouped_gemm(srm::kUp, tm_x, tm_w13, p, num_sms(),
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
+                             const float *topk_gate, const int32_t *offsets, const int32_t *sorted,
+                             void *ws, size_t ws_bytes, void *stream) {
+  WsLayout L;
+  moe_status_t st = check_stage(cfg, ws, ws_bytes, &L);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!weights || !weights->w2 || !topk_gate || !offsets || !sorted) return MOE_ERR_ARG;
+  if (!aligned(weights->w2, 16) || !aligned(topk_gate, 4) || !aligned(offsets, 4) ||
+      !aligned(sorted, 4))
+    return MOE_ERR_ALIGN;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  const int H = cfg->H, I = cfg->I, E = cfg->E;
+  CUtensorMap tm_h, tm_w2;
+  if (!make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(rows_y(*cfg)), 64, 128) ||
+      !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(E + 1) * H, 64, 256))
+    return MOE_ERR_CUDA;
+  GemmArgs p = gemm_args(*cfg, offsets, sorted, topk_gate, wsb, L);
+  p.out = wsb + L.ybuf;
+  p.n_total = H;
+  p.k_total = I;
+  p.out_ld = H;
+  return cuda_status(srm::launch_grouped_gemm(srm::kDown, tm_h, tm_w2, p, num_sms(),
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_combine(const moe_cfg_t *cfg, void *y, void *ws, size_t ws_bytes, void *stream) {
+  WsLayout L;
+  moe_status_t st = check_stage(cfg, ws, ws_bytes, &L);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!y) return MOE_ERR_ARG;
+  if (!aligned(y, 16)) return MOE_ERR_ALIGN;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  return cuda_status(srm::launch_combine(reinterpret_cast<const uint16_t *>(wsb + L.ybuf),
+                                         static_cast<uint16_t *>(y), static_cast<int>(cfg->T),
+                                         cfg->H, cfg->K, cfg->has_shared, num_sms(),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *weights, const void *x,
+                         const float *topk_gate, const int32_t *offsets, const int32_t *sorted,
+                         void *y, void *ws, size_t ws_bytes, void *stream) {
+  moe_status_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!weights || !weights->w13 || !weights->w2 || !x || !topk_gate || !offsets || !sorted || !y ||
+      !ws)
+    return MOE_ERR_ARG;
+  st = moe_expert_up(cfg, weights, x, offsets, sorted, ws, ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  st = moe_expert_down(cfg, weights, topk_gate, offsets, sorted, ws, ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  return moe_combine(cfg, y, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_get_device_error(void *ws, moe_status_t *device_status, void *stream) {
+  if (!ws || !device_status) return MOE_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (v != 0) {
+    if (cudaMemsetAsync(ws, 0, sizeof v, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  *device_status = static_cast<moe_status_t>(v);
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,53 @@
+// kernels.h -- internal launch interface between the C-ABI host layer
+// (api.cu) and the CUDA kernels of libsrm_moe.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace srm {
+
+constexpr int kUp = 0;    // W1|W3 contraction + SwiGLU epilogue
+constexpr int kDown = 1;  // W2 contraction + gate epilogue
+
+struct GemmArgs {
+  const int32_t *offsets;  // [groups + 1] first expert-sorted row of each group
+  const int32_t *sorted;   // expert-sorted row ids (t*K + slot, or T*K + t for the shared expert)
+  const float *gate;       // [T*K] routing gates (kDown)
+  void *out;               // kUp: h bf16 [rows][I];  kDown: Y bf16 [n_rows_y][H]
+  int *err;                // device error word
+  int T;
+  int K;
+  int tk;                  // T * K
+  int n_rows_y;            // T*K + T*has_shared: valid row ids are [0, n_rows_y)
+  int groups;              // E + has_shared
+  int n_total;             // output columns per group (2I for kUp, H for kDown)
+  int k_total;             // reduction length (H for kUp, I for kDown)
+  int out_ld;              // elements per output row (I for kUp, H for kDown)
+};
+
+size_t grouped_gemm_smem_bytes();
+cudaError_t launch_grouped_gemm(int mode, const CUtensorMap &ta, const CUtensorMap &tb,
+                                const GemmArgs &p, int grid, cudaStream_t stream);
+
+cudaError_t launch_route(const uint16_t *x, const float *w_r, const float *bias, int T, int H, int E,
+                         int K, float scale, int32_t *idx, float *gate, float *margin,
+                         cudaStream_t stream);
+
+// chunk scratch: int32 [E * nchunks]
+int permute_num_chunks(int64_t n_assign);
+cudaError_t launch_permute(const int32_t *idx, int T, int E, int K, int has_shared, int32_t *counts,
+                           int32_t *offsets, int32_t *sorted, int32_t *chunk_scratch, int *err,
+                           cudaStream_t stream);
+
+cudaError_t launch_combine(const uint16_t *Y, uint16_t *y, int T, int H, int K, int has_shared,
+                           int num_sms, cudaStream_t stream);
+
+cudaError_t launch_pack(const uint16_t *w1, const uint16_t *w3, const uint16_t *w2,
+                        const uint16_t *ws1, const uint16_t *ws3, const uint16_t *ws2, int H, int I,
+                        int E, int has_shared, uint16_t *w13_out, uint16_t *w2_out, int num_sms,
+                        cudaStream_t stream);
+
+}  // namespace srm

@@ -1,0 +1,73 @@
+// pack.cu -- one-time re-layout of the expert weights for the grouped GEMMs
+// (data movement only).
+//   w13_out [(E+1)*2I][H]: group g, row block j (256 rows) = W1_g rows
+//       128j..128j+127 then W3_g rows 128j..128j+127, so one 256-column
+//       output tile of the up projection holds matching gate and up columns;
+//       the gate-then-up order is the fused gate_up_proj order of the nnterp
+//       GLM-4 page (section 03, "The MLP is GLM's fused one").
+//   w2_out [(E+1)*H][I]: W2_g for g < E, the shared expert's W2 as group E.
+// A missing shared expert (has_shared == 0) leaves group E zero.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace srm {
+
+__global__ void __launch_bounds__(256)
+    pack_w13_kernel(const uint16_t *__restrict__ w1, const uint16_t *__restrict__ w3,
+                    const uint16_t *__restrict__ ws1, const uint16_t *__restrict__ ws3, int H, int I,
+                    int E, int has_shared, uint16_t *__restrict__ out) {
+  const int vecs = H / 8;
+  const int64_t rows = static_cast<int64_t>(E + 1) * 2 * I;
+  const int64_t total = rows * vecs;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / vecs;
+    const int64_t col = (i - r * vecs) * 8;
+    const int64_t g = r / (2 * I);
+    const int64_t within = r - g * 2 * I;
+    const int64_t j = within / 256, k = within % 256;
+    const int64_t src_row = j * 128 + (k & 127);
+    const bool up = k >= 128;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (g < E) {
+      const uint16_t *src = (up ? w3 : w1) + (g * I + src_row) * H + col;
+      v = *reinterpret_cast<const uint4 *>(src);
+    } else if (has_shared) {
+      const uint16_t *src = (up ? ws3 : ws1) + src_row * H + col;
+      v = *reinterpret_cast<const uint4 *>(src);
+    }
+    *reinterpret_cast<uint4 *>(out + r * H + col) = v;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    pack_w2_kernel(const uint16_t *__restrict__ w2, const uint16_t *__restrict__ ws2, int H, int I,
+                   int E, int has_shared, uint16_t *__restrict__ out) {
+  const int vecs = I / 8;
+  const int64_t rows = static_cast<int64_t>(E + 1) * H;
+  const int64_t total = rows * vecs;
+  const int64_t routed_rows = static_cast<int64_t>(E) * H;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / vecs;
+    const int64_t col = (i - r * vecs) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < routed_rows)
+      v = *reinterpret_cast<const uint4 *>(w2 + r * I + col);
+    else if (has_shared)
+      v = *reinterpret_cast<const uint4 *>(ws2 + (r - routed_rows) * I + col);
+    *reinterpret_cast<uint4 *>(out + r * I + col) = v;
+  }
+}
+
+cudaError_t launch_pack(const uint16_t *w1, const uint16_t *w3, const uint16_t *w2,
+                        const uint16_t *ws1, const uint16_t *ws3, const uint16_t *ws2, int H, int I,
+                        int E, int has_shared, uint16_t *w13_out, uint16_t *w2_out, int num_sms,
+                        cudaStream_t stream) {
+  const int grid = num_sms * 8;
+  pack_w13_kernel<<<grid, 256, 0, stream>>>(w1, w3, ws1, ws3, H, I, E, has_shared, w13_out);
+  pack_w2_kernel<<<grid, 256, 0, stream>>>(w2, ws2, H, I, E, has_shared, w2_out);
+  return cudaGetLastError();
+}
+
+}  // namespace srm

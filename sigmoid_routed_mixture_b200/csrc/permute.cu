@@ -1,0 +1,145 @@
+// permute.cu -- deterministic expert-sorted permutation of the T*K routing
+// assignments (histogram -> exclusive scan -> stable scatter).
+//
+// The pages route every token to K experts (expert_indices [batch, seq,
+// top_k], nnterp GLM-5 page, The API table) and sum the experts' weighted
+// outputs; grouping the assignments by expert is how the grouped GEMMs find
+// their rows.  Result (identical to a sequential counting sort):
+//   counts[g]  rows of group g (g == E: the shared expert, T rows)
+//   offsets    exclusive prefix sum of counts, E + 2 entries
+//   sorted     row ids of each group in ascending assignment order
+//              (routed row id t*K + slot; shared row id T*K + t).
+// No step depends on the order in which atomics land: the per-chunk
+// histograms only count, and the scatter ranks entries with warp matches and
+// per-warp counts in a fixed order.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace srm {
+
+namespace pm {
+constexpr int CHUNK = 1024;  // assignments per chunk
+constexpr int THREADS = 256;
+constexpr int WARPS = THREADS / 32;
+constexpr int MAX_E = 256;
+}  // namespace pm
+
+int permute_num_chunks(int64_t n_assign) {
+  return static_cast<int>((n_assign + pm::CHUNK - 1) / pm::CHUNK);
+}
+
+// 1) chunk histograms: scratch[e * nchunks + c] = entries of chunk c equal to e
+__global__ void __launch_bounds__(pm::THREADS)
+    permute_hist_kernel(const int32_t *__restrict__ idx, int n, int E, int nchunks,
+                        int32_t *__restrict__ scratch, int *err) {
+  __shared__ int hist[pm::MAX_E];
+  const int c = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += pm::THREADS) hist[e] = 0;
+  __syncthreads();
+  const int end = min(n, (c + 1) * pm::CHUNK);
+  for (int i = c * pm::CHUNK + threadIdx.x; i < end; i += pm::THREADS) {
+    const int e = idx[i];
+    if (e < 0 || e >= E)
+      record_error(err, MOE_ERR_BAD_INDEX);
+    else
+      atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += pm::THREADS) scratch[e * nchunks + c] = hist[e];
+}
+
+// 2) one CTA: per-expert running sums over the chunks (turning the scratch
+// into each chunk's first destination), counts, and the group offsets.
+__global__ void __launch_bounds__(pm::THREADS)
+    permute_scan_kernel(int32_t *__restrict__ scratch, int E, int nchunks, int T, int has_shared,
+                        int32_t *__restrict__ counts, int32_t *__restrict__ offsets) {
+  __shared__ int tot[pm::MAX_E];
+  __shared__ int scan[pm::MAX_E];
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < E) {
+    for (int c = 0; c < nchunks; ++c) {
+      const int v = scratch[e * nchunks + c];
+      scratch[e * nchunks + c] = run;
+      run += v;
+    }
+  }
+  tot[e] = e < E ? run : 0;
+  scan[e] = tot[e];
+  __syncthreads();
+  for (int d = 1; d < pm::MAX_E; d <<= 1) {  // inclusive Hillis-Steele scan
+    const int v = e >= d ? scan[e - d] : 0;
+    __syncthreads();
+    scan[e] += v;
+    __syncthreads();
+  }
+  const int excl = scan[e] - tot[e];
+  if (e < E) {
+    counts[e] = tot[e];
+    offsets[e] = excl;
+    for (int c = 0; c < nchunks; ++c) scratch[e * nchunks + c] += excl;
+  }
+  if (e == 0) {
+    const int routed = scan[pm::MAX_E - 1];
+    counts[E] = has_shared ? T : 0;
+    offsets[E] = routed;
+    offsets[E + 1] = routed + (has_shared ? T : 0);
+  }
+}
+
+// 3) stable scatter of each chunk, entries in ascending order.
+__global__ void __launch_bounds__(pm::THREADS)
+    permute_scatter_kernel(const int32_t *__restrict__ idx, int n, int E, int nchunks,
+                           const int32_t *__restrict__ scratch, int T, int has_shared,
+                           const int32_t *__restrict__ offsets, int32_t *__restrict__ sorted) {
+  __shared__ int cursor[pm::MAX_E];
+  __shared__ int wcnt[pm::WARPS][pm::MAX_E];
+  const int c = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < E; e += pm::THREADS) cursor[e] = scratch[e * nchunks + c];
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int r = 0; r < pm::CHUNK / pm::THREADS; ++r) {
+    for (int k = tid; k < pm::WARPS * pm::MAX_E; k += pm::THREADS) (&wcnt[0][0])[k] = 0;
+    __syncthreads();
+    const int i = c * pm::CHUNK + r * pm::THREADS + tid;
+    int e = i < n ? idx[i] : -1;
+    if (e >= E) e = -1;
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(same & lt_mask);
+    if (e >= 0 && rank == 0) wcnt[warp][e] = __popc(same);
+    __syncthreads();
+    if (e >= 0) {
+      int before = 0;
+      for (int w = 0; w < warp; ++w) before += wcnt[w][e];
+      sorted[cursor[e] + before + rank] = i;
+    }
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += pm::THREADS) {
+      int add = 0;
+      for (int w = 0; w < pm::WARPS; ++w) add += wcnt[w][ee];
+      cursor[ee] += add;
+    }
+    __syncthreads();
+  }
+  if (has_shared) {
+    const int base = offsets[E];
+    const int tk = n;
+    for (int t = blockIdx.x * pm::THREADS + tid; t < T; t += gridDim.x * pm::THREADS)
+      sorted[base + t] = tk + t;
+  }
+}
+
+cudaError_t launch_permute(const int32_t *idx, int T, int E, int K, int has_shared, int32_t *counts,
+                           int32_t *offsets, int32_t *sorted, int32_t *scratch, int *err,
+                           cudaStream_t stream) {
+  const int n = T * K;
+  const int nchunks = permute_num_chunks(n);
+  permute_hist_kernel<<<nchunks, pm::THREADS, 0, stream>>>(idx, n, E, nchunks, scratch, err);
+  permute_scan_kernel<<<1, pm::THREADS, 0, stream>>>(scratch, E, nchunks, T, has_shared, counts,
+                                                     offsets);
+  permute_scatter_kernel<<<nchunks, pm::THREADS, 0, stream>>>(idx, n, E, nchunks, scratch, T,
+                                                              has_shared, offsets, sorted);
+  return cudaGetLastError();
+}
+
+}  // namespace srm

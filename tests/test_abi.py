@@ -1,0 +1,103 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/srm_moe.h declares, sizes its workspace and rejects
+invalid arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sigmoid_routed_mixture_b200 import build as B
+from sigmoid_routed_mixture_b200 import moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return moe.lib()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(L):
+    declared = declared_functions()
+    assert {"moe_route", "moe_permute", "moe_forward"} <= declared
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(moe.SYMBOLS) <= declared
+
+
+def test_status_strings(L):
+    for code in range(8):
+        s = L.moe_status_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert L.moe_status_string(0) == b"ok"
+
+
+def cfg(**kw):
+    base = dict(T=64, H=256, I=128, E=16, K=4, routed_scale=2.5, has_shared=True)
+    base.update(kw)
+    return moe.Config(**base)
+
+
+def test_workspace_size_grows_with_tokens(L):
+    small = moe.workspace_bytes(cfg(T=64))
+    big = moe.workspace_bytes(cfg(T=4096))
+    assert big > small > 0
+    # h [rows, I] and Y [rows, H] in bf16 dominate: rows = T*(K+1)
+    rows = 4096 * 5
+    assert big >= 2 * rows * (128 + 256)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(K=0), 1), (dict(K=17, E=32), 2), (dict(E=300, K=8), 2), (dict(K=20, E=16), 1),
+    (dict(H=200), 2), (dict(I=96), 2), (dict(T=-1), 1), (dict(routed_scale=float("nan")), 1),
+    (dict(T=1 << 29, K=8), 2),
+])
+def test_invalid_configs_rejected(L, bad, code):
+    c = cfg(**bad).c()
+    assert L.moe_workspace_size(ctypes.byref(c)) == 0
+    rc = L.moe_route(ctypes.byref(c), None, None, None, None, None, None, None)
+    assert rc == code
+
+
+def test_null_pointers_rejected_before_launch(L):
+    c = cfg().c()
+    assert L.moe_route(ctypes.byref(c), None, None, None, None, None, None, None) == 1
+    assert L.moe_permute(ctypes.byref(c), None, None, None, None, None, 0, None) == 1
+    assert L.moe_forward(ctypes.byref(c), None, None, None, None, None, None, None, 0, None) == 1
+    assert L.moe_pack_weights(ctypes.byref(c), None, None, None, None, None, None, None, None, None) == 1
+    st = ctypes.c_int(0)
+    assert L.moe_get_device_error(None, ctypes.byref(st), None) == 1
+
+
+def test_misaligned_and_small_workspace_rejected(L):
+    c = cfg().c()
+    fake = ctypes.c_void_p(0x10001)  # never dereferenced: validation fails first
+    aligned = ctypes.c_void_p(0x100000)
+    assert L.moe_route(ctypes.byref(c), fake, aligned, aligned, aligned, aligned, None, None) == 3
+    need = L.moe_workspace_size(ctypes.byref(c))
+    assert L.moe_permute(ctypes.byref(c), aligned, aligned, aligned, aligned, aligned, need - 1, None) == 4
+
+
+def test_zero_tokens_is_a_no_op(L):
+    c = cfg(T=0).c()
+    assert L.moe_route(ctypes.byref(c), None, None, None, None, None, None, None) == 0
+    assert L.moe_forward(ctypes.byref(c), None, None, None, None, None, None, None, 0, None) == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(moe, "_lib", None)
+    with pytest.raises(RuntimeError, match="not found"):
+        moe.lib()

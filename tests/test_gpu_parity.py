@@ -1,0 +1,161 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on
+seeded inputs, at every workload size and on the method's edge cases.
+Tolerances and the near-tie rule are stated in tests/moe_harness.py."""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from sigmoid_routed_mixture_b200 import moe
+from sigmoid_routed_mixture_b200 import workloads as W
+
+import moe_harness as MH
+
+pytestmark = pytest.mark.gpu
+
+
+def free():
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def full_check(w, forward_tokens=None):
+    case = MH.Case(w)
+    res = case.run()
+    assert res["err"] == 0
+    MH.check_route(case, res)
+    MH.check_permute(case, res)
+    tokens = np.arange(w.T) if forward_tokens is None else forward_tokens(res)
+    rel = MH.check_forward(case, res, tokens)
+    return case, res, rel
+
+
+def test_tiny_full_parity():
+    full_check(W.WORKLOADS["tiny"])
+
+
+@pytest.mark.parametrize("T", [1, 3, 127, 129, 300])
+def test_ragged_token_counts(T):
+    full_check(W.WORKLOADS["tiny"].replace(T=T, seed=2000 + T))
+
+
+def test_k_equals_e_dense():
+    w = W.WORKLOADS["tiny"].replace(K=16, seed=2100)
+    case, res, _ = full_check(w)
+    assert all(sorted(r) == list(range(16)) for r in res["idx"].tolist())
+    assert np.all(np.isinf(res["margin"]))
+
+
+def test_without_shared_expert():
+    full_check(W.WORKLOADS["tiny"].replace(has_shared=False, T=200, seed=2200))
+
+
+def test_every_token_on_one_expert():
+    """A large bias on expert 5 sends all 1000 tokens there: one group spans
+    eight 128-row tiles with a ragged last one; other groups stay small."""
+    w = W.WORKLOADS["tiny"].replace(T=1000, seed=2300)
+    x, w_r, b = W.router_inputs(w)
+    b[5] = 100.0
+    case = MH.Case(w, x, w_r, b)
+    res = case.run()
+    assert res["err"] == 0
+    assert res["counts"][5] == 1000
+    MH.check_route(case, res)
+    MH.check_permute(case, res)
+    MH.check_forward(case, res, np.arange(1000))
+
+
+def test_glm47flash_parity():
+    w = W.WORKLOADS["glm47flash"]
+    full_check(w, lambda res: MH.sample_tokens(res, w.T, 192))
+    free()
+
+
+def test_glm47flash_page_scale():
+    """The GLM-4.7-Flash config's own routed_scaling_factor 1.8 (nnterp Config)."""
+    w = W.WORKLOADS["glm47flash"].replace(T=512, scale=1.8, seed=2400)
+    full_check(w, lambda res: MH.sample_tokens(res, w.T, 64))
+    free()
+
+
+def test_glm5_decode_parity():
+    full_check(W.WORKLOADS["glm5_decode"])
+    free()
+
+
+@pytest.mark.parametrize("name", ["glm5_prefill", "glm5_skewed"])
+def test_glm5_full_size_sampled(name):
+    """Full-size launch (the benchmark's configuration); the router is compared
+    on a 2048-token subset, the permutation on all tokens, the output on a
+    seeded token sample that includes ragged group tails."""
+    w = W.WORKLOADS[name]
+    case = MH.Case(w)
+    res = case.run()
+    assert res["err"] == 0
+    sub = np.sort(np.random.default_rng(1).choice(w.T, size=2048, replace=False))
+    near = MH.check_route(case, res, sub)
+    assert near < 0.05 * len(sub)
+    MH.check_permute(case, res)
+    MH.check_forward(case, res, MH.sample_tokens(res, w.T, 10))
+    if w.skew:
+        counts = res["counts"][:w.E]
+        assert (counts == 0).sum() > 0      # empty groups exist
+        assert counts.max() >= w.T // 2     # the top expert takes a large share
+    del case, res
+    free()
+
+
+def test_ablation_uses_gates_as_given():
+    """Zeroing the gates of every slot that chose expert 3 (and only those)
+    changes the output exactly by those slots; zero gates leave the shared
+    expert alone."""
+    w = W.WORKLOADS["tiny"].replace(T=256, seed=2500)
+    case = MH.Case(w)
+    res = case.run()
+    blk = res["block"]
+    idx = res["idx"]
+    assert np.any(idx == 3)
+    for gate_h in (np.where(idx == 3, 0.0, res["gate"]).astype(np.float32),
+                   np.zeros_like(res["gate"])):
+        g_dev = torch.from_numpy(gate_h).cuda()
+        y = moe.forward(case.cfg, blk.weights, case.x_dev, g_dev, blk.offsets, blk.sorted, blk.ws)
+        torch.cuda.synchronize()
+        y_g = MH.bf16_to_f64(y)
+        y_o = case.oracle_forward(np.arange(w.T), idx, gate_h.astype(np.float64))
+        rms = float(np.sqrt(np.mean(y_o ** 2)))
+        assert np.max(np.abs(y_g - y_o)) <= MH.Y_TOL * rms
+
+
+def test_deterministic_and_token_permutation_invariant():
+    w = W.WORKLOADS["tiny"].replace(T=300, seed=2600)
+    case = MH.Case(w)
+    r1 = case.run()
+    r2 = case.run()
+    assert np.array_equal(r1["y"], r2["y"]) and np.array_equal(r1["sorted"], r2["sorted"])
+    perm = np.random.default_rng(0).permutation(w.T)
+    case_p = MH.Case(w, case.x[perm], case.w_r, case.b, weights=case.weights)
+    rp = case_p.run()
+    assert np.array_equal(r1["idx"][perm], rp["idx"])
+    assert np.array_equal(r1["gate"][perm], rp["gate"])
+    assert np.array_equal(r1["y"][perm], rp["y"])
+
+
+def test_zero_tokens():
+    w = W.WORKLOADS["tiny"].replace(T=0)
+    case = MH.Case(w)
+    res = case.run()
+    assert res["y"].shape == (0, w.H)
+    assert np.all(res["counts"] == 0) and np.all(res["offsets"] == 0)
+
+
+def test_out_of_range_expert_id_is_flagged():
+    w = W.WORKLOADS["tiny"]
+    cfg = moe.Config.of(w)
+    idx = torch.randint(0, w.E, (w.T, w.K), dtype=torch.int32, device="cuda")
+    idx[7, 2] = w.E + 3
+    ws = moe.workspace(cfg)
+    moe.permute(cfg, idx, ws)
+    assert moe.device_error(ws) == 5
+    assert moe.device_error(ws) == 0  # read clears it

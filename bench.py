@@ -410,7 +410,7 @@ def main():
             if name == "w3":
                 rows_ = [w13[(e * 2 * I + j * 256 + 128): (e * 2 * I + (j + 1) * 256)] for j in range(2 * I // 256)]
                 return W.torch_bf16_to_bits(torch.cat(rows_))
-            return W.torch_bf16_to_bits(w2p[e * H:(e + 1) * H])
+            return W.torch_bf16_to_bits(w2p[e * H:(e + 1) * H].to(torch.bfloat16))
 
         tables = host_expert_tables(w, experts, getter)
         shared = [getter("w1", w.E), getter("w3", w.E), getter("w2", w.E)]

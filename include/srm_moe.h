@@ -73,7 +73,8 @@ typedef struct {
  *        projection) followed by rows 128j..128j+127 of W3_g (up projection);
  *        the gate-then-up order is the fused gate_up_proj order of the nnterp
  *        GLM-4 page (section 03, "The MLP is GLM's fused one").
- *   w2:  [(E+1) * H][I]  W2_g (down projection) for g = 0..E, shared last. */
+ *   w2:  [(E+1) * H][I]  W2_g (down projection) for g = 0..E, shared last,
+ *        stored as IEEE fp16 (see moe_pack_weights). */
 typedef struct {
     const void *w13;
     const void *w2;
@@ -87,8 +88,12 @@ size_t moe_workspace_size(const moe_cfg_t *cfg);
  *   w1, w3: bf16 [E][I][H];  w2: bf16 [E][H][I];
  *   ws1, ws3: bf16 [I][H];  ws2: bf16 [H][I] (shared expert; ignored and may
  *   be NULL when has_shared == 0, in which case group E is zero-filled);
- *   w13_out: bf16 [(E+1)*2I][H];  w2_out: bf16 [(E+1)*H][I].
- * Pure data movement (no arithmetic).  cfg->T is not used. */
+ *   w13_out: bf16 [(E+1)*2I][H];  w2_out: fp16 [(E+1)*H][I].
+ * A re-layout; W2 is also converted from bf16 to fp16, which is exact for
+ * magnitudes in [2^-17, 65504] (smaller ones keep fp16's subnormal spacing of
+ * 2^-24, larger ones saturate).  The down projection multiplies fp16 h by
+ * fp16 W2: fp16 holds h with three more mantissa bits than bf16 at the same
+ * tensor-core rate.  cfg->T is not used. */
 moe_status_t moe_pack_weights(const moe_cfg_t *cfg, const void *w1, const void *w3, const void *w2,
                               const void *ws1, const void *ws3, const void *ws2, void *w13_out,
                               void *w2_out, void *stream);
@@ -120,7 +125,7 @@ moe_status_t moe_permute(const moe_cfg_t *cfg, const int32_t *topk_idx, int32_t 
 
 /* Expert FFNs and combine:
  *   y[t] = sum over slots k = 0..K-1 (in order) of topk_gate[t][k] * E_{idx}(x_t)
- *          + shared(x_t)   (fp32 sums of bf16 per-slot outputs, one final
+ *          + shared(x_t)   (fp32 per-slot outputs summed in fp32, one final
  *          rounding to bf16).
  * Gates are used AS GIVEN (no renormalisation), so a caller may zero or edit
  * them (expert ablation).  Inputs: x bf16 [T][H]; topk_gate fp32 [T][K];
@@ -138,13 +143,14 @@ moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *weights, con
  * moe_expert_up: for every group g and its rows (expert-sorted, the token row
  *   x_t gathered per row id), h = silu(x W1_g) (.) (x W3_g)  ("GLM-5 . MoE
  *   transformer block", Mixture of experts: g = x W1, u = x W3,
- *   a = g sigmoid(g), h = a (.) u); h is kept in bf16 in the workspace. */
+ *   a = g sigmoid(g), h = a (.) u); h is kept in fp16 in the workspace
+ *   (magnitudes above 65504 saturate). */
 moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights, const void *x,
                            const int32_t *offsets, const int32_t *sorted, void *ws, size_t ws_bytes,
                            void *stream);
 
 /* moe_expert_down: per row, E_g = h W2_g multiplied by that row's gate
- *   (topk_gate[t][slot]; 1 for the shared expert), written in bf16 to the
+ *   (topk_gate[t][slot]; 1 for the shared expert), written in fp32 to the
  *   row's (token, slot) position in the workspace ("expert_outputs: each
  *   routing slot's weighted expert output", nnterp GLM-5 page, The API). */
 moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,

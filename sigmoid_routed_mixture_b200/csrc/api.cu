@@ -53,7 +53,7 @@ WsLayout layout(const moe_cfg_t &c) {
   L.h = off;
   off = align_up(off + 2ull * static_cast<size_t>(rows_y(c)) * static_cast<size_t>(c.I), 1024);
   L.ybuf = off;
-  off = align_up(off + 2ull * static_cast<size_t>(rows_y(c)) * static_cast<size_t>(c.H), 1024);
+  off = align_up(off + 4ull * static_cast<size_t>(rows_y(c)) * static_cast<size_t>(c.H), 1024);
   L.total = off;
   return L;
 }
@@ -95,17 +95,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 row-major matrix [rows][inner] -> tensor map with a box of
-// box_rows x box_inner elements and 128-byte swizzling.
+// 16-bit row-major matrix [rows][inner] (bf16 or fp16) -> tensor map with a
+// box of box_rows x box_inner elements and 128-byte swizzling.
 bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, uint32_t box_inner,
-               uint32_t box_rows) {
+               uint32_t box_rows, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {inner * 2};
   const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box,
+  return enc(m, dtype, 2, const_cast<void *>(ptr), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -262,8 +262,10 @@ moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   const int H = cfg->H, I = cfg->I, E = cfg->E;
   CUtensorMap tm_h, tm_w2;
-  if (!make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(rows_y(*cfg)), 64, 128) ||
-      !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(E + 1) * H, 64, 256))
+  if (!make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(rows_y(*cfg)), 64, 128,
+                 CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(E + 1) * H, 64, 256,
+                 CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_CUDA;
   GemmArgs p = gemm_args(*cfg, offsets, sorted, topk_gate, wsb, L);
   p.out = wsb + L.ybuf;
@@ -282,7 +284,7 @@ moe_status_t moe_combine(const moe_cfg_t *cfg, void *y, void *ws, size_t ws_byte
   if (!y) return MOE_ERR_ARG;
   if (!aligned(y, 16)) return MOE_ERR_ALIGN;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
-  return cuda_status(srm::launch_combine(reinterpret_cast<const uint16_t *>(wsb + L.ybuf),
+  return cuda_status(srm::launch_combine(reinterpret_cast<const float *>(wsb + L.ybuf),
                                          static_cast<uint16_t *>(y), static_cast<int>(cfg->T),
                                          cfg->H, cfg->K, cfg->has_shared, num_sms(),
                                          static_cast<cudaStream_t>(stream)));

@@ -7,24 +7,28 @@
 // final addition, and Delta_ffn = y_routed + y_shared ("GLM-5 . MoE
 // transformer block", "All 43 steps").
 //
-// Pure streaming: each thread owns 8 consecutive columns (16 bytes) of one
-// token, loads K+1 16-byte vectors and stores one.
+// Pure streaming: each thread owns 8 consecutive columns of one token, loads
+// K+1 rows of 32 fp32 bytes and stores 16 bytes of bf16.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace srm {
 
-__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    acc[2 * k] += __uint_as_float(w[k] << 16);
-    acc[2 * k + 1] += __uint_as_float(w[k] & 0xFFFF0000u);
-  }
+__device__ __forceinline__ void add8(float (&acc)[8], const float *src) {
+  const float4 a = __ldcs(reinterpret_cast<const float4 *>(src));
+  const float4 b = __ldcs(reinterpret_cast<const float4 *>(src) + 1);
+  acc[0] += a.x;
+  acc[1] += a.y;
+  acc[2] += a.z;
+  acc[3] += a.w;
+  acc[4] += b.x;
+  acc[5] += b.y;
+  acc[6] += b.z;
+  acc[7] += b.w;
 }
 
 __global__ void __launch_bounds__(256)
-    combine_kernel(const uint16_t *__restrict__ Y, uint16_t *__restrict__ y, int T, int H, int K,
+    combine_kernel(const float *__restrict__ Y, uint16_t *__restrict__ y, int T, int H, int K,
                    int has_shared) {
   const int vecs = H / 8;
   const int64_t total = static_cast<int64_t>(T) * vecs;
@@ -34,10 +38,8 @@ __global__ void __launch_bounds__(256)
     const int64_t t = i / vecs;
     const int64_t col = (i - t * vecs) * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k < K; ++k)
-      add_bf16x8(acc, __ldcs(reinterpret_cast<const uint4 *>(Y + (t * K + k) * H + col)));
-    if (has_shared)
-      add_bf16x8(acc, __ldcs(reinterpret_cast<const uint4 *>(Y + (tk + t) * H + col)));
+    for (int k = 0; k < K; ++k) add8(acc, Y + (t * K + k) * H + col);
+    if (has_shared) add8(acc, Y + (tk + t) * H + col);
     uint4 o;
     o.x = pack_bf16x2(acc[0], acc[1]);
     o.y = pack_bf16x2(acc[2], acc[3]);
@@ -47,7 +49,7 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-cudaError_t launch_combine(const uint16_t *Y, uint16_t *y, int T, int H, int K, int has_shared,
+cudaError_t launch_combine(const float *Y, uint16_t *y, int T, int H, int K, int has_shared,
                            int num_sms, cudaStream_t stream) {
   const int64_t total = static_cast<int64_t>(T) * (H / 8);
   int64_t blocks = (total + 255) / 256;

@@ -8,6 +8,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -26,6 +27,15 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t v) {
 // Two floats -> one 32-bit word of two bf16 (round to nearest even), low half first.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&p);
+}
+
+// Two floats -> one 32-bit word of two fp16 (round to nearest even), low half
+// first; magnitudes beyond the largest finite fp16 saturate to +-65504.
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
+  lo = fminf(fmaxf(lo, -65504.f), 65504.f);
+  hi = fminf(fmaxf(hi, -65504.f), 65504.f);
+  __half2 p = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&p);
 }
 
@@ -146,12 +156,12 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_byte_addr) {
   return d;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulator,
-// both operands K-major, shape M x N.
-//   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format
-//   (1 = bf16), 15/16 A/B major (0 = K), 17-22 N >> 3, 24-28 M >> 4.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+// Instruction descriptor of kind::f16 with an fp32 accumulator, both operands
+// K-major, shape M x N; A and B share one type: bf16 (ab_bf16 = 1) or fp16 (0).
+//   bits 4-5 D format (1 = f32), 7-9 A format, 10-12 B format (0 = f16,
+//   1 = bf16), 15/16 A/B major (0 = K), 17-22 N >> 3, 24-28 M >> 4.
+__host__ __device__ constexpr uint32_t umma_idesc_f32acc(int M, int N, uint32_t ab_bf16) {
+  return (1u << 4) | (ab_bf16 << 7) | (ab_bf16 << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 

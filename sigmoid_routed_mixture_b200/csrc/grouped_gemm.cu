@@ -12,10 +12,15 @@
 //   kUp   : for every group g (routed experts 0..E-1, shared expert E) and its
 //           rows (expert-sorted), [g | u] = x_rows . W13_g^T with the rows of x
 //           gathered by TMA (tile::gather4) straight from the token matrix;
-//           epilogue h = silu(g) * u -> bf16 h[row][I].
-//   kDown : Y[a] = G[a] * (h_rows . W2_g^T), rows of h contiguous, epilogue
+//           epilogue h = silu(g) * u -> fp16 h[row][I] (three more mantissa
+//           bits than bf16 at the same tensor-core rate; |h| saturates at
+//           65504).
+//   kDown : Y[a] = G[a] * (h_rows . W2_g^T) in fp16 x fp16 (W2 packed as
+//           fp16, an exact conversion of bf16 weights in fp16's normal
+//           range), rows of h contiguous, epilogue
 //           multiplies by the routing gate (1 for the shared expert) and
-//           scatters bf16 rows to their (token, slot) position a.
+//           scatters fp32 rows to their (token, slot) position a (fp32 so that
+//           the only roundings after the tensor cores are h and the final y).
 //
 // Tiling: one work tile = 128 rows x 256 output columns, K loop in steps of
 // 64 (one 128-byte swizzle atom), 4-stage TMA ring, two 128x256 fp32
@@ -46,7 +51,6 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
 constexpr int MAX_GROUPS = 257;
-constexpr uint32_t IDESC = umma_idesc_bf16_f32(BM, BN);
 
 struct Smem {
   uint64_t full[STAGES];
@@ -108,6 +112,8 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
   const int groups = p.groups;
   const int n_tiles = p.n_total / BN;
   const int kblocks = p.k_total / BK;
+  // up: bf16 x times bf16 W13; down: fp16 h times fp16 W2
+  constexpr uint32_t IDESC = umma_idesc_f32acc(BM, BN, kMode == kUp ? 1u : 0u);
 
   // ---- prologue: barriers, tensor memory, per-group tile starts
   if (threadIdx.x == 0) {
@@ -285,7 +291,7 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
             for (int j = 0; j < 16; ++j) {
               const float g0 = __uint_as_float(gr[2 * j]), g1 = __uint_as_float(gr[2 * j + 1]);
               const float u0 = __uint_as_float(ur[2 * j]), u1 = __uint_as_float(ur[2 * j + 1]);
-              packed[j] = pack_bf16x2(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1);
+              packed[j] = pack_f16x2_sat(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1);
             }
             uint4 *dst = reinterpret_cast<uint4 *>(hrow + ch * 32);
 #pragma unroll
@@ -296,22 +302,18 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
         }
       } else {
         const float gv = (a < p.tk) ? p.gate[valid ? a : 0] : 1.0f;
-        uint16_t *yrow = reinterpret_cast<uint16_t *>(p.out) + static_cast<size_t>(a) * p.out_ld + c.n0;
+        float *yrow = reinterpret_cast<float *>(p.out) + static_cast<size_t>(a) * p.out_ld + c.n0;
 #pragma unroll 1
         for (int ch = 0; ch < BN / 32; ++ch) {
           uint32_t r[32];
           tmem_ld32(taddr + ch * 32, r);
           tmem_ld_wait();
           if (valid) {
-            uint32_t packed[16];
+            float4 *dst = reinterpret_cast<float4 *>(yrow + ch * 32);
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              packed[j] = pack_bf16x2(gv * __uint_as_float(r[2 * j]), gv * __uint_as_float(r[2 * j + 1]));
-            uint4 *dst = reinterpret_cast<uint4 *>(yrow + ch * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
-                                  packed[4 * v + 3]);
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(gv * __uint_as_float(r[4 * v]), gv * __uint_as_float(r[4 * v + 1]),
+                                   gv * __uint_as_float(r[4 * v + 2]), gv * __uint_as_float(r[4 * v + 3]));
           }
         }
       }

@@ -1,11 +1,12 @@
-// pack.cu -- one-time re-layout of the expert weights for the grouped GEMMs
-// (data movement only).
+// pack.cu -- one-time re-layout of the expert weights for the grouped GEMMs.
 //   w13_out [(E+1)*2I][H]: group g, row block j (256 rows) = W1_g rows
 //       128j..128j+127 then W3_g rows 128j..128j+127, so one 256-column
 //       output tile of the up projection holds matching gate and up columns;
 //       the gate-then-up order is the fused gate_up_proj order of the nnterp
 //       GLM-4 page (section 03, "The MLP is GLM's fused one").
-//   w2_out [(E+1)*H][I]: W2_g for g < E, the shared expert's W2 as group E.
+//   w2_out [(E+1)*H][I]: W2_g for g < E, the shared expert's W2 as group E,
+//       converted from bf16 to fp16 (the down projection multiplies fp16 h by
+//       fp16 W2; the conversion is exact for |w| in [2^-17, 65504]).
 // A missing shared expert (has_shared == 0) leaves group E zero.
 #include "common.cuh"
 #include "kernels.h"
@@ -56,7 +57,13 @@ __global__ void __launch_bounds__(256)
       v = *reinterpret_cast<const uint4 *>(w2 + r * I + col);
     else if (has_shared)
       v = *reinterpret_cast<const uint4 *>(ws2 + (r - routed_rows) * I + col);
-    *reinterpret_cast<uint4 *>(out + r * I + col) = v;
+    // bf16 -> fp16: exact for |w| in [2^-17, 65504]; smaller magnitudes keep
+    // fp16's subnormal spacing 2^-24, larger ones saturate
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      w[k] = pack_f16x2_sat(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u));
+    *reinterpret_cast<uint4 *>(out + r * I + col) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 

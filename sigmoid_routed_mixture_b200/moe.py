@@ -176,7 +176,7 @@ def workspace(cfg: Config, device=None) -> torch.Tensor:
 
 
 def pack_weights(cfg: Config, w1, w3, w2, ws1=None, ws3=None, ws2=None, stream=None):
-    """Returns (w13 [(E+1)*2I, H], w2p [(E+1)*H, I]) bf16 in the kernels' layout."""
+    """Returns (w13 bf16 [(E+1)*2I, H], w2p fp16 [(E+1)*H, I]) in the kernels' layout."""
     E, I, H = cfg.E, cfg.I, cfg.H
     bf = torch.bfloat16
     _req(w1, bf, (E, I, H), "w1")
@@ -187,7 +187,7 @@ def pack_weights(cfg: Config, w1, w3, w2, ws1=None, ws3=None, ws2=None, stream=N
         _req(ws3, bf, (I, H), "ws3")
         _req(ws2, bf, (H, I), "ws2")
     w13 = torch.empty(((E + 1) * 2 * I, H), dtype=bf, device=w1.device)
-    w2p = torch.empty(((E + 1) * H, I), dtype=bf, device=w1.device)
+    w2p = torch.empty(((E + 1) * H, I), dtype=torch.float16, device=w1.device)
     _check(lib().moe_pack_weights(ctypes.byref(cfg.c()), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(ws1),
                                   _ptr(ws3), _ptr(ws2), _ptr(w13), _ptr(w2p), _stream(stream)),
            "moe_pack_weights")
@@ -234,7 +234,7 @@ def forward(cfg: Config, weights, x, topk_gate, offsets, sorted_, ws, y=None, st
     _req(offsets, torch.int32, (cfg.E + 2,), "offsets")
     _req(sorted_, torch.int32, (cfg.rows,), "sorted")
     _req(w13, torch.bfloat16, ((cfg.E + 1) * 2 * cfg.I, cfg.H), "w13")
-    _req(w2p, torch.bfloat16, ((cfg.E + 1) * cfg.H, cfg.I), "w2")
+    _req(w2p, torch.float16, ((cfg.E + 1) * cfg.H, cfg.I), "w2")
     if y is None:
         y = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=x.device)
     W = _Weights(w13.data_ptr(), w2p.data_ptr())
@@ -247,7 +247,7 @@ def forward(cfg: Config, weights, x, topk_gate, offsets, sorted_, ws, y=None, st
 def _weights_struct(cfg, weights):
     w13, w2p = weights
     _req(w13, torch.bfloat16, ((cfg.E + 1) * 2 * cfg.I, cfg.H), "w13")
-    _req(w2p, torch.bfloat16, ((cfg.E + 1) * cfg.H, cfg.I), "w2")
+    _req(w2p, torch.float16, ((cfg.E + 1) * cfg.H, cfg.I), "w2")
     return _Weights(w13.data_ptr(), w2p.data_ptr())
 
 

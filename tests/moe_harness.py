@@ -9,8 +9,12 @@ Acceptance rules (the layer's own tolerance, written here once):
   * permutation: counts / offsets / sorted bit-identical to the oracle's
     counting sort of the GPU's own indices;
   * gates: |G_gpu - G_oracle| <= GATE_TOL per expert on tokens with equal sets;
-  * output: max |y_gpu - y_oracle| <= Y_TOL * RMS(y_oracle), where the oracle
-    uses the GPU's selection with gates recomputed in double.
+  * output: |y_gpu - y_oracle| <= Y_TOL * RMS(y_oracle) + half_ulp_bf16(y_oracle)
+    element by element, where the oracle is exact (double) and uses the GPU's
+    selection with gates recomputed in double.  The half-ulp term is the
+    representation error of the bf16 result itself, which no implementation
+    avoids: for |y| in [16, 32) it is 0.0625, more than 2e-2 x RMS whenever
+    RMS < 3.1.  The raw max |y_gpu - y_oracle| / RMS is returned for reporting.
 """
 from __future__ import annotations
 
@@ -28,6 +32,21 @@ Y_TOL = 2e-2
 
 def to_dev_bf16(bits: np.ndarray, device="cuda") -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def half_ulp_bf16(v: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers at |v| (8 significant bits)."""
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(a, np.finfo(np.float64).tiny)))
+    return np.where(a > 0, np.exp2(e - 8), 0.0)
+
+
+def within_tolerance(y_g, y_o):
+    """(ok, raw max|dy|/rms, worst excess) under the output rule above."""
+    rms = float(np.sqrt(np.mean(y_o ** 2)))
+    err = np.abs(y_g - y_o)
+    bound = Y_TOL * rms + half_ulp_bf16(y_o)
+    return bool(np.all(err <= bound)), float(err.max() / rms) if rms > 0 else 0.0, float((err - bound).max())
 
 
 def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
@@ -141,11 +160,10 @@ def check_forward(case: Case, res, tokens):
         gate = O.gates_for(z, idx, case.w.scale)
     y_o = case.oracle_forward(tokens, idx, gate)
     y_g = res["y"][tokens]
-    rms = float(np.sqrt(np.mean(y_o ** 2)))
-    err = float(np.max(np.abs(y_g - y_o)))
-    assert rms > 0
-    assert err <= Y_TOL * rms, "max|dy| %g > %g * rms %g" % (err, Y_TOL, rms)
-    return err / rms
+    assert np.sqrt(np.mean(y_o ** 2)) > 0
+    ok, rel, excess = within_tolerance(y_g, y_o)
+    assert ok, "output outside 2e-2*rms + half-ulp: max|dy|/rms %g, worst excess %g" % (rel, excess)
+    return rel
 
 
 def sample_tokens(res, T, n_random, seed=0):

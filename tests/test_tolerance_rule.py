@@ -9,6 +9,7 @@ from sigmoid_routed_mixture_b200 import workloads as W
 def test_half_ulp_bounds_bf16_rounding_tightly():
     rng = np.random.default_rng(0)
     v = np.concatenate([rng.standard_normal(200000) * s for s in (0.01, 1.0, 3.0, 40.0)])
+    v = v.astype(np.float32).astype(np.float64)  # one rounding only: fp32 -> bf16
     r = W.bf16_bits_to_f32(W.f32_to_bf16_bits(v.astype(np.float32))).astype(np.float64)
     hu = MH.half_ulp_bf16(v)
     err = np.abs(r - v)

@@ -55,6 +55,9 @@ WORKLOADS = {
                              seed=1003),
     "glm5_skewed": Workload("glm5_skewed", T=8192, H=6144, I=2048, E=256, K=8, scale=2.5,
                             seed=1004, skew=True),
+    # GLM-5 expert shapes with 32 experts: 2.5 GB of weights, small enough for
+    # multi-pass profiler captures, still far larger than the 126 MB L2
+    "glm5_e32": Workload("glm5_e32", T=8192, H=6144, I=2048, E=32, K=8, scale=2.5, seed=1005),
 }
 
 

@@ -35,7 +35,7 @@ from sigmoid_routed_mixture_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-block tokens/s (GLM-5 shape, bf16, 1 B200)"
 UNIT = "tokens/s"
-KERNELS_PER_STEP = 7  # route 1 + permute 3 + up 1 + down 1 + combine 1
+KERNELS_PER_STEP = 9  # route 1 + permute 3 + row gather 2 + up 1 + down 1 + combine 1
 
 
 def peaks():

@@ -140,8 +140,9 @@ moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *weights, con
  * (intermediate h and the per-slot outputs), so the same ws, cfg, offsets and
  * sorted must be used for all three.
  *
- * moe_expert_up: for every group g and its rows (expert-sorted, the token row
- *   x_t gathered per row id), h = silu(x W1_g) (.) (x W3_g)  ("GLM-5 . MoE
+ * moe_expert_up: for every group g and its rows (expert-sorted: the token rows
+ *   are first copied into that order in the workspace, each row of x read
+ *   once), h = silu(x W1_g) (.) (x W3_g)  ("GLM-5 . MoE
  *   transformer block", Mixture of experts: g = x W1, u = x W3,
  *   a = g sigmoid(g), h = a (.) u); h is kept in fp16 in the workspace
  *   (magnitudes above 65504 saturate). */

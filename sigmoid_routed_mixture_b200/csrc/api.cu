@@ -19,7 +19,7 @@ using srm::GemmArgs;
 constexpr int kMaxDevices = 64;
 
 struct WsLayout {
-  size_t err, scratch, h, ybuf, total;
+  size_t err, scratch, pos, xs, h, ybuf, total;
 };
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -50,6 +50,10 @@ WsLayout layout(const moe_cfg_t &c) {
   off = align_up(off + sizeof(int32_t) * static_cast<size_t>(c.E) *
                            static_cast<size_t>(srm::permute_num_chunks(c.T * c.K)),
                  1024);
+  L.pos = off;
+  off = align_up(off + sizeof(int32_t) * static_cast<size_t>(rows_y(c)), 1024);
+  L.xs = off;
+  off = align_up(off + 2ull * static_cast<size_t>(rows_y(c)) * static_cast<size_t>(c.H), 1024);
   L.h = off;
   off = align_up(off + 2ull * static_cast<size_t>(rows_y(c)) * static_cast<size_t>(c.I), 1024);
   L.ybuf = off;
@@ -235,17 +239,22 @@ moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights, c
     return MOE_ERR_ALIGN;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   const int H = cfg->H, I = cfg->I, E = cfg->E;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tm_x, tm_w13;
-  if (!make_tmap(&tm_x, x, H, static_cast<uint64_t>(cfg->T), 64, 1) ||
+  if (!make_tmap(&tm_x, wsb + L.xs, H, static_cast<uint64_t>(rows_y(*cfg)), 64, 128) ||
       !make_tmap(&tm_w13, weights->w13, H, static_cast<uint64_t>(E + 1) * 2 * I, 64, 256))
+    return MOE_ERR_CUDA;
+  if (srm::launch_gather_rows(static_cast<const uint16_t *>(x), sorted, static_cast<int>(cfg->T), H,
+                              cfg->K, cfg->has_shared, reinterpret_cast<int32_t *>(wsb + L.pos),
+                              reinterpret_cast<uint16_t *>(wsb + L.xs),
+                              reinterpret_cast<int *>(wsb + L.err), num_sms(), s) != cudaSuccess)
     return MOE_ERR_CUDA;
   GemmArgs p = gemm_args(*cfg, offsets, sorted, nullptr, wsb, L);
   p.out = wsb + L.h;
   p.n_total = 2 * I;
   p.k_total = H;
   p.out_ld = I;
-  return cuda_status(srm::launch_grouped_gemm(srm::kUp, tm_x, tm_w13, p, num_sms(),
-                                              static_cast<cudaStream_t>(stream)));
+  return cuda_status(srm::launch_grouped_gemm(srm::kUp, tm_x, tm_w13, p, num_sms(), s));
 }
 
 moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,

@@ -127,18 +127,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, uint64_
       : "memory");
 }
 
-// Row gather: four rows r0..r3 (each one box row of the map) at inner
-// coordinate c0, written back to back into shared memory.
-__device__ __forceinline__ void tma_gather4(void *dst, const void *tmap, uint64_t *bar, int32_t c0,
-                                            int32_t r0, int32_t r1, int32_t r2, int32_t r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_addr(bar)), "r"(c0), "r"(r0), "r"(r1),
-      "r"(r2), "r"(r3)
-      : "memory");
-}
-
 // ----------------------------------------------------------------- tcgen05
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA

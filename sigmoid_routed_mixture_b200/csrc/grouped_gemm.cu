@@ -10,9 +10,8 @@
 // output", nnterp GLM-5 page, The API table).
 //
 //   kUp   : for every group g (routed experts 0..E-1, shared expert E) and its
-//           rows (expert-sorted), [g | u] = x_rows . W13_g^T with the rows of x
-//           gathered by TMA (tile::gather4) straight from the token matrix;
-//           epilogue h = silu(g) * u -> fp16 h[row][I] (three more mantissa
+//           rows, [g | u] = xs_rows . W13_g^T where xs holds the token rows in
+//           expert-sorted order (gather.cu); epilogue h = silu(g) * u -> fp16 h[row][I] (three more mantissa
 //           bits than bf16 at the same tensor-core rate; |h| saturates at
 //           65504).
 //   kDown : Y[a] = G[a] * (h_rows . W2_g^T) in fp16 x fp16 (W2 packed as
@@ -26,7 +25,7 @@
 // 64 (one 128-byte swizzle atom), 4-stage TMA ring, two 128x256 fp32
 // accumulators in tensor memory (512 columns) so the epilogue of one tile
 // overlaps the main loop of the next.  Warp roles (6 warps):
-//   warp 0: TMA producer (all 32 lanes issue gathers in kUp)
+//   warp 0: TMA producer (one lane issues the A and B tile loads)
 //   warp 1: tensor-memory allocation + single-thread MMA issue
 //   warps 2-5: epilogue (tensor memory -> registers -> global)
 // Work tiles are (group, 128-row block, 256-column block), column block
@@ -177,24 +176,6 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
     uint32_t stage = 0, phase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       const TileCoord c = decode_tile(s, groups, n_tiles, tile);
-      int tok[4] = {0, 0, 0, 0};
-      if (kMode == kUp) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int r = lane * 4 + j;
-          const int a = p.sorted[c.row_base + (r < c.rows ? r : 0)];
-          int t;
-          if (a >= 0 && a < p.tk)
-            t = a / p.K;
-          else
-            t = a - p.tk;
-          if (a < 0 || a >= p.n_rows_y || t < 0 || t >= p.T) {
-            record_error(p.err, MOE_ERR_BAD_INDEX);
-            t = 0;
-          }
-          tok[j] = t;
-        }
-      }
       const int b_row = c.g * p.n_total + c.n0;
       bool ok = true;
       for (int kb = 0; kb < kblocks; ++kb) {
@@ -204,14 +185,10 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
         }
         if (lane == 0) mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
         __syncwarp();
-        uint8_t *a_dst = sA + stage * A_BYTES;
-        if (kMode == kUp) {
-          tma_gather4(a_dst + lane * 4 * (BK * 2), &tmap_a, &s.full[stage], kb * BK, tok[0], tok[1],
-                      tok[2], tok[3]);
-        } else if (lane == 0) {
-          tma_load_2d(a_dst, &tmap_a, &s.full[stage], kb * BK, c.row_base);
+        if (lane == 0) {
+          tma_load_2d(sA + stage * A_BYTES, &tmap_a, &s.full[stage], kb * BK, c.row_base);
+          tma_load_2d(sB + stage * B_BYTES, &tmap_b, &s.full[stage], kb * BK, b_row);
         }
-        if (lane == 0) tma_load_2d(sB + stage * B_BYTES, &tmap_b, &s.full[stage], kb * BK, b_row);
         ++issued;
         if (++stage == STAGES) {
           stage = 0;

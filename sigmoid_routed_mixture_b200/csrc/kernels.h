@@ -42,6 +42,12 @@ cudaError_t launch_permute(const int32_t *idx, int T, int E, int K, int has_shar
                            int32_t *offsets, int32_t *sorted, int32_t *chunk_scratch, int *err,
                            cudaStream_t stream);
 
+// token rows in expert-sorted order: xs[p] = x[token of sorted[p]]; pos is
+// int32 scratch [rows] (row id -> sorted position)
+cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *sorted, int T, int H, int K,
+                               int has_shared, int32_t *pos, uint16_t *xs, int *err, int num_sms,
+                               cudaStream_t stream);
+
 cudaError_t launch_combine(const float *Y, uint16_t *y, int T, int H, int K, int has_shared,
                            int num_sms, cudaStream_t stream);
 

@@ -35,7 +35,7 @@ from sigmoid_routed_mixture_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-block tokens/s (GLM-5 shape, bf16, 1 B200)"
 UNIT = "tokens/s"
-KERNELS_PER_STEP = 9  # route 1 + permute 3 + row gather 2 + up 1 + down 1 + combine 1
+KERNELS_PER_STEP = 11  # route 3 + permute 3 + row gather 2 + up 1 + down 1 + combine 1
 
 
 def peaks():
@@ -258,7 +258,7 @@ def main():
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        moe.route(cfg, x_dev, blk.w_router, blk.bias, out=(blk.idx, blk.gate, blk.margin))
+        moe.route(cfg, x_dev, blk.w_router, blk.bias, blk.ws, out=(blk.idx, blk.gate, blk.margin))
         if ev is not None:
             ev[1].record(stream)
         moe.permute(cfg, blk.idx, blk.ws, out=(blk.counts, blk.offsets, blk.sorted))

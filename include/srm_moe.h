@@ -80,8 +80,8 @@ typedef struct {
     const void *w2;
 } moe_weights_t;
 
-/* Bytes of device workspace moe_permute and moe_forward need for `cfg`
- * (one buffer serves both).  Returns 0 for an invalid cfg. */
+/* Bytes of device workspace moe_route, moe_permute and moe_forward need for
+ * `cfg` (one buffer serves all three).  Returns 0 for an invalid cfg. */
 size_t moe_workspace_size(const moe_cfg_t *cfg);
 
 /* Pack per-expert weights into the moe_weights_t layout.
@@ -107,9 +107,14 @@ moe_status_t moe_pack_weights(const moe_cfg_t *cfg, const void *w1, const void *
  *              s + b, equal keys in ascending expert index
  *   topk_gate: fp32 [T][K]   out: G per slot (sums to routed_scale)
  *   margin:    fp32 [T] or NULL; out: (K-th key) - ((K+1)-th key) in the
- *              same order, +inf when K == E.  z accumulates in fp32. */
+ *              same order, +inf when K == E.
+ *   ws, ws_bytes: workspace of at least moe_workspace_size(cfg) bytes (holds
+ *              the bf16 split of W_r and the partial logits).
+ * z is computed on the tensor cores from an exact three-part bf16 split of
+ * W_r (each product exact, fp32 accumulation): fp32-accurate logits. */
 moe_status_t moe_route(const moe_cfg_t *cfg, const void *x, const float *w_router, const float *bias,
-                       int32_t *topk_idx, float *topk_gate, float *margin, void *stream);
+                       int32_t *topk_idx, float *topk_gate, float *margin, void *ws, size_t ws_bytes,
+                       void *stream);
 
 /* Expert-sorted permutation of the T*K assignments (deterministic).
  *   topk_idx: int32 [T][K] (as written by moe_route, or by the caller)

@@ -19,7 +19,7 @@ using srm::GemmArgs;
 constexpr int kMaxDevices = 64;
 
 struct WsLayout {
-  size_t err, scratch, pos, xs, h, ybuf, total;
+  size_t err, scratch, wsplit, zp, pos, xs, h, ybuf, total;
 };
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -49,6 +49,12 @@ WsLayout layout(const moe_cfg_t &c) {
   L.scratch = off;
   off = align_up(off + sizeof(int32_t) * static_cast<size_t>(c.E) *
                            static_cast<size_t>(srm::permute_num_chunks(c.T * c.K)),
+                 1024);
+  L.wsplit = off;
+  off = align_up(off + 2ull * 3 * static_cast<size_t>(srm::router_e_pad(c.E)) * c.H, 1024);
+  L.zp = off;
+  off = align_up(off + 4ull * static_cast<size_t>(srm::router_splits(static_cast<int>(c.T), c.H)) *
+                           static_cast<size_t>(c.T) * srm::router_e_pad(c.E),
                  1024);
   L.pos = off;
   off = align_up(off + sizeof(int32_t) * static_cast<size_t>(rows_y(c)), 1024);
@@ -158,18 +164,28 @@ moe_status_t moe_pack_weights(const moe_cfg_t *cfg, const void *w1, const void *
 }
 
 moe_status_t moe_route(const moe_cfg_t *cfg, const void *x, const float *w_router, const float *bias,
-                       int32_t *topk_idx, float *topk_gate, float *margin, void *stream) {
+                       int32_t *topk_idx, float *topk_gate, float *margin, void *ws, size_t ws_bytes,
+                       void *stream) {
   moe_status_t st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
-  if (!x || !w_router || !bias || !topk_idx || !topk_gate) return MOE_ERR_ARG;
+  if (!x || !w_router || !bias || !topk_idx || !topk_gate || !ws) return MOE_ERR_ARG;
   if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(bias, 4) || !aligned(topk_idx, 4) ||
-      !aligned(topk_gate, 4) || (margin && !aligned(margin, 4)))
+      !aligned(topk_gate, 4) || (margin && !aligned(margin, 4)) || !aligned(ws, 256))
     return MOE_ERR_ALIGN;
-  return cuda_status(srm::launch_route(static_cast<const uint16_t *>(x), w_router, bias,
-                                       static_cast<int>(cfg->T), cfg->H, cfg->E, cfg->K,
-                                       cfg->routed_scale, topk_idx, topk_gate, margin,
-                                       static_cast<cudaStream_t>(stream)));
+  const WsLayout L = layout(*cfg);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  const int e_pad = srm::router_e_pad(cfg->E);
+  CUtensorMap tm_x, tm_w;
+  if (!make_tmap(&tm_x, x, cfg->H, static_cast<uint64_t>(cfg->T), 64, 128) ||
+      !make_tmap(&tm_w, wsb + L.wsplit, cfg->H, 3ull * e_pad, 64, static_cast<uint32_t>(e_pad)))
+    return MOE_ERR_CUDA;
+  return cuda_status(srm::launch_route(
+      tm_x, tm_w, w_router, bias, static_cast<int>(cfg->T), cfg->H, cfg->E, cfg->K,
+      cfg->routed_scale, reinterpret_cast<uint16_t *>(wsb + L.wsplit),
+      reinterpret_cast<float *>(wsb + L.zp), topk_idx, topk_gate, margin,
+      reinterpret_cast<int *>(wsb + L.err), num_sms(), static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_permute(const moe_cfg_t *cfg, const int32_t *topk_idx, int32_t *counts,

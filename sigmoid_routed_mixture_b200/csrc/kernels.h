@@ -32,9 +32,15 @@ size_t grouped_gemm_smem_bytes();
 cudaError_t launch_grouped_gemm(int mode, const CUtensorMap &ta, const CUtensorMap &tb,
                                 const GemmArgs &p, int grid, cudaStream_t stream);
 
-cudaError_t launch_route(const uint16_t *x, const float *w_r, const float *bias, int T, int H, int E,
-                         int K, float scale, int32_t *idx, float *gate, float *margin,
-                         cudaStream_t stream);
+// router: W_r split into bf16 parts [3][e_pad][H] (wsplit), fp32 partial logits
+// zp [splits][T][e_pad]; tmap_x: x [T][H] box 64 x 128, tmap_w: wsplit [3*e_pad][H]
+// box 64 x e_pad
+int router_e_pad(int E);
+int router_splits(int T, int H);
+cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, const float *w_r,
+                         const float *bias, int T, int H, int E, int K, float scale,
+                         uint16_t *wsplit, float *zp, int32_t *idx, float *gate, float *margin,
+                         int *err, int num_sms, cudaStream_t stream);
 
 // chunk scratch: int32 [E * nchunks]
 int permute_num_chunks(int64_t n_assign);

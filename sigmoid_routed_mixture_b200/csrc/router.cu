@@ -1,5 +1,5 @@
-// router.cu -- fused router: logits, sigmoid scores, biased top-K selection
-// and renormalised, scaled gates in one kernel.
+// router.cu -- the router: logits on the tensor cores, then sigmoid scores,
+// biased top-K selection and renormalised, scaled gates.
 //
 // Definition ("GLM-5 . MoE transformer block", "All 43 steps", Mixture of
 // experts):  z = x W_r;  s = sigmoid(z);  E_sel_i = [i in top_K(s + b)];
@@ -9,12 +9,22 @@
 // scores, a selection bias, renormalized weights").  Ties between equal keys
 // go to the lower expert index; the slots come out in descending key order.
 //
-// One CTA = 64 tokens x all experts (E <= 256).  Stage 1: z for the tile with
-// fp32 FMA (bf16 x widened exactly, fp32 W_r, fp32 accumulation; each thread
-// owns 8 tokens x NE experts).  Stage 2: z goes to shared memory and each warp
-// selects for 8 tokens: every lane holds NE candidate keys and K rounds of a
-// warp arg-max (key descending, index ascending) pick the slots; one more
-// round gives the (K+1)-th key for the selection margin.
+// W_r is fp32 and x is bf16.  W_r is split exactly-to-fp32-precision into
+// three bf16 parts (hi = bf16(W), mid = bf16(W - hi), lo = bf16(W - hi - mid);
+// what is left is below 2^-24 |W|), so z = x.hi + x.mid + x.lo with every
+// product exact and fp32 accumulation: fp32-accurate logits at bf16 tensor-
+// core speed.
+//   1) router_split_kernel: W_r -> [3][E_pad][H] bf16 (E_pad = E rounded up
+//      to 32, padding rows zero), once per call (6 MB read, 9 MB written at
+//      the GLM-5 shape).
+//   2) router_logits_kernel: 128 tokens x E_pad experts per CTA, tcgen05.mma
+//      kind::f16 (bf16) into tensor memory, TMA-fed ring; the H range may be
+//      split over S CTAs (S > 1 when there are few 128-token tiles) and each
+//      CTA writes fp32 partial logits zp[s][t][e].
+//   3) router_select_kernel: one warp per token sums the S partials in order
+//      (deterministic), then s, keys, K rounds of a warp arg-max (key
+//      descending, index ascending), one more round for the margin, gates.
+#include <cuda.h>
 #include <math.h>
 
 #include "common.cuh"
@@ -23,171 +33,327 @@
 namespace srm {
 
 namespace rt {
-constexpr int TT = 64;     // tokens per CTA
-constexpr int HC = 32;     // reduction chunk
-constexpr int THREADS = 256;
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int THREADS = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int MAX_SMEM = 232448;  // 227 KB dynamic shared memory per CTA
 }  // namespace rt
 
-template <int NE>
-__global__ void __launch_bounds__(rt::THREADS)
-    route_kernel(const uint16_t *__restrict__ x, const float *__restrict__ w_r,
-                 const float *__restrict__ bias, int T, int H, int E, int K, float scale,
-                 int32_t *__restrict__ idx, float *__restrict__ gate, float *__restrict__ margin) {
+int router_e_pad(int E) { return (E + 31) / 32 * 32; }
+
+int router_stage_bytes(int e_pad) { return rt::A_BYTES + 3 * e_pad * rt::BK * 2; }
+
+struct RouterSmem;
+int router_stages(int e_pad);
+
+int router_splits(int T, int H) {
+  const int m_tiles = (T + rt::BM - 1) / rt::BM;
+  const int kblocks = H / rt::BK;
+  int s = 148 / (m_tiles > 0 ? m_tiles : 1);
+  const int max_s = kblocks / 2 > 0 ? kblocks / 2 : 1;
+  if (s > max_s) s = max_s;
+  if (s < 1) s = 1;
+  return s;
+}
+
+// ---------------------------------------------------------------- 1) split
+
+__device__ __forceinline__ uint16_t bf16_rn_bits(float v) {
+  __nv_bfloat16 b = __float2bfloat16_rn(v);
+  return *reinterpret_cast<uint16_t *>(&b);
+}
+
+__global__ void __launch_bounds__(256)
+    router_split_kernel(const float *__restrict__ w_r, int E, int e_pad, int H,
+                        uint16_t *__restrict__ wsplit) {
+  const int64_t n = static_cast<int64_t>(e_pad) * H;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t e = i / H;
+    const float w = e < E ? w_r[i] : 0.f;
+    const uint16_t hi = bf16_rn_bits(w);
+    const float r1 = w - bf16_bits_to_float(hi);
+    const uint16_t mid = bf16_rn_bits(r1);
+    const float r2 = r1 - bf16_bits_to_float(mid);
+    const uint16_t lo = bf16_rn_bits(r2);
+    wsplit[i] = hi;
+    wsplit[n + i] = mid;
+    wsplit[2 * n + i] = lo;
+  }
+}
+
+// ---------------------------------------------------------------- 2) logits
+
+struct RouterSmem {
+  uint64_t full[4];
+  uint64_t empty[4];
+  uint64_t done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int mma_consumed;
+};
+
+__global__ void __launch_bounds__(rt::THREADS, 1)
+    router_logits_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                         const __grid_constant__ CUtensorMap tmap_w, int T, int e_pad,
+                         int kb_per_split, int kblocks, int stages, uint32_t tmem_cols,
+                         float *__restrict__ zp, int *err) {
   using namespace rt;
-  constexpr int EP = NE * 32;  // padded expert count
-  extern __shared__ float smem_f[];
-  float *xs = smem_f;                  // [TT][HC + 1]
-  float *ws = smem_f + TT * (HC + 1);  // [EP][HC + 1]
-  float *zs = smem_f;                  // [TT][EP + 1], reused after stage 1
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  uint8_t *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const int stage_bytes = A_BYTES + 3 * e_pad * BK * 2;
+  RouterSmem &s = *reinterpret_cast<RouterSmem *>(base + stages * stage_bytes);
 
-  const int tid = threadIdx.x;
-  const int tx = tid & 31;
-  const int ty = tid >> 5;
-  const int t0 = blockIdx.x * TT;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * BM;
+  const int split = blockIdx.y;
+  const int kb0 = split * kb_per_split;
+  const int kb1 = min(kblocks, kb0 + kb_per_split);
+  const uint32_t part_bytes = static_cast<uint32_t>(e_pad) * BK * 2;
 
-  float acc[8][NE];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < NE; ++j) acc[i][j] = 0.f;
-
-  for (int h0 = 0; h0 < H; h0 += HC) {
-    {  // x tile: 64 tokens x 32 features, 8 bf16 per thread
-      const int tt = tid >> 2, part = (tid & 3) * 8;
-      const int t = t0 + tt;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t < T) v = *reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t) * H + h0 + part);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        xs[tt * (HC + 1) + part + 2 * k] = __uint_as_float(w[k] << 16);
-        xs[tt * (HC + 1) + part + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-      }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
     }
-    // W_r tile: EP experts x 32 features
-    for (int i = tid; i < EP * (HC / 4); i += THREADS) {
-      const int e = i / (HC / 4), part = (i % (HC / 4)) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < E) v = *reinterpret_cast<const float4 *>(w_r + static_cast<size_t>(e) * H + h0 + part);
-      ws[e * (HC + 1) + part + 0] = v.x;
-      ws[e * (HC + 1) + part + 1] = v.y;
-      ws[e * (HC + 1) + part + 2] = v.z;
-      ws[e * (HC + 1) + part + 3] = v.w;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int h = 0; h < HC; ++h) {
-      float a[8], b[NE];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) a[i] = xs[(ty * 8 + i) * (HC + 1) + h];
-#pragma unroll
-      for (int j = 0; j < NE; ++j) b[j] = ws[(tx + 32 * j) * (HC + 1) + h];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < NE; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
+    mbar_init(&s.done, 1);
+    mbar_init(&s.drain, 1);
+    s.abort_flag = 0;
+    s.mma_consumed = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmap_x);
+    tma_prefetch_desc(&tmap_w);
   }
-
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < NE; ++j) zs[(ty * 8 + i) * (EP + 1) + tx + 32 * j] = acc[i][j];
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  volatile int *abort_flag = &s.abort_flag;
+  int issued = 0;
 
-  // ---- selection: warp `ty` handles tokens ty*8 .. ty*8+7 of the tile
-  float bj[NE];
-#pragma unroll
-  for (int j = 0; j < NE; ++j) {
-    const int e = tx + 32 * j;
-    bj[j] = e < E ? bias[e] : 0.f;
-  }
-  for (int i = 0; i < 8; ++i) {
-    const int tt = ty * 8 + i;
-    const int t = t0 + tt;
-    if (t >= T) break;  // uniform across the warp
-    float key[NE], sv[NE];
-#pragma unroll
-    for (int j = 0; j < NE; ++j) {
-      const int e = tx + 32 * j;
-      const float sj = sigmoidf_(zs[tt * (EP + 1) + e]);
-      sv[j] = sj;
-      key[j] = e < E ? sj + bj[j] : -INFINITY;
+  if (warp == 0) {
+    uint32_t stage = 0, phase = 0;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, err)) break;
+      if (lane == 0) {
+        uint8_t *st = base + stage * stage_bytes;
+        mbar_arrive_expect_tx(&s.full[stage], stage_bytes);
+        tma_load_2d(st, &tmap_x, &s.full[stage], kb * BK, m0);
+        for (int part = 0; part < 3; ++part)
+          tma_load_2d(st + A_BYTES + part * part_bytes, &tmap_w, &s.full[stage], kb * BK,
+                      part * e_pad);
+      }
+      __syncwarp();
+      ++issued;
+      if (++stage == static_cast<uint32_t>(stages)) {
+        stage = 0;
+        phase ^= 1u;
+      }
     }
-    int my_e = 0;
-    float my_s = 0.f, kth_key = 0.f, next_key = -INFINITY;
-    const int rounds = K < E ? K + 1 : K;
-    for (int k = 0; k < rounds; ++k) {
-      float bk = -INFINITY, bs = 0.f;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < NE; ++j) {
-        if (key[j] > bk) {  // j ascending = expert index ascending: strict > keeps the lower
-          bk = key[j];
-          be = tx + 32 * j;
-          bs = sv[j];
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-        if (ok > bk || (ok == bk && oe < be)) {
-          bk = ok;
-          be = oe;
-          bs = os;
-        }
-      }
-      if (k == K) {
-        next_key = bk;
+  } else if (warp == 1) {
+    const uint32_t idesc = umma_idesc_f32acc(BM, e_pad, 1u);
+    uint32_t stage = 0, phase = 0;
+    int consumed = 0;
+    bool ok = true;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(&s.full[stage], phase, abort_flag, err)) {
+        ok = false;
         break;
       }
-      if (tx == k) {
-        my_e = be;
-        my_s = bs;
-      }
-      if (k == K - 1) kth_key = bk;
+      tc_fence_after();
+      ++consumed;
+      if (lane == 0) {
+        const uint32_t a_addr = smem_addr(base + stage * stage_bytes);
 #pragma unroll
-      for (int j = 0; j < NE; ++j)
-        if (be == tx + 32 * j) key[j] = -INFINITY;
+        for (int part = 0; part < 3; ++part) {
+          const uint32_t b_addr = a_addr + A_BYTES + part * part_bytes;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16(tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), idesc,
+                      (kb > kb0 || part > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(&s.empty[stage]);
+      }
+      __syncwarp();
+      if (++stage == static_cast<uint32_t>(stages)) {
+        stage = 0;
+        phase ^= 1u;
+      }
     }
-    float denom = 0.f;
-    for (int k = 0; k < K; ++k) denom += __shfl_sync(0xffffffffu, my_s, k);
-    if (tx < K) {
-      idx[static_cast<size_t>(t) * K + tx] = my_e;
-      gate[static_cast<size_t>(t) * K + tx] = scale * my_s / denom;
+    if (ok && lane == 0) umma_commit(&s.done);
+    if (lane == 0) s.mma_consumed = consumed;
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int t = m0 + row;
+    if (mbar_wait(&s.done, 0, abort_flag, err)) {
+      tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      float *dst = zp + (static_cast<size_t>(split) * T + t) * e_pad;
+      for (int c = 0; c < e_pad / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(taddr + c * 32, r);
+        tmem_ld_wait();
+        if (t < T) {
+          float4 *d4 = reinterpret_cast<float4 *>(dst + c * 32);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            d4[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+        }
+      }
     }
-    if (margin && tx == 0) margin[t] = K < E ? kth_key - next_key : INFINITY;
+  }
+
+  __syncthreads();
+  if (s.abort_flag) {  // error path: let copies and MMAs in flight land first
+    if (warp == 0 && lane == 0) {
+      for (int i = s.mma_consumed; i < issued; ++i) {
+        const uint32_t a = smem_addr(&s.full[i % stages]);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(a, static_cast<uint32_t>((i / stages) & 1)) &&
+               global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+    if (warp == 1 && lane == 0) {
+      umma_commit(&s.drain);
+      const uint32_t a = smem_addr(&s.drain);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(a, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
   }
 }
 
-template <int NE>
-static cudaError_t launch_ne(const uint16_t *x, const float *w_r, const float *bias, int T, int H,
-                             int E, int K, float scale, int32_t *idx, float *gate, float *margin,
-                             cudaStream_t stream) {
-  using namespace rt;
-  constexpr int EP = NE * 32;
-  const size_t stage1 = sizeof(float) * (TT * (HC + 1) + EP * (HC + 1));
-  const size_t stage2 = sizeof(float) * TT * (EP + 1);
-  const size_t smem = stage1 > stage2 ? stage1 : stage2;
-  cudaError_t e = cudaFuncSetAttribute(route_kernel<NE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  const int grid = (T + TT - 1) / TT;
-  route_kernel<NE><<<grid, THREADS, smem, stream>>>(x, w_r, bias, T, H, E, K, scale, idx, gate,
-                                                   margin);
-  return cudaGetLastError();
+int router_stages(int e_pad) {
+  int s = static_cast<int>((rt::MAX_SMEM - 1024 - sizeof(RouterSmem)) / router_stage_bytes(e_pad));
+  return s > 4 ? 4 : s;
 }
 
-cudaError_t launch_route(const uint16_t *x, const float *w_r, const float *bias, int T, int H, int E,
-                         int K, float scale, int32_t *idx, float *gate, float *margin,
-                         cudaStream_t stream) {
-  if (E <= 32) return launch_ne<1>(x, w_r, bias, T, H, E, K, scale, idx, gate, margin, stream);
-  if (E <= 64) return launch_ne<2>(x, w_r, bias, T, H, E, K, scale, idx, gate, margin, stream);
-  if (E <= 128) return launch_ne<4>(x, w_r, bias, T, H, E, K, scale, idx, gate, margin, stream);
-  return launch_ne<8>(x, w_r, bias, T, H, E, K, scale, idx, gate, margin, stream);
+// ---------------------------------------------------------------- 3) select
+
+template <int NE>
+__global__ void __launch_bounds__(256)
+    router_select_kernel(const float *__restrict__ zp, int splits, const float *__restrict__ bias,
+                         int T, int E, int e_pad, int K, float scale, int32_t *__restrict__ idx,
+                         float *__restrict__ gate, float *__restrict__ margin) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;  // whole warp
+  float key[NE], sv[NE];
+#pragma unroll
+  for (int j = 0; j < NE; ++j) {
+    const int e = lane + 32 * j;
+    float z = 0.f;
+    if (e < E)
+      for (int sp = 0; sp < splits; ++sp) z += zp[(static_cast<size_t>(sp) * T + t) * e_pad + e];
+    const float sj = sigmoidf_(z);
+    sv[j] = sj;
+    key[j] = e < E ? sj + bias[e] : -INFINITY;
+  }
+  int my_e = 0;
+  float my_s = 0.f, kth_key = 0.f, next_key = -INFINITY;
+  const int rounds = K < E ? K + 1 : K;
+  for (int k = 0; k < rounds; ++k) {
+    float bk = -INFINITY, bs = 0.f;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NE; ++j) {
+      if (key[j] > bk) {  // j ascending = expert index ascending: strict > keeps the lower
+        bk = key[j];
+        be = lane + 32 * j;
+        bs = sv[j];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+      if (ok > bk || (ok == bk && oe < be)) {
+        bk = ok;
+        be = oe;
+        bs = os;
+      }
+    }
+    if (k == K) {
+      next_key = bk;
+      break;
+    }
+    if (lane == k) {
+      my_e = be;
+      my_s = bs;
+    }
+    if (k == K - 1) kth_key = bk;
+#pragma unroll
+    for (int j = 0; j < NE; ++j)
+      if (be == lane + 32 * j) key[j] = -INFINITY;
+  }
+  float denom = 0.f;
+  for (int k = 0; k < K; ++k) denom += __shfl_sync(0xffffffffu, my_s, k);
+  if (lane < K) {
+    idx[static_cast<size_t>(t) * K + lane] = my_e;
+    gate[static_cast<size_t>(t) * K + lane] = scale * my_s / denom;
+  }
+  if (margin && lane == 0) margin[t] = K < E ? kth_key - next_key : INFINITY;
+}
+
+// ---------------------------------------------------------------- launch
+
+size_t router_logits_smem_bytes(int e_pad) {
+  return 1024 + static_cast<size_t>(router_stages(e_pad)) * router_stage_bytes(e_pad) +
+         sizeof(RouterSmem);
+}
+
+cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, const float *w_r,
+                         const float *bias, int T, int H, int E, int K, float scale,
+                         uint16_t *wsplit, float *zp, int32_t *idx, float *gate, float *margin,
+                         int *err, int num_sms, cudaStream_t stream) {
+  const int e_pad = router_e_pad(E);
+  router_split_kernel<<<num_sms * 4, 256, 0, stream>>>(w_r, E, e_pad, H, wsplit);
+  const int kblocks = H / rt::BK;
+  const int splits = router_splits(T, H);
+  const int kb_per = (kblocks + splits - 1) / splits;
+  const int stages = router_stages(e_pad);
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(e_pad)) cols <<= 1;
+  const size_t smem = router_logits_smem_bytes(e_pad);
+  cudaError_t e = cudaFuncSetAttribute(router_logits_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((T + rt::BM - 1) / rt::BM, (kblocks + kb_per - 1) / kb_per);
+  router_logits_kernel<<<grid, rt::THREADS, smem, stream>>>(tmap_x, tmap_w, T, e_pad, kb_per,
+                                                            kblocks, stages, cols, zp, err);
+  const int used_splits = static_cast<int>(grid.y);
+  const int blocks = (T + 7) / 8;
+  if (E <= 32)
+    router_select_kernel<1><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
+                                                        idx, gate, margin);
+  else if (E <= 64)
+    router_select_kernel<2><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
+                                                        idx, gate, margin);
+  else if (E <= 128)
+    router_select_kernel<4><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
+                                                        idx, gate, margin);
+  else
+    router_select_kernel<8><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
+                                                        idx, gate, margin);
+  return cudaGetLastError();
 }
 
 }  // namespace srm

@@ -7,7 +7,7 @@ fallback of any kind: if the library is missing, every call raises.
     cfg = moe.Config(T, H, I, E, K, routed_scale=2.5)
     w13, w2 = moe.pack_weights(cfg, w1, w3, w2, ws1, ws3, ws2)
     ws = moe.workspace(cfg)
-    idx, gate, margin = moe.route(cfg, x, w_router, bias)
+    idx, gate, margin = moe.route(cfg, x, w_router, bias, ws)
     counts, offsets, sorted_ = moe.permute(cfg, idx, ws)
     y = moe.forward(cfg, (w13, w2), x, gate, offsets, sorted_, ws)
 """
@@ -108,7 +108,7 @@ def lib():
         L.moe_pack_weights.restype = ctypes.c_int
         L.moe_pack_weights.argtypes = [P(_Cfg)] + [vp] * 9
         L.moe_route.restype = ctypes.c_int
-        L.moe_route.argtypes = [P(_Cfg)] + [vp] * 7
+        L.moe_route.argtypes = [P(_Cfg)] + [vp] * 7 + [ctypes.c_size_t, vp]
         L.moe_permute.restype = ctypes.c_int
         L.moe_permute.argtypes = [P(_Cfg), vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.moe_forward.restype = ctypes.c_int
@@ -194,7 +194,7 @@ def pack_weights(cfg: Config, w1, w3, w2, ws1=None, ws3=None, ws2=None, stream=N
     return w13, w2p
 
 
-def route(cfg: Config, x, w_router, bias, want_margin=True, out=None, stream=None):
+def route(cfg: Config, x, w_router, bias, ws, want_margin=True, out=None, stream=None):
     """Router: returns (topk_idx int32 [T,K], topk_gate fp32 [T,K], margin fp32 [T] or None)."""
     T, H, E, K = cfg.T, cfg.H, cfg.E, cfg.K
     _req(x, torch.bfloat16, (T, H), "x")
@@ -207,7 +207,7 @@ def route(cfg: Config, x, w_router, bias, want_margin=True, out=None, stream=Non
     else:
         idx, gate, margin = out
     _check(lib().moe_route(ctypes.byref(cfg.c()), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(idx),
-                           _ptr(gate), _ptr(margin), _stream(stream)), "moe_route")
+                           _ptr(gate), _ptr(margin), _ptr(ws), ws.numel(), _stream(stream)), "moe_route")
     return idx, gate, margin
 
 
@@ -301,7 +301,8 @@ class MoeBlock:
         self.y = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
 
     def __call__(self, x, stream=None):
-        route(self.cfg, x, self.w_router, self.bias, out=(self.idx, self.gate, self.margin), stream=stream)
+        route(self.cfg, x, self.w_router, self.bias, self.ws, out=(self.idx, self.gate, self.margin),
+              stream=stream)
         permute(self.cfg, self.idx, self.ws, out=(self.counts, self.offsets, self.sorted), stream=stream)
         return forward(self.cfg, self.weights, x, self.gate, self.offsets, self.sorted, self.ws, y=self.y,
                        stream=stream)

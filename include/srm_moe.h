@@ -108,13 +108,15 @@ moe_status_t moe_pack_weights(const moe_cfg_t *cfg, const void *w1, const void *
  *   topk_gate: fp32 [T][K]   out: G per slot (sums to routed_scale)
  *   margin:    fp32 [T] or NULL; out: (K-th key) - ((K+1)-th key) in the
  *              same order, +inf when K == E.
+ *   logits:    fp32 [T][E] or NULL; out: z, the router logits before the
+ *              sigmoid and the bias (the pages' router_logits value).
  *   ws, ws_bytes: workspace of at least moe_workspace_size(cfg) bytes (holds
  *              the bf16 split of W_r and the partial logits).
  * z is computed on the tensor cores from an exact three-part bf16 split of
  * W_r (each product exact, fp32 accumulation): fp32-accurate logits. */
 moe_status_t moe_route(const moe_cfg_t *cfg, const void *x, const float *w_router, const float *bias,
-                       int32_t *topk_idx, float *topk_gate, float *margin, void *ws, size_t ws_bytes,
-                       void *stream);
+                       int32_t *topk_idx, float *topk_gate, float *margin, float *logits, void *ws,
+                       size_t ws_bytes, void *stream);
 
 /* Expert-sorted permutation of the T*K assignments (deterministic).
  *   topk_idx: int32 [T][K] (as written by moe_route, or by the caller)

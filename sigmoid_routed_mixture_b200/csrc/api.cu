@@ -164,14 +164,15 @@ moe_status_t moe_pack_weights(const moe_cfg_t *cfg, const void *w1, const void *
 }
 
 moe_status_t moe_route(const moe_cfg_t *cfg, const void *x, const float *w_router, const float *bias,
-                       int32_t *topk_idx, float *topk_gate, float *margin, void *ws, size_t ws_bytes,
-                       void *stream) {
+                       int32_t *topk_idx, float *topk_gate, float *margin, float *logits, void *ws,
+                       size_t ws_bytes, void *stream) {
   moe_status_t st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
   if (!x || !w_router || !bias || !topk_idx || !topk_gate || !ws) return MOE_ERR_ARG;
   if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(bias, 4) || !aligned(topk_idx, 4) ||
-      !aligned(topk_gate, 4) || (margin && !aligned(margin, 4)) || !aligned(ws, 256))
+      !aligned(topk_gate, 4) || (margin && !aligned(margin, 4)) || (logits && !aligned(logits, 4)) ||
+      !aligned(ws, 256))
     return MOE_ERR_ALIGN;
   const WsLayout L = layout(*cfg);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
@@ -184,7 +185,7 @@ moe_status_t moe_route(const moe_cfg_t *cfg, const void *x, const float *w_route
   return cuda_status(srm::launch_route(
       tm_x, tm_w, w_router, bias, static_cast<int>(cfg->T), cfg->H, cfg->E, cfg->K,
       cfg->routed_scale, reinterpret_cast<uint16_t *>(wsb + L.wsplit),
-      reinterpret_cast<float *>(wsb + L.zp), topk_idx, topk_gate, margin,
+      reinterpret_cast<float *>(wsb + L.zp), topk_idx, topk_gate, margin, logits,
       reinterpret_cast<int *>(wsb + L.err), num_sms(), static_cast<cudaStream_t>(stream)));
 }
 

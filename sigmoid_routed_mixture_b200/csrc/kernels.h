@@ -40,7 +40,7 @@ int router_splits(int T, int H);
 cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, const float *w_r,
                          const float *bias, int T, int H, int E, int K, float scale,
                          uint16_t *wsplit, float *zp, int32_t *idx, float *gate, float *margin,
-                         int *err, int num_sms, cudaStream_t stream);
+                         float *logits, int *err, int num_sms, cudaStream_t stream);
 
 // chunk scratch: int32 [E * nchunks]
 int permute_num_chunks(int64_t n_assign);

@@ -15,12 +15,13 @@
 // product exact and fp32 accumulation: fp32-accurate logits at bf16 tensor-
 // core speed.
 //   1) router_split_kernel: W_r -> [3][E_pad][H] bf16 (E_pad = E rounded up
-//      to 32, padding rows zero), once per call (6 MB read, 9 MB written at
+//      to 64, padding rows zero), once per call (6 MB read, 9 MB written at
 //      the GLM-5 shape).
 //   2) router_logits_kernel: 128 tokens x E_pad experts per CTA, tcgen05.mma
-//      kind::f16 (bf16) into tensor memory, TMA-fed ring; the H range may be
-//      split over S CTAs (S > 1 when there are few 128-token tiles) and each
-//      CTA writes fp32 partial logits zp[s][t][e].
+//      kind::f16 (bf16) into tensor memory, TMA-fed ring, short accumulation
+//      chains promoted to fp32 registers (see below); the H range may be split
+//      over S CTAs (S > 1 when there are few 128-token tiles) and each CTA
+//      writes fp32 partial logits zp[s][t][e].
 //   3) router_select_kernel: one warp per token sums the S partials in order
 //      (deterministic), then s, keys, K rounds of a warp arg-max (key
 //      descending, index ascending), one more round for the margin, gates.
@@ -35,12 +36,14 @@ namespace srm {
 namespace rt {
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int THREADS = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;  // warp 0 TMA, warp 1 MMA + TMEM, 8 epilogue warps
+constexpr int CHUNK = 2;                      // k-blocks per tensor-core accumulation chain
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int MAX_SMEM = 232448;  // 227 KB dynamic shared memory per CTA
 }  // namespace rt
 
-int router_e_pad(int E) { return (E + 31) / 32 * 32; }
+int router_e_pad(int E) { return (E + 63) / 64 * 64; }
 
 int router_stage_bytes(int e_pad) { return rt::A_BYTES + 3 * e_pad * rt::BK * 2; }
 
@@ -85,26 +88,37 @@ __global__ void __launch_bounds__(256)
 
 // ---------------------------------------------------------------- 2) logits
 
+// The tensor core's fp32 accumulator loses precision over long chains of
+// MMAs (measured on B200: max |dz| 1.5e-4 after 1152 chained MMAs against
+// 4e-6 for an fp32 blocked sum).  So each chunk of CHUNK k-blocks goes to one
+// of two ping-pong accumulators, starting from zero, and the epilogue warps
+// add every finished chunk into fp32 registers: no accumulation chain is
+// longer than CHUNK * 12 MMAs.
 struct RouterSmem {
   uint64_t full[4];
   uint64_t empty[4];
-  uint64_t done;
+  uint64_t tfull[2];
+  uint64_t tempty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
   int mma_consumed;
 };
 
+// NH = e_pad / 64: each epilogue thread keeps half a row (e_pad / 2 columns).
+template <int NH>
 __global__ void __launch_bounds__(rt::THREADS, 1)
     router_logits_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                         const __grid_constant__ CUtensorMap tmap_w, int T, int e_pad,
-                         int kb_per_split, int kblocks, int stages, uint32_t tmem_cols,
-                         float *__restrict__ zp, int *err) {
+                         const __grid_constant__ CUtensorMap tmap_w, int T, int kb_per_split,
+                         int kblocks, int stages, uint32_t tmem_cols, float *__restrict__ zp,
+                         int *err) {
   using namespace rt;
+  constexpr int e_pad = NH * 64;
+  constexpr int HALF = e_pad / 2;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   uint8_t *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  const int stage_bytes = A_BYTES + 3 * e_pad * BK * 2;
+  constexpr int stage_bytes = A_BYTES + 3 * e_pad * BK * 2;
   RouterSmem &s = *reinterpret_cast<RouterSmem *>(base + stages * stage_bytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -112,14 +126,18 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
   const int split = blockIdx.y;
   const int kb0 = split * kb_per_split;
   const int kb1 = min(kblocks, kb0 + kb_per_split);
-  const uint32_t part_bytes = static_cast<uint32_t>(e_pad) * BK * 2;
+  const int nchunks = (kb1 - kb0 + CHUNK - 1) / CHUNK;
+  constexpr uint32_t part_bytes = static_cast<uint32_t>(e_pad) * BK * 2;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < stages; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
-    mbar_init(&s.done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], EPI_WARPS);
+    }
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
     s.mma_consumed = 0;
@@ -139,6 +157,7 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
   int issued = 0;
 
   if (warp == 0) {
+    // ---------------------------------------------------------- producer
     uint32_t stage = 0, phase = 0;
     for (int kb = kb0; kb < kb1; ++kb) {
       if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, err)) break;
@@ -158,58 +177,85 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
       }
     }
   } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
     const uint32_t idesc = umma_idesc_f32acc(BM, e_pad, 1u);
     uint32_t stage = 0, phase = 0;
     int consumed = 0;
     bool ok = true;
-    for (int kb = kb0; kb < kb1; ++kb) {
-      if (!mbar_wait(&s.full[stage], phase, abort_flag, err)) {
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const uint32_t slot = c & 1;
+      if (!mbar_wait(&s.tempty[slot], ((c >> 1) & 1) ^ 1u, abort_flag, err)) break;
+      tc_fence_after();
+      const uint32_t d = tmem + slot * e_pad;
+      const int ka = kb0 + c * CHUNK, kz = min(kb1, ka + CHUNK);
+      for (int kb = ka; kb < kz; ++kb) {
+        if (!mbar_wait(&s.full[stage], phase, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        ++consumed;
+        if (lane == 0) {
+          const uint32_t a_addr = smem_addr(base + stage * stage_bytes);
+#pragma unroll
+          for (int part = 0; part < 3; ++part) {
+            const uint32_t b_addr = a_addr + A_BYTES + part * part_bytes;
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              umma_bf16(d, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), idesc,
+                        (kb > ka || part > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&s.empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == static_cast<uint32_t>(stages)) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok && lane == 0) umma_commit(&s.tfull[slot]);
+      __syncwarp();
+    }
+    if (lane == 0) s.mma_consumed = consumed;
+  } else {
+    // ---------------------------------------------------------- epilogue
+    // warps 2..9: lane quarter q = warp % 4 (the TMEM lanes this warp may
+    // read), column half hf; each thread owns row q*32 + lane, HALF columns
+    const int q = warp & 3;
+    const int hf = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    const int t = m0 + row;
+    float acc[HALF];
+#pragma unroll
+    for (int j = 0; j < HALF; ++j) acc[j] = 0.f;
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      const uint32_t slot = c & 1;
+      if (!mbar_wait(&s.tfull[slot], (c >> 1) & 1, abort_flag, err)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      ++consumed;
-      if (lane == 0) {
-        const uint32_t a_addr = smem_addr(base + stage * stage_bytes);
+      const uint32_t taddr =
+          tmem + slot * e_pad + hf * HALF + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll
-        for (int part = 0; part < 3; ++part) {
-          const uint32_t b_addr = a_addr + A_BYTES + part * part_bytes;
-#pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_bf16(tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), idesc,
-                      (kb > kb0 || part > 0 || k > 0) ? 1u : 0u);
-        }
-        umma_commit(&s.empty[stage]);
-      }
-      __syncwarp();
-      if (++stage == static_cast<uint32_t>(stages)) {
-        stage = 0;
-        phase ^= 1u;
-      }
-    }
-    if (ok && lane == 0) umma_commit(&s.done);
-    if (lane == 0) s.mma_consumed = consumed;
-    __syncwarp();
-  } else {
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const int t = m0 + row;
-    if (mbar_wait(&s.done, 0, abort_flag, err)) {
-      tc_fence_after();
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      float *dst = zp + (static_cast<size_t>(split) * T + t) * e_pad;
-      for (int c = 0; c < e_pad / 32; ++c) {
+      for (int cc = 0; cc < HALF / 32; ++cc) {
         uint32_t r[32];
-        tmem_ld32(taddr + c * 32, r);
+        tmem_ld32(taddr + cc * 32, r);
         tmem_ld_wait();
-        if (t < T) {
-          float4 *d4 = reinterpret_cast<float4 *>(dst + c * 32);
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            d4[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-        }
+        for (int j = 0; j < 32; ++j) acc[cc * 32 + j] += __uint_as_float(r[j]);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.tempty[slot]);
+    }
+    if (ok && t < T) {
+      float4 *d4 = reinterpret_cast<float4 *>(zp + (static_cast<size_t>(split) * T + t) * e_pad +
+                                              hf * HALF);
+#pragma unroll
+      for (int v = 0; v < HALF / 4; ++v)
+        d4[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
     }
   }
 
@@ -251,7 +297,8 @@ template <int NE>
 __global__ void __launch_bounds__(256)
     router_select_kernel(const float *__restrict__ zp, int splits, const float *__restrict__ bias,
                          int T, int E, int e_pad, int K, float scale, int32_t *__restrict__ idx,
-                         float *__restrict__ gate, float *__restrict__ margin) {
+                         float *__restrict__ gate, float *__restrict__ margin,
+                         float *__restrict__ logits) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;  // whole warp
@@ -260,8 +307,10 @@ __global__ void __launch_bounds__(256)
   for (int j = 0; j < NE; ++j) {
     const int e = lane + 32 * j;
     float z = 0.f;
-    if (e < E)
+    if (e < E) {
       for (int sp = 0; sp < splits; ++sp) z += zp[(static_cast<size_t>(sp) * T + t) * e_pad + e];
+      if (logits) logits[static_cast<size_t>(t) * E + e] = z;
+    }
     const float sj = sigmoidf_(z);
     sv[j] = sj;
     key[j] = e < E ? sj + bias[e] : -INFINITY;
@@ -315,6 +364,19 @@ __global__ void __launch_bounds__(256)
 
 // ---------------------------------------------------------------- launch
 
+template <int NH>
+static cudaError_t launch_logits(dim3 grid, size_t smem, const CUtensorMap &tmap_x,
+                                 const CUtensorMap &tmap_w, int T, int kb_per, int kblocks,
+                                 int stages, uint32_t cols, float *zp, int *err,
+                                 cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<NH>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  router_logits_kernel<NH><<<grid, rt::THREADS, smem, stream>>>(tmap_x, tmap_w, T, kb_per, kblocks,
+                                                                stages, cols, zp, err);
+  return cudaGetLastError();
+}
+
 size_t router_logits_smem_bytes(int e_pad) {
   return 1024 + static_cast<size_t>(router_stages(e_pad)) * router_stage_bytes(e_pad) +
          sizeof(RouterSmem);
@@ -323,7 +385,7 @@ size_t router_logits_smem_bytes(int e_pad) {
 cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, const float *w_r,
                          const float *bias, int T, int H, int E, int K, float scale,
                          uint16_t *wsplit, float *zp, int32_t *idx, float *gate, float *margin,
-                         int *err, int num_sms, cudaStream_t stream) {
+                         float *logits, int *err, int num_sms, cudaStream_t stream) {
   const int e_pad = router_e_pad(E);
   router_split_kernel<<<num_sms * 4, 256, 0, stream>>>(w_r, E, e_pad, H, wsplit);
   const int kblocks = H / rt::BK;
@@ -331,28 +393,31 @@ cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, c
   const int kb_per = (kblocks + splits - 1) / splits;
   const int stages = router_stages(e_pad);
   uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(e_pad)) cols <<= 1;
+  while (cols < static_cast<uint32_t>(2 * e_pad)) cols <<= 1;  // two ping-pong accumulators
   const size_t smem = router_logits_smem_bytes(e_pad);
-  cudaError_t e = cudaFuncSetAttribute(router_logits_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   dim3 grid((T + rt::BM - 1) / rt::BM, (kblocks + kb_per - 1) / kb_per);
-  router_logits_kernel<<<grid, rt::THREADS, smem, stream>>>(tmap_x, tmap_w, T, e_pad, kb_per,
-                                                            kblocks, stages, cols, zp, err);
+  cudaError_t e = cudaSuccess;
+  switch (e_pad / 64) {
+    case 1: e = launch_logits<1>(grid, smem, tmap_x, tmap_w, T, kb_per, kblocks, stages, cols, zp, err, stream); break;
+    case 2: e = launch_logits<2>(grid, smem, tmap_x, tmap_w, T, kb_per, kblocks, stages, cols, zp, err, stream); break;
+    case 3: e = launch_logits<3>(grid, smem, tmap_x, tmap_w, T, kb_per, kblocks, stages, cols, zp, err, stream); break;
+    default: e = launch_logits<4>(grid, smem, tmap_x, tmap_w, T, kb_per, kblocks, stages, cols, zp, err, stream); break;
+  }
+  if (e != cudaSuccess) return e;
   const int used_splits = static_cast<int>(grid.y);
   const int blocks = (T + 7) / 8;
   if (E <= 32)
     router_select_kernel<1><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
-                                                        idx, gate, margin);
+                                                        idx, gate, margin, logits);
   else if (E <= 64)
     router_select_kernel<2><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
-                                                        idx, gate, margin);
+                                                        idx, gate, margin, logits);
   else if (E <= 128)
     router_select_kernel<4><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
-                                                        idx, gate, margin);
+                                                        idx, gate, margin, logits);
   else
     router_select_kernel<8><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
-                                                        idx, gate, margin);
+                                                        idx, gate, margin, logits);
   return cudaGetLastError();
 }
 

@@ -108,7 +108,7 @@ def lib():
         L.moe_pack_weights.restype = ctypes.c_int
         L.moe_pack_weights.argtypes = [P(_Cfg)] + [vp] * 9
         L.moe_route.restype = ctypes.c_int
-        L.moe_route.argtypes = [P(_Cfg)] + [vp] * 7 + [ctypes.c_size_t, vp]
+        L.moe_route.argtypes = [P(_Cfg)] + [vp] * 8 + [ctypes.c_size_t, vp]
         L.moe_permute.restype = ctypes.c_int
         L.moe_permute.argtypes = [P(_Cfg), vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.moe_forward.restype = ctypes.c_int
@@ -194,8 +194,9 @@ def pack_weights(cfg: Config, w1, w3, w2, ws1=None, ws3=None, ws2=None, stream=N
     return w13, w2p
 
 
-def route(cfg: Config, x, w_router, bias, ws, want_margin=True, out=None, stream=None):
-    """Router: returns (topk_idx int32 [T,K], topk_gate fp32 [T,K], margin fp32 [T] or None)."""
+def route(cfg: Config, x, w_router, bias, ws, want_margin=True, out=None, logits=None, stream=None):
+    """Router: returns (topk_idx int32 [T,K], topk_gate fp32 [T,K], margin fp32 [T] or None).
+    ``logits``: optional fp32 [T, E] tensor that receives z (router_logits)."""
     T, H, E, K = cfg.T, cfg.H, cfg.E, cfg.K
     _req(x, torch.bfloat16, (T, H), "x")
     _req(w_router, torch.float32, (E, H), "w_router")
@@ -207,7 +208,8 @@ def route(cfg: Config, x, w_router, bias, ws, want_margin=True, out=None, stream
     else:
         idx, gate, margin = out
     _check(lib().moe_route(ctypes.byref(cfg.c()), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(idx),
-                           _ptr(gate), _ptr(margin), _ptr(ws), ws.numel(), _stream(stream)), "moe_route")
+                           _ptr(gate), _ptr(margin), _ptr(logits), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_route")
     return idx, gate, margin
 
 
@@ -300,9 +302,9 @@ class MoeBlock:
         self.sorted = torch.empty((cfg.rows,), dtype=torch.int32, device=dev)
         self.y = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
 
-    def __call__(self, x, stream=None):
+    def __call__(self, x, stream=None, logits=None):
         route(self.cfg, x, self.w_router, self.bias, self.ws, out=(self.idx, self.gate, self.margin),
-              stream=stream)
+              logits=logits, stream=stream)
         permute(self.cfg, self.idx, self.ws, out=(self.counts, self.offsets, self.sorted), stream=stream)
         return forward(self.cfg, self.weights, x, self.gate, self.offsets, self.sorted, self.ws, y=self.y,
                        stream=stream)

@@ -8,6 +8,9 @@ Acceptance rules (the layer's own tolerance, written here once):
     the index comparison and counted;
   * permutation: counts / offsets / sorted bit-identical to the oracle's
     counting sort of the GPU's own indices;
+  * logits: |z_gpu - z_oracle| <= Z_TOL * (1 + max|z|) (fp32-accurate);
+  * slot order: descending exact key, except between selected keys closer
+    than ORDER_TOL (within the router's precision either order is correct);
   * gates: |G_gpu - G_oracle| <= GATE_TOL per expert on tokens with equal sets;
   * output: |y_gpu - y_oracle| <= Y_TOL * RMS(y_oracle) + half_ulp_bf16(y_oracle)
     element by element, where the oracle is exact (double) and uses the GPU's
@@ -26,6 +29,8 @@ from sigmoid_routed_mixture_b200 import moe
 from sigmoid_routed_mixture_b200 import workloads as W
 
 MARGIN_TOL = 1e-4
+Z_TOL = 2e-6
+ORDER_TOL = 1e-5
 GATE_TOL = 2e-5
 Y_TOL = 2e-2
 
@@ -76,13 +81,14 @@ class Case:
     def run(self):
         """Route + permute + forward on the GPU; returns host copies of every output."""
         blk = self.block()
-        y = blk(self.x_dev)
+        logits = torch.empty((self.w.T, self.w.E), dtype=torch.float32, device="cuda")
+        y = blk(self.x_dev, logits=logits)
         torch.cuda.synchronize()
         err = moe.device_error(blk.ws)
         return dict(idx=blk.idx.cpu().numpy(), gate=blk.gate.cpu().numpy(),
                     margin=blk.margin.cpu().numpy(), counts=blk.counts.cpu().numpy(),
                     offsets=blk.offsets.cpu().numpy(), sorted=blk.sorted.cpu().numpy(),
-                    y=bf16_to_f64(y), err=err, block=blk)
+                    y=bf16_to_f64(y), logits=logits.cpu().numpy(), err=err, block=blk)
 
     def host_expert(self, name, e):
         key = (name, e)
@@ -114,7 +120,10 @@ def check_route(case: Case, res, tokens=None):
     """Selection, gate and margin parity on `tokens` (all when None); returns near-tie count."""
     w = case.w
     tok = np.arange(w.T) if tokens is None else np.asarray(tokens)
-    idx_o, gate_o, margin_o, _ = O.route(case.x[tok], case.w_r, case.b, w.K, w.scale)
+    idx_o, gate_o, margin_o, z_o = O.route(case.x[tok], case.w_r, case.b, w.K, w.scale)
+    # logits: fp32-accurate (three-part split of W_r, fp32 accumulation)
+    dz = np.abs(res["logits"][tok] - z_o)
+    assert dz.max() <= Z_TOL * (1.0 + np.abs(z_o).max()), "router logits off by %g" % dz.max()
     idx_g, gate_g, margin_g = res["idx"][tok], res["gate"][tok], res["margin"][tok]
     clear = margin_o > MARGIN_TOL
     near = int((~clear).sum())
@@ -125,11 +134,10 @@ def check_route(case: Case, res, tokens=None):
         for k in range(w.K):
             assert abs(gate_g[r, k] - go[int(idx_g[r, k])]) <= GATE_TOL
     # slot order: descending key where the oracle's adjacent keys are clearly apart
-    z_o = O.logits(case.x[tok], case.w_r)
     key_o = 1.0 / (1.0 + np.exp(-z_o)) + case.b.astype(np.float64)
     for r in np.nonzero(clear)[0]:
         ks = key_o[r, idx_g[r]]
-        assert np.all(np.diff(ks) <= 1e-6), "slot order not descending at token %d" % tok[r]
+        assert np.all(np.diff(ks) <= ORDER_TOL), "slot order not descending at token %d" % tok[r]
     # gates sum to the scale; margins agree where the GPU saw the same choice
     assert np.max(np.abs(gate_g.sum(axis=1) - w.scale)) <= 8 * w.K * np.spacing(np.float32(w.scale))
     finite = np.isfinite(margin_o) & clear

@@ -67,13 +67,13 @@ def test_workspace_size_grows_with_tokens(L):
 def test_invalid_configs_rejected(L, bad, code):
     c = cfg(**bad).c()
     assert L.moe_workspace_size(ctypes.byref(c)) == 0
-    rc = L.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, 0, None)
+    rc = L.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None, 0, None)
     assert rc == code
 
 
 def test_null_pointers_rejected_before_launch(L):
     c = cfg().c()
-    assert L.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, 0, None) == 1
+    assert L.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None, 0, None) == 1
     assert L.moe_permute(ctypes.byref(c), None, None, None, None, None, 0, None) == 1
     assert L.moe_forward(ctypes.byref(c), None, None, None, None, None, None, None, 0, None) == 1
     assert L.moe_pack_weights(ctypes.byref(c), None, None, None, None, None, None, None, None, None) == 1
@@ -85,14 +85,15 @@ def test_misaligned_and_small_workspace_rejected(L):
     c = cfg().c()
     fake = ctypes.c_void_p(0x10001)  # never dereferenced: validation fails first
     aligned = ctypes.c_void_p(0x100000)
-    assert L.moe_route(ctypes.byref(c), fake, aligned, aligned, aligned, aligned, None, aligned, 1 << 40, None) == 3
+    assert L.moe_route(ctypes.byref(c), fake, aligned, aligned, aligned, aligned, None, None, aligned, 1 << 40,
+                       None) == 3
     need = L.moe_workspace_size(ctypes.byref(c))
     assert L.moe_permute(ctypes.byref(c), aligned, aligned, aligned, aligned, aligned, need - 1, None) == 4
 
 
 def test_zero_tokens_is_a_no_op(L):
     c = cfg(T=0).c()
-    assert L.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, 0, None) == 0
+    assert L.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None, 0, None) == 0
     assert L.moe_forward(ctypes.byref(c), None, None, None, None, None, None, None, 0, None) == 0
 
 

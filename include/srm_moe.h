@@ -170,6 +170,30 @@ moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
  *   (Delta_ffn = y_routed + y_shared). */
 moe_status_t moe_combine(const moe_cfg_t *cfg, void *y, void *ws, size_t ws_bytes, void *stream);
 
+/* moe_permute for callers that cannot allocate device memory (the pages have
+ * no counterpart of this entry point; it exists for embedding).  Some hosts
+ * cannot call cudaMalloc for a workspace: an engine that has reserved all
+ * device memory for its own pool, a serving loop where cudaMalloc's implicit
+ * device-wide synchronisation is not allowed, or a plugin that only receives
+ * the tensors it works on.  This variant computes exactly what moe_permute
+ * computes (same counts, offsets and sorted, bit for bit) with its scratch in
+ * a static device array inside the library instead of a workspace.
+ *   Limit: T * K <= 262144 (e.g. 32768 tokens at top-8), E <= 256; larger
+ *   calls return MOE_ERR_UNSUPPORTED before any launch.
+ *   Memory: every GPU that loads the library holds the array (about 256 KB)
+ *   until the process exits.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (with that device current); make that first call before any stream
+ *   capture.
+ *   Sharing: all calls use the same array and it keeps the last call's
+ *   contents (each call clears its error word first); calls that overlap on
+ *   the GPU (unordered streams) race on it.
+ *   Errors: an expert id outside [0, E) is skipped and reported in-band by
+ *   setting offsets[0] = -1 (always 0 otherwise); the outputs are then not
+ *   usable. */
+moe_status_t moe_permute_noalloc(const moe_cfg_t *cfg, const int32_t *topk_idx, int32_t *counts,
+                                 int32_t *offsets, int32_t *sorted, void *stream);
+
 /* Read (and clear) the device error word of a workspace.  Synchronises
  * `stream`.  *device_status receives MOE_OK or the first device-side error
  * recorded since the last read.  Returns MOE_ERR_CUDA if the copy fails. */

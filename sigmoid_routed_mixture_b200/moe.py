@@ -34,6 +34,7 @@ SYMBOLS = (
     "moe_combine",
     "moe_get_device_error",
     "moe_status_string",
+    "moe_permute_noalloc",
 )
 
 STATUS = {
@@ -121,6 +122,8 @@ def lib():
         L.moe_combine.argtypes = [P(_Cfg), vp, vp, ctypes.c_size_t, vp]
         L.moe_get_device_error.restype = ctypes.c_int
         L.moe_get_device_error.argtypes = [vp, P(ctypes.c_int), vp]
+        L.moe_permute_noalloc.restype = ctypes.c_int
+        L.moe_permute_noalloc.argtypes = [P(_Cfg), vp, vp, vp, vp, vp]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [ctypes.c_int]
         _lib = L
@@ -225,6 +228,21 @@ def permute(cfg: Config, topk_idx, ws, out=None, stream=None):
         counts, offsets, sorted_ = out
     _check(lib().moe_permute(ctypes.byref(cfg.c()), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
                              _ptr(sorted_), _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
+    return counts, offsets, sorted_
+
+
+def permute_noalloc(cfg: Config, topk_idx, out=None, stream=None):
+    """moe_permute without a workspace (library-held scratch; T*K <= 262144)."""
+    _req(topk_idx, torch.int32, (cfg.T, cfg.K), "topk_idx")
+    dev = topk_idx.device
+    if out is None:
+        counts = torch.empty((cfg.E + 1,), dtype=torch.int32, device=dev)
+        offsets = torch.empty((cfg.E + 2,), dtype=torch.int32, device=dev)
+        sorted_ = torch.empty((cfg.rows,), dtype=torch.int32, device=dev)
+    else:
+        counts, offsets, sorted_ = out
+    _check(lib().moe_permute_noalloc(ctypes.byref(cfg.c()), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                                     _ptr(sorted_), _stream(stream)), "moe_permute_noalloc")
     return counts, offsets, sorted_
 
 

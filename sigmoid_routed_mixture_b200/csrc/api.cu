@@ -259,7 +259,7 @@ moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights, c
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tm_x, tm_w13;
   if (!make_tmap(&tm_x, wsb + L.xs, H, static_cast<uint64_t>(rows_y(*cfg)), 64, 128) ||
-      !make_tmap(&tm_w13, weights->w13, H, static_cast<uint64_t>(E + 1) * 2 * I, 64, 256))
+      !make_tmap(&tm_w13, weights->w13, H, static_cast<uint64_t>(E + 1) * 2 * I, 64, 128))
     return MOE_ERR_CUDA;
   if (srm::launch_gather_rows(static_cast<const uint16_t *>(x), sorted, static_cast<int>(cfg->T), H,
                               cfg->K, cfg->has_shared, reinterpret_cast<int32_t *>(wsb + L.pos),
@@ -290,7 +290,7 @@ moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
   CUtensorMap tm_h, tm_w2;
   if (!make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(rows_y(*cfg)), 64, 128,
                  CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-      !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(E + 1) * H, 64, 256,
+      !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(E + 1) * H, 64, 128,
                  CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_CUDA;
   GemmArgs p = gemm_args(*cfg, offsets, sorted, topk_gate, wsb, L);

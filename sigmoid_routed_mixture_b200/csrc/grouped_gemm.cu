@@ -1,6 +1,7 @@
 // grouped_gemm.cu -- the two expert contractions of the mixture on the
 // 5th-generation tensor cores (tcgen05.mma, accumulators in tensor memory),
-// fed by TMA, as one persistent, warp-specialised kernel template.
+// fed by TMA, as one persistent, warp-specialised kernel template that runs
+// on CTA pairs.
 //
 // Definition ("GLM-5 . MoE transformer block", "All 43 steps", Mixture of
 // experts): per expert i and token row x,
@@ -11,27 +12,42 @@
 //
 //   kUp   : for every group g (routed experts 0..E-1, shared expert E) and its
 //           rows, [g | u] = xs_rows . W13_g^T where xs holds the token rows in
-//           expert-sorted order (gather.cu); epilogue h = silu(g) * u -> fp16 h[row][I] (three more mantissa
-//           bits than bf16 at the same tensor-core rate; |h| saturates at
-//           65504).
+//           expert-sorted order (gather.cu); epilogue h = silu(g) * u -> fp16
+//           h[row][I] (three more mantissa bits than bf16 at the same
+//           tensor-core rate; |h| saturates at 65504).
 //   kDown : Y[a] = G[a] * (h_rows . W2_g^T) in fp16 x fp16 (W2 packed as
 //           fp16, an exact conversion of bf16 weights in fp16's normal
-//           range), rows of h contiguous, epilogue
-//           multiplies by the routing gate (1 for the shared expert) and
-//           scatters fp32 rows to their (token, slot) position a (fp32 so that
-//           the only roundings after the tensor cores are h and the final y).
+//           range), rows of h contiguous, epilogue multiplies by the routing
+//           gate (1 for the shared expert) and scatters fp32 rows to their
+//           (token, slot) position a (fp32 so that the only roundings after
+//           the tensor cores are h and the final y).
 //
-// Tiling: one work tile = 128 rows x 256 output columns, K loop in steps of
-// 64 (one 128-byte swizzle atom), 4-stage TMA ring, two 128x256 fp32
-// accumulators in tensor memory (512 columns) so the epilogue of one tile
-// overlaps the main loop of the next.  Warp roles (6 warps):
-//   warp 0: TMA producer (one lane issues the A and B tile loads)
-//   warp 1: tensor-memory allocation + single-thread MMA issue
+// Tiling: a cluster of two CTAs (a CTA pair) owns one work tile of 256 rows x
+// 256 output columns: each CTA loads its 128 rows of A and 128 of the 256
+// rows of B (so every B byte crosses L2 once per pair, not once per CTA), and
+// the leader CTA issues tcgen05.mma.cta_group::2 with M = 256 that reads both
+// CTAs' shared memory and leaves each CTA's 128 x 256 fp32 accumulator in its
+// own tensor memory.  K loop in steps of 64 (one 128-byte swizzle atom), a
+// 6-stage TMA ring per CTA, two accumulators per CTA (512 TMEM columns) so the
+// epilogue of one tile overlaps the main loop of the next.
+// Warp roles (6 warps per CTA):
+//   warp 0: TMA producer (one lane issues the CTA's A and B tile loads)
+//   warp 1: tensor-memory allocation; in the leader also single-thread MMA issue
 //   warps 2-5: epilogue (tensor memory -> registers -> global)
-// Work tiles are (group, 128-row block, 256-column block), column block
-// fastest, dealt round-robin over a grid of one CTA per SM; the per-group
+// Work tiles are (group, 256-row block, 256-column block), column block
+// fastest, dealt round-robin over the persistent CTA pairs; the per-group
 // row-block counts come from the group offsets on the device, so the host
 // never synchronises.
+//
+// Barrier protocol of a pair (no TMA multicast anywhere):
+//   full[s]   (leader's)  producer of the leader arms it with both CTAs' bytes;
+//                         both CTAs' loads complete on it
+//   empty[s]  (each CTA)  the leader's commit multicasts to both when the
+//                         MMAs reading stage s are done
+//   tfull[a]  (each CTA)  the leader's commit multicasts to both when
+//                         accumulator a is complete
+//   tempty[a] (leader's)  the 4 epilogue warps of each CTA arrive (8 in all)
+//                         when they have drained accumulator a
 #include <cuda.h>
 
 #include "common.cuh"
@@ -40,12 +56,14 @@
 namespace srm {
 
 namespace gg {
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;        // rows per CTA (256 per pair)
+constexpr int PAIR_M = 256;
+constexpr int BN = 256;        // output columns per tile
+constexpr int BN_HALF = 128;   // B rows loaded by each CTA
 constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;   // 16 KB
-constexpr int B_BYTES = BN * BK * 2;   // 32 KB
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK * 2;        // 16 KB
+constexpr int B_BYTES = BN_HALF * BK * 2;   // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
@@ -69,13 +87,13 @@ constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 
 
 struct TileCoord {
   int g;          // group
-  int row_base;   // first row of the tile in the expert-sorted order
-  int rows;       // valid rows in the tile (1..128)
+  int row_base;   // first row of this CTA's half of the tile (expert-sorted order)
+  int rows;       // valid rows of this CTA's half (0..128)
   int n0;         // first output column
 };
 
 __device__ __forceinline__ TileCoord decode_tile(const gg::Smem &s, int groups, int n_tiles,
-                                                 int tile) {
+                                                 int tile, int rank) {
   const int mt = tile / n_tiles;
   const int nt = tile - mt * n_tiles;
   int lo = 0, hi = groups - 1;  // last g with tile_start[g] <= mt
@@ -88,14 +106,14 @@ __device__ __forceinline__ TileCoord decode_tile(const gg::Smem &s, int groups, 
   }
   TileCoord c;
   c.g = lo;
-  c.row_base = s.grp_off[lo] + (mt - s.tile_start[lo]) * gg::BM;
-  c.rows = min(gg::BM, s.grp_off[lo + 1] - c.row_base);
+  c.row_base = s.grp_off[lo] + (mt - s.tile_start[lo]) * gg::PAIR_M + rank * gg::BM;
+  c.rows = max(0, min(gg::BM, s.grp_off[lo + 1] - c.row_base));
   c.n0 = nt * gg::BN;
   return c;
 }
 
 template <int kMode>
-__global__ void __launch_bounds__(gg::THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         const __grid_constant__ CUtensorMap tmap_b, GemmArgs p) {
   using namespace gg;
@@ -108,11 +126,15 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
   const int groups = p.groups;
   const int n_tiles = p.n_total / BN;
   const int kblocks = p.k_total / BK;
   // up: bf16 x times bf16 W13; down: fp16 h times fp16 W2
-  constexpr uint32_t IDESC = umma_idesc_f32acc(BM, BN, kMode == kUp ? 1u : 0u);
+  constexpr uint32_t IDESC = umma_idesc_f32acc(PAIR_M, BN, kMode == kUp ? 1u : 0u);
 
   // ---- prologue: barriers, tensor memory, per-group tile starts
   if (threadIdx.x == 0) {
@@ -122,7 +144,7 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.tfull[i], 1);
-      mbar_init(&s.tempty[i], 4);
+      mbar_init(&s.tempty[i], 8);
     }
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
@@ -132,18 +154,18 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
     tma_prefetch_desc(&tmap_b);
   }
   if (warp == 1) {
-    tmem_alloc(&s.tmem_base, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(&s.tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   if (warp == 0) {
-    // group offsets and an exclusive scan of ceil(count / BM) over the groups
+    // group offsets and an exclusive scan of ceil(count / 256) over the groups
     const int per = (groups + 31) / 32;
     const int g0 = lane * per;
     int local = 0;
     for (int g = g0; g < min(g0 + per, groups); ++g) {
       const int o0 = p.offsets[g], o1 = p.offsets[g + 1];
       s.grp_off[g] = o0;
-      local += (o1 - o0 + BM - 1) / BM;
+      local += (o1 - o0 + PAIR_M - 1) / PAIR_M;
     }
     int incl = local;
 #pragma unroll
@@ -154,7 +176,7 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
     int run = incl - local;
     for (int g = g0; g < min(g0 + per, groups); ++g) {
       s.tile_start[g] = run;
-      run += (p.offsets[g + 1] - p.offsets[g] + BM - 1) / BM;
+      run += (p.offsets[g + 1] - p.offsets[g] + PAIR_M - 1) / PAIR_M;
     }
     if (lane == 31) {
       s.total_mtiles = incl;
@@ -163,32 +185,33 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // the peer's barriers are initialised before any remote use
   tc_fence_after();
 
   const uint32_t tmem_base = s.tmem_base;
   const int total_tiles = s.total_mtiles * n_tiles;
   volatile int *abort_flag = &s.abort_flag;
-  int issued = 0;  // k-blocks armed by the producer (lane 0's count)
+  int issued = 0;  // k-blocks this CTA's producer has loaded
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     uint32_t stage = 0, phase = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const TileCoord c = decode_tile(s, groups, n_tiles, tile);
-      const int b_row = c.g * p.n_total + c.n0;
+    for (int tile = pair; tile < total_tiles; tile += num_pairs) {
+      const TileCoord c = decode_tile(s, groups, n_tiles, tile, rank);
+      const int b_row = c.g * p.n_total + c.n0 + rank * BN_HALF;
       bool ok = true;
       for (int kb = 0; kb < kblocks; ++kb) {
         if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, p.err)) {
           ok = false;
           break;
         }
-        if (lane == 0) mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
-        __syncwarp();
         if (lane == 0) {
-          tma_load_2d(sA + stage * A_BYTES, &tmap_a, &s.full[stage], kb * BK, c.row_base);
-          tma_load_2d(sB + stage * B_BYTES, &tmap_b, &s.full[stage], kb * BK, b_row);
+          const uint32_t full_leader = cluster_map(&s.full[stage], 0);
+          if (leader) mbar_arrive_expect_tx(&s.full[stage], 2 * STAGE_BYTES);
+          tma_load_2d_pair(sA + stage * A_BYTES, &tmap_a, full_leader, kb * BK, c.row_base);
+          tma_load_2d_pair(sB + stage * B_BYTES, &tmap_b, full_leader, kb * BK, b_row);
         }
+        __syncwarp();
         ++issued;
         if (++stage == STAGES) {
           stage = 0;
@@ -198,51 +221,53 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
       if (!ok) break;
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-    int consumed = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag, p.err)) break;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * BN;
-      bool ok = true;
-      for (int kb = 0; kb < kblocks; ++kb) {
-        if (!mbar_wait(&s.full[stage], phase, abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader) {
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      int consumed = 0;
+      for (int tile = pair; tile < total_tiles; tile += num_pairs) {
+        if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag, p.err)) break;
         tc_fence_after();
-        ++consumed;
-        if (lane == 0) {
-          const uint32_t a_addr = smem_addr(sA + stage * A_BYTES);
-          const uint32_t b_addr = smem_addr(sB + stage * B_BYTES);
-#pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            umma_bf16(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32),
-                      IDESC, (kb | k) != 0 ? 1u : 0u);
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&s.full[stage], phase, abort_flag, p.err)) {
+            ok = false;
+            break;
           }
-          umma_commit(&s.empty[stage]);
+          tc_fence_after();
+          ++consumed;
+          if (lane == 0) {
+            const uint32_t a_addr = smem_addr(sA + stage * A_BYTES);
+            const uint32_t b_addr = smem_addr(sB + stage * B_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k) {
+              umma_pair(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32),
+                        IDESC, (kb | k) != 0 ? 1u : 0u);
+            }
+            umma_commit_pair(&s.empty[stage], 0x3);
+          }
+          __syncwarp();
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
+        if (!ok) break;
+        if (lane == 0) umma_commit_pair(&s.tfull[acc], 0x3);
         __syncwarp();
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
       }
-      if (!ok) break;
-      if (lane == 0) umma_commit(&s.tfull[acc]);
-      __syncwarp();
-      acc ^= 1u;
-      if (acc == 0) acc_phase ^= 1u;
+      if (lane == 0) s.mma_consumed = consumed;
     }
-    if (lane == 0) s.mma_consumed = consumed;
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // tensor-memory lane quarter this warp may access
     const int row = q * 32 + lane;
     uint32_t acc = 0, acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const TileCoord c = decode_tile(s, groups, n_tiles, tile);
+    for (int tile = pair; tile < total_tiles; tile += num_pairs) {
+      const TileCoord c = decode_tile(s, groups, n_tiles, tile, rank);
       if (!mbar_wait(&s.tfull[acc], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
       bool valid = row < c.rows;
@@ -296,27 +321,41 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.tempty[acc]);
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(&s.tempty[acc]);
+        else
+          mbar_arrive_remote(cluster_map(&s.tempty[acc], 0));
+      }
       acc ^= 1u;
       if (acc == 0) acc_phase ^= 1u;
     }
   }
 
   // ---- teardown.  On the error path wait (bounded) for copies and MMAs still
-  // in flight before the shared and tensor memory are given back.
+  // in flight before shared and tensor memory are given back; then both CTAs
+  // of the pair meet so neither leaves while the other may still touch its
+  // shared memory.
   __syncthreads();
   if (s.abort_flag) {
     if (warp == 0 && lane == 0) {
-      for (int i = s.mma_consumed; i < issued; ++i) {
-        const uint32_t a = smem_addr(&s.full[i % STAGES]);
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(a, static_cast<uint32_t>((i / STAGES) & 1)) &&
-               global_timer_ns() - t0 < kWaitLimitNs) {
+      // the leader's full barriers count both CTAs' bytes; the peer waits a
+      // bounded time for its own copies to land
+      const uint64_t t0 = global_timer_ns();
+      if (leader) {
+        for (int i = s.mma_consumed; i < issued; ++i) {
+          const uint32_t a = smem_addr(&s.full[i % STAGES]);
+          while (!mbar_try_wait(a, static_cast<uint32_t>((i / STAGES) & 1)) &&
+                 global_timer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      } else {
+        while (global_timer_ns() - t0 < 1000000ull) {
         }
       }
     }
-    if (warp == 1 && lane == 0) {
-      umma_commit(&s.drain);
+    if (warp == 1 && lane == 0 && leader) {
+      umma_commit_pair(&s.drain, 0x1);
       const uint32_t a = smem_addr(&s.drain);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(a, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
@@ -325,9 +364,10 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -335,12 +375,34 @@ size_t grouped_gemm_smem_bytes() { return gg::SMEM_BYTES; }
 
 template <int kMode>
 static cudaError_t launch_mode(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p,
-                               int grid, cudaStream_t stream) {
+                               int num_sms, cudaStream_t stream) {
   auto kern = grouped_gemm_kernel<kMode>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, gg::THREADS, gg::SMEM_BYTES, stream>>>(ta, tb, p);
+  // persistent: as many CTA pairs as can be resident at once
+  static int cached_pairs[2][64] = {{0}};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int &pairs = cached_pairs[kMode][dev & 63];
+  if (pairs == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_sms & ~1);
+    cfg.blockDim = dim3(gg::THREADS);
+    cfg.dynamicSmemBytes = gg::SMEM_BYTES;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters <= 0)
+      clusters = num_sms / 2;
+    pairs = clusters;
+  }
+  kern<<<2 * pairs, gg::THREADS, gg::SMEM_BYTES, stream>>>(ta, tb, p);
   return cudaGetLastError();
 }
 

@@ -257,9 +257,11 @@ moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights, c
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   const int H = cfg->H, I = cfg->I, E = cfg->E;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool pair = srm::gemm_use_pairs(cfg->T, cfg->K, cfg->E);
   CUtensorMap tm_x, tm_w13;
   if (!make_tmap(&tm_x, wsb + L.xs, H, static_cast<uint64_t>(rows_y(*cfg)), 64, 128) ||
-      !make_tmap(&tm_w13, weights->w13, H, static_cast<uint64_t>(E + 1) * 2 * I, 64, 128))
+      !make_tmap(&tm_w13, weights->w13, H, static_cast<uint64_t>(E + 1) * 2 * I, 64,
+                 static_cast<uint32_t>(srm::gemm_b_box_rows(pair))))
     return MOE_ERR_CUDA;
   if (srm::launch_gather_rows(static_cast<const uint16_t *>(x), sorted, static_cast<int>(cfg->T), H,
                               cfg->K, cfg->has_shared, reinterpret_cast<int32_t *>(wsb + L.pos),
@@ -271,7 +273,7 @@ moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights, c
   p.n_total = 2 * I;
   p.k_total = H;
   p.out_ld = I;
-  return cuda_status(srm::launch_grouped_gemm(srm::kUp, tm_x, tm_w13, p, num_sms(), s));
+  return cuda_status(srm::launch_grouped_gemm(srm::kUp, pair, tm_x, tm_w13, p, num_sms(), s));
 }
 
 moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
@@ -287,18 +289,19 @@ moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
     return MOE_ERR_ALIGN;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   const int H = cfg->H, I = cfg->I, E = cfg->E;
+  const bool pair = srm::gemm_use_pairs(cfg->T, cfg->K, cfg->E);
   CUtensorMap tm_h, tm_w2;
   if (!make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(rows_y(*cfg)), 64, 128,
                  CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-      !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(E + 1) * H, 64, 128,
-                 CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+      !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(E + 1) * H, 64,
+                 static_cast<uint32_t>(srm::gemm_b_box_rows(pair)), CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_CUDA;
   GemmArgs p = gemm_args(*cfg, offsets, sorted, topk_gate, wsb, L);
   p.out = wsb + L.ybuf;
   p.n_total = H;
   p.k_total = I;
   p.out_ld = H;
-  return cuda_status(srm::launch_grouped_gemm(srm::kDown, tm_h, tm_w2, p, num_sms(),
+  return cuda_status(srm::launch_grouped_gemm(srm::kDown, pair, tm_h, tm_w2, p, num_sms(),
                                               static_cast<cudaStream_t>(stream)));
 }
 

@@ -56,22 +56,31 @@
 namespace srm {
 
 namespace gg {
-constexpr int BM = 128;        // rows per CTA (256 per pair)
-constexpr int PAIR_M = 256;
+constexpr int BM = 128;        // rows per CTA
 constexpr int BN = 256;        // output columns per tile
-constexpr int BN_HALF = 128;   // B rows loaded by each CTA
 constexpr int BK = 64;
-constexpr int STAGES = 6;
-constexpr int A_BYTES = BM * BK * 2;        // 16 KB
-constexpr int B_BYTES = BN_HALF * BK * 2;   // 16 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
 constexpr int MAX_GROUPS = 257;
+constexpr int MAX_STAGES = 6;
+
+// kPair: a CTA pair shares each 256-row tile (M = 256, each CTA loads half of
+// B); solo: one CTA per 128-row tile (M = 128, the CTA loads all of B).
+template <bool kPair>
+struct Cfg {
+  static constexpr int TILE_M = kPair ? 2 * BM : BM;
+  static constexpr int B_ROWS = kPair ? BN / 2 : BN;     // B rows loaded per CTA
+  static constexpr int STAGES = kPair ? 6 : 4;
+  static constexpr int A_BYTES = BM * BK * 2;            // 16 KB
+  static constexpr int B_BYTES = B_ROWS * BK * 2;        // 16 or 32 KB
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TX_BYTES = (kPair ? 2 : 1) * STAGE_BYTES;
+  static constexpr uint32_t EPI_ARRIVALS = kPair ? 8 : 4;
+};
 
 struct Smem {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -82,7 +91,10 @@ struct Smem {
   int tile_start[MAX_GROUPS + 1];
   int grp_off[MAX_GROUPS + 1];
 };
-constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + sizeof(Smem);
+template <bool kPair>
+constexpr size_t smem_bytes() {
+  return 1024 /*alignment slack*/ + Cfg<kPair>::STAGES * Cfg<kPair>::STAGE_BYTES + sizeof(Smem);
+}
 }  // namespace gg
 
 struct TileCoord {
@@ -92,6 +104,7 @@ struct TileCoord {
   int n0;         // first output column
 };
 
+template <bool kPair>
 __device__ __forceinline__ TileCoord decode_tile(const gg::Smem &s, int groups, int n_tiles,
                                                  int tile, int rank) {
   const int mt = tile / n_tiles;
@@ -106,35 +119,40 @@ __device__ __forceinline__ TileCoord decode_tile(const gg::Smem &s, int groups, 
   }
   TileCoord c;
   c.g = lo;
-  c.row_base = s.grp_off[lo] + (mt - s.tile_start[lo]) * gg::PAIR_M + rank * gg::BM;
+  c.row_base = s.grp_off[lo] + (mt - s.tile_start[lo]) * gg::Cfg<kPair>::TILE_M + rank * gg::BM;
   c.rows = max(0, min(gg::BM, s.grp_off[lo + 1] - c.row_base));
   c.n0 = nt * gg::BN;
   return c;
 }
 
-template <int kMode>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                        const __grid_constant__ CUtensorMap tmap_b, GemmArgs p) {
+template <int kMode, bool kPair>
+__device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b,
+                                                  const GemmArgs &p) {
   using namespace gg;
+  using C = Cfg<kPair>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int A_BYTES = C::A_BYTES;
+  constexpr int B_BYTES = C::B_BYTES;
+  constexpr int TILE_M = C::TILE_M;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   uint8_t *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t *sA = base;
   uint8_t *sB = base + STAGES * A_BYTES;
-  Smem &s = *reinterpret_cast<Smem *>(base + STAGES * STAGE_BYTES);
+  Smem &s = *reinterpret_cast<Smem *>(base + STAGES * C::STAGE_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
+  const uint32_t rank = kPair ? cluster_ctarank() : 0;
   const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1;
-  const int num_pairs = gridDim.x >> 1;
+  // a "unit" is a CTA pair (kPair) or a single CTA
+  const int pair = kPair ? (blockIdx.x >> 1) : blockIdx.x;
+  const int num_pairs = kPair ? (gridDim.x >> 1) : gridDim.x;
   const int groups = p.groups;
   const int n_tiles = p.n_total / BN;
   const int kblocks = p.k_total / BK;
   // up: bf16 x times bf16 W13; down: fp16 h times fp16 W2
-  constexpr uint32_t IDESC = umma_idesc_f32acc(PAIR_M, BN, kMode == kUp ? 1u : 0u);
+  constexpr uint32_t IDESC = umma_idesc_f32acc(TILE_M, BN, kMode == kUp ? 1u : 0u);
 
   // ---- prologue: barriers, tensor memory, per-group tile starts
   if (threadIdx.x == 0) {
@@ -144,7 +162,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.tfull[i], 1);
-      mbar_init(&s.tempty[i], 8);
+      mbar_init(&s.tempty[i], C::EPI_ARRIVALS);
     }
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
@@ -154,18 +172,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
     tma_prefetch_desc(&tmap_b);
   }
   if (warp == 1) {
-    tmem_alloc_pair(&s.tmem_base, TMEM_COLS);
-    tmem_relinquish_pair();
+    if (kPair) {
+      tmem_alloc_pair(&s.tmem_base, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&s.tmem_base, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   if (warp == 0) {
-    // group offsets and an exclusive scan of ceil(count / 256) over the groups
+    // group offsets and an exclusive scan of ceil(count / TILE_M) over the groups
     const int per = (groups + 31) / 32;
     const int g0 = lane * per;
     int local = 0;
     for (int g = g0; g < min(g0 + per, groups); ++g) {
       const int o0 = p.offsets[g], o1 = p.offsets[g + 1];
       s.grp_off[g] = o0;
-      local += (o1 - o0 + PAIR_M - 1) / PAIR_M;
+      local += (o1 - o0 + TILE_M - 1) / TILE_M;
     }
     int incl = local;
 #pragma unroll
@@ -176,7 +199,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
     int run = incl - local;
     for (int g = g0; g < min(g0 + per, groups); ++g) {
       s.tile_start[g] = run;
-      run += (p.offsets[g + 1] - p.offsets[g] + PAIR_M - 1) / PAIR_M;
+      run += (p.offsets[g + 1] - p.offsets[g] + TILE_M - 1) / TILE_M;
     }
     if (lane == 31) {
       s.total_mtiles = incl;
@@ -185,7 +208,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
     }
   }
   tc_fence_before();
-  cluster_sync();  // the peer's barriers are initialised before any remote use
+  if (kPair)
+    cluster_sync();  // the peer's barriers are initialised before any remote use
+  else
+    __syncthreads();
   tc_fence_after();
 
   const uint32_t tmem_base = s.tmem_base;
@@ -197,8 +223,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
     // ------------------------------------------------------------ producer
     uint32_t stage = 0, phase = 0;
     for (int tile = pair; tile < total_tiles; tile += num_pairs) {
-      const TileCoord c = decode_tile(s, groups, n_tiles, tile, rank);
-      const int b_row = c.g * p.n_total + c.n0 + rank * BN_HALF;
+      const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, tile, rank);
+      const int b_row = c.g * p.n_total + c.n0 + rank * C::B_ROWS;
       bool ok = true;
       for (int kb = 0; kb < kblocks; ++kb) {
         if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, p.err)) {
@@ -206,10 +232,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
           break;
         }
         if (lane == 0) {
-          const uint32_t full_leader = cluster_map(&s.full[stage], 0);
-          if (leader) mbar_arrive_expect_tx(&s.full[stage], 2 * STAGE_BYTES);
-          tma_load_2d_pair(sA + stage * A_BYTES, &tmap_a, full_leader, kb * BK, c.row_base);
-          tma_load_2d_pair(sB + stage * B_BYTES, &tmap_b, full_leader, kb * BK, b_row);
+          if (leader) mbar_arrive_expect_tx(&s.full[stage], C::TX_BYTES);
+          if (kPair) {
+            const uint32_t full_leader = cluster_map(&s.full[stage], 0);
+            tma_load_2d_pair(sA + stage * A_BYTES, &tmap_a, full_leader, kb * BK, c.row_base);
+            tma_load_2d_pair(sB + stage * B_BYTES, &tmap_b, full_leader, kb * BK, b_row);
+          } else {
+            tma_load_2d(sA + stage * A_BYTES, &tmap_a, &s.full[stage], kb * BK, c.row_base);
+            tma_load_2d(sB + stage * B_BYTES, &tmap_b, &s.full[stage], kb * BK, b_row);
+          }
         }
         __syncwarp();
         ++issued;
@@ -242,10 +273,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
             const uint32_t b_addr = smem_addr(sB + stage * B_BYTES);
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k) {
-              umma_pair(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32),
-                        IDESC, (kb | k) != 0 ? 1u : 0u);
+              if (kPair)
+                umma_pair(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32),
+                          IDESC, (kb | k) != 0 ? 1u : 0u);
+              else
+                umma_bf16(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32),
+                          IDESC, (kb | k) != 0 ? 1u : 0u);
             }
-            umma_commit_pair(&s.empty[stage], 0x3);
+            if (kPair)
+              umma_commit_pair(&s.empty[stage], 0x3);
+            else
+              umma_commit(&s.empty[stage]);
           }
           __syncwarp();
           if (++stage == STAGES) {
@@ -254,7 +292,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
           }
         }
         if (!ok) break;
-        if (lane == 0) umma_commit_pair(&s.tfull[acc], 0x3);
+        if (lane == 0) {
+          if (kPair)
+            umma_commit_pair(&s.tfull[acc], 0x3);
+          else
+            umma_commit(&s.tfull[acc]);
+        }
         __syncwarp();
         acc ^= 1u;
         if (acc == 0) acc_phase ^= 1u;
@@ -267,7 +310,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
     const int row = q * 32 + lane;
     uint32_t acc = 0, acc_phase = 0;
     for (int tile = pair; tile < total_tiles; tile += num_pairs) {
-      const TileCoord c = decode_tile(s, groups, n_tiles, tile, rank);
+      const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, tile, rank);
       if (!mbar_wait(&s.tfull[acc], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
       bool valid = row < c.rows;
@@ -355,7 +398,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
       }
     }
     if (warp == 1 && lane == 0 && leader) {
-      umma_commit_pair(&s.drain, 0x1);
+      if (kPair)
+        umma_commit_pair(&s.drain, 0x1);
+      else
+        umma_commit(&s.drain);
       const uint32_t a = smem_addr(&s.drain);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(a, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
@@ -364,52 +410,78 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync();
+  if (kPair) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    if (kPair)
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
-size_t grouped_gemm_smem_bytes() { return gg::SMEM_BYTES; }
+template <int kMode>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                             const __grid_constant__ CUtensorMap tmap_b, GemmArgs p) {
+  grouped_gemm_body<kMode, true>(tmap_a, tmap_b, p);
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(gg::THREADS, 1)
+    grouped_gemm_solo_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                             const __grid_constant__ CUtensorMap tmap_b, GemmArgs p) {
+  grouped_gemm_body<kMode, false>(tmap_a, tmap_b, p);
+}
+
+bool gemm_use_pairs(int64_t T, int K, int E) { return T * K >= 512LL * E; }
+
+int gemm_b_box_rows(bool pair) { return pair ? gg::Cfg<true>::B_ROWS : gg::Cfg<false>::B_ROWS; }
 
 template <int kMode>
 static cudaError_t launch_mode(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p,
-                               int num_sms, cudaStream_t stream) {
-  auto kern = grouped_gemm_kernel<kMode>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gg::SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  // persistent: as many CTA pairs as can be resident at once
-  static int cached_pairs[2][64] = {{0}};
+                               bool pair, int num_sms, cudaStream_t stream) {
+  static int cached_units[2][2][64] = {{{0}}};
   int dev = 0;
   cudaGetDevice(&dev);
-  int &pairs = cached_pairs[kMode][dev & 63];
-  if (pairs == 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(num_sms & ~1);
-    cfg.blockDim = dim3(gg::THREADS);
-    cfg.dynamicSmemBytes = gg::SMEM_BYTES;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 2;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters <= 0)
-      clusters = num_sms / 2;
-    pairs = clusters;
+  int &units = cached_units[kMode][pair ? 1 : 0][dev & 63];
+  if (pair) {
+    auto kern = grouped_gemm_pair_kernel<kMode>;
+    constexpr size_t smem = gg::smem_bytes<true>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (units == 0) {  // persistent: as many CTA pairs as can be resident at once
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(num_sms & ~1);
+      cfg.blockDim = dim3(gg::THREADS);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 2;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters <= 0)
+        clusters = num_sms / 2;
+      units = clusters;
+    }
+    kern<<<2 * units, gg::THREADS, smem, stream>>>(ta, tb, p);
+  } else {
+    auto kern = grouped_gemm_solo_kernel<kMode>;
+    constexpr size_t smem = gg::smem_bytes<false>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<num_sms, gg::THREADS, smem, stream>>>(ta, tb, p);
   }
-  kern<<<2 * pairs, gg::THREADS, gg::SMEM_BYTES, stream>>>(ta, tb, p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_grouped_gemm(int mode, const CUtensorMap &ta, const CUtensorMap &tb,
-                                const GemmArgs &p, int grid, cudaStream_t stream) {
-  if (mode == kUp) return launch_mode<kUp>(ta, tb, p, grid, stream);
-  return launch_mode<kDown>(ta, tb, p, grid, stream);
+cudaError_t launch_grouped_gemm(int mode, bool pair, const CUtensorMap &ta, const CUtensorMap &tb,
+                                const GemmArgs &p, int num_sms, cudaStream_t stream) {
+  if (mode == kUp) return launch_mode<kUp>(ta, tb, p, pair, num_sms, stream);
+  return launch_mode<kDown>(ta, tb, p, pair, num_sms, stream);
 }
 
 }  // namespace srm

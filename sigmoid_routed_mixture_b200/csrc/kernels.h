@@ -28,9 +28,15 @@ struct GemmArgs {
   int out_ld;              // elements per output row (I for kUp, H for kDown)
 };
 
-size_t grouped_gemm_smem_bytes();
-cudaError_t launch_grouped_gemm(int mode, const CUtensorMap &ta, const CUtensorMap &tb,
-                                const GemmArgs &p, int grid, cudaStream_t stream);
+// Tile shape of the grouped GEMMs: CTA pairs with 256-row tiles when the
+// experts get many rows each (T*K >= 512*E), single CTAs with 128-row tiles
+// otherwise (less padding of each expert's last tile, more weight bytes in
+// flight per SM for small batches).  A tiles are 128 rows; the B box has
+// gemm_b_box_rows(pair) rows.
+bool gemm_use_pairs(int64_t T, int K, int E);
+int gemm_b_box_rows(bool pair);
+cudaError_t launch_grouped_gemm(int mode, bool pair, const CUtensorMap &ta, const CUtensorMap &tb,
+                                const GemmArgs &p, int num_sms, cudaStream_t stream);
 
 // router: W_r split into bf16 parts [3][e_pad][H] (wsplit), fp32 partial logits
 // zp [splits][T][e_pad]; tmap_x: x [T][H] box 64 x 128, tmap_w: wsplit [3*e_pad][H]

@@ -48,6 +48,15 @@ def test_k_equals_e_dense():
     assert np.all(np.isinf(res["margin"]))
 
 
+@pytest.mark.parametrize("T", [2048, 3001])
+def test_cta_pair_tiles(T):
+    """Enough tokens per expert (T*K >= 512*E) for the CTA-pair GEMM tiles of
+    256 rows; 3001 tokens leave ragged 256-row and 128-row tails."""
+    w = W.WORKLOADS["tiny"].replace(T=T, seed=2700 + T)
+    assert T * w.K >= 512 * w.E
+    full_check(w, lambda res: MH.sample_tokens(res, w.T, 400))
+
+
 def test_without_shared_expert():
     full_check(W.WORKLOADS["tiny"].replace(has_shared=False, T=200, seed=2200))
 

@@ -51,7 +51,9 @@ typedef enum {
     MOE_ERR_WORKSPACE = 4,    /* ws_bytes < moe_workspace_size(cfg) */
     MOE_ERR_BAD_INDEX = 5,    /* device: an expert id outside [0, E) in topk_idx */
     MOE_ERR_TIMEOUT = 6,      /* device: a pipeline wait exceeded its time limit */
-    MOE_ERR_CUDA = 7          /* a CUDA runtime or driver call failed */
+    MOE_ERR_CUDA = 7,         /* a CUDA runtime or driver call failed */
+    MOE_ERR_RANGE = 8         /* device: an fp16 intermediate (h or a slot output) exceeded
+                                 +-65504 and was saturated; the result is inexact */
 } moe_status_t;
 
 /* Shape and constants of one MoE block.
@@ -132,8 +134,9 @@ moe_status_t moe_permute(const moe_cfg_t *cfg, const int32_t *topk_idx, int32_t 
 
 /* Expert FFNs and combine:
  *   y[t] = sum over slots k = 0..K-1 (in order) of topk_gate[t][k] * E_{idx}(x_t)
- *          + shared(x_t)   (fp32 per-slot outputs summed in fp32, one final
- *          rounding to bf16).
+ *          + shared(x_t)   (fp16 per-slot outputs summed in fp32, one final
+ *          rounding to bf16; an intermediate beyond the fp16 range saturates
+ *          and is flagged MOE_ERR_RANGE on the device).
  * Gates are used AS GIVEN (no renormalisation), so a caller may zero or edit
  * them (expert ablation).  Inputs: x bf16 [T][H]; topk_gate fp32 [T][K];
  * offsets, sorted from moe_permute.  Output y: bf16 [T][H].
@@ -158,7 +161,7 @@ moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights, c
                            void *stream);
 
 /* moe_expert_down: per row, E_g = h W2_g multiplied by that row's gate
- *   (topk_gate[t][slot]; 1 for the shared expert), written in fp32 to the
+ *   (topk_gate[t][slot]; 1 for the shared expert), written in fp16 to the
  *   row's (token, slot) position in the workspace ("expert_outputs: each
  *   routing slot's weighted expert output", nnterp GLM-5 page, The API). */
 moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,

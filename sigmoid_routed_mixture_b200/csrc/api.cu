@@ -63,7 +63,7 @@ WsLayout layout(const moe_cfg_t &c) {
   L.h = off;
   off = align_up(off + 2ull * static_cast<size_t>(rows_y(c)) * static_cast<size_t>(c.I), 1024);
   L.ybuf = off;
-  off = align_up(off + 4ull * static_cast<size_t>(rows_y(c)) * static_cast<size_t>(c.H), 1024);
+  off = align_up(off + 2ull * static_cast<size_t>(rows_y(c)) * static_cast<size_t>(c.H), 1024);
   L.total = off;
   return L;
 }
@@ -139,6 +139,7 @@ const char *moe_status_string(moe_status_t s) {
     case MOE_ERR_BAD_INDEX: return "expert index out of range (device)";
     case MOE_ERR_TIMEOUT: return "pipeline wait timed out (device)";
     case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_RANGE: return "fp16 intermediate saturated (device)";
   }
   return "unknown status";
 }
@@ -313,7 +314,7 @@ moe_status_t moe_combine(const moe_cfg_t *cfg, void *y, void *ws, size_t ws_byte
   if (!y) return MOE_ERR_ARG;
   if (!aligned(y, 16)) return MOE_ERR_ALIGN;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
-  return cuda_status(srm::launch_combine(reinterpret_cast<const float *>(wsb + L.ybuf),
+  return cuda_status(srm::launch_combine(reinterpret_cast<const uint16_t *>(wsb + L.ybuf),
                                          static_cast<uint16_t *>(y), static_cast<int>(cfg->T),
                                          cfg->H, cfg->K, cfg->has_shared, num_sms(),
                                          static_cast<cudaStream_t>(stream)));

@@ -8,27 +8,26 @@
 // transformer block", "All 43 steps").
 //
 // Pure streaming: each thread owns 8 consecutive columns of one token, loads
-// K+1 rows of 32 fp32 bytes and stores 16 bytes of bf16.
+// K+1 16-byte vectors of fp16 and stores 16 bytes of bf16.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace srm {
 
-__device__ __forceinline__ void add8(float (&acc)[8], const float *src) {
-  const float4 a = __ldcs(reinterpret_cast<const float4 *>(src));
-  const float4 b = __ldcs(reinterpret_cast<const float4 *>(src) + 1);
-  acc[0] += a.x;
-  acc[1] += a.y;
-  acc[2] += a.z;
-  acc[3] += a.w;
-  acc[4] += b.x;
-  acc[5] += b.y;
-  acc[6] += b.z;
-  acc[7] += b.w;
+// 8 fp16 values (16 bytes) added to the fp32 sums
+__device__ __forceinline__ void add8(float (&acc)[8], const uint16_t *src) {
+  const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(src));
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[k]));
+    acc[2 * k] += f.x;
+    acc[2 * k + 1] += f.y;
+  }
 }
 
 __global__ void __launch_bounds__(256)
-    combine_kernel(const float *__restrict__ Y, uint16_t *__restrict__ y, int T, int H, int K,
+    combine_kernel(const uint16_t *__restrict__ Y, uint16_t *__restrict__ y, int T, int H, int K,
                    int has_shared) {
   const int vecs = H / 8;
   const int64_t total = static_cast<int64_t>(T) * vecs;
@@ -49,7 +48,7 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-cudaError_t launch_combine(const float *Y, uint16_t *y, int T, int H, int K, int has_shared,
+cudaError_t launch_combine(const uint16_t *Y, uint16_t *y, int T, int H, int K, int has_shared,
                            int num_sms, cudaStream_t stream) {
   const int64_t total = static_cast<int64_t>(T) * (H / 8);
   int64_t blocks = (total + 255) / 256;

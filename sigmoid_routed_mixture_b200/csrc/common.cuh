@@ -31,8 +31,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Two floats -> one 32-bit word of two fp16 (round to nearest even), low half
-// first; magnitudes beyond the largest finite fp16 saturate to +-65504.
-__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
+// first; magnitudes beyond the largest finite fp16 saturate to +-65504 and
+// set `sat`.
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi, bool &sat) {
+  sat |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
   lo = fminf(fmaxf(lo, -65504.f), 65504.f);
   hi = fminf(fmaxf(hi, -65504.f), 65504.f);
   __half2 p = __floats2half2_rn(lo, hi);

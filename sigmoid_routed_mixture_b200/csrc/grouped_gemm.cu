@@ -14,13 +14,13 @@
 //           rows, [g | u] = xs_rows . W13_g^T where xs holds the token rows in
 //           expert-sorted order (gather.cu); epilogue h = silu(g) * u -> fp16
 //           h[row][I] (three more mantissa bits than bf16 at the same
-//           tensor-core rate; |h| saturates at 65504).
+//           tensor-core rate; |h| saturates at 65504, flagged MOE_ERR_RANGE).
 //   kDown : Y[a] = G[a] * (h_rows . W2_g^T) in fp16 x fp16 (W2 packed as
 //           fp16, an exact conversion of bf16 weights in fp16's normal
 //           range), rows of h contiguous, epilogue multiplies by the routing
-//           gate (1 for the shared expert) and scatters fp32 rows to their
-//           (token, slot) position a (fp32 so that the only roundings after
-//           the tensor cores are h and the final y).
+//           gate (1 for the shared expert) and scatters fp16 rows to their
+//           (token, slot) position a (fp16: 8x finer rounding than bf16 in
+//           the same two bytes; saturation at 65504 is flagged MOE_ERR_RANGE).
 //
 // Tiling: a cluster of two CTAs (a CTA pair) owns one work tile of 256 rows x
 // 256 output columns: each CTA loads its 128 rows of A and 128 of the 256
@@ -320,6 +320,7 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
         valid = false;
       }
       const uint32_t taddr = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
+      bool sat = false;
       if (kMode == kUp) {
         // columns 0..127 of the tile are gate rows, 128..255 the matching up rows
         uint16_t *hrow = reinterpret_cast<uint16_t *>(p.out) +
@@ -336,7 +337,7 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
             for (int j = 0; j < 16; ++j) {
               const float g0 = __uint_as_float(gr[2 * j]), g1 = __uint_as_float(gr[2 * j + 1]);
               const float u0 = __uint_as_float(ur[2 * j]), u1 = __uint_as_float(ur[2 * j + 1]);
-              packed[j] = pack_f16x2_sat(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1);
+              packed[j] = pack_f16x2_sat(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1, sat);
             }
             uint4 *dst = reinterpret_cast<uint4 *>(hrow + ch * 32);
 #pragma unroll
@@ -347,21 +348,26 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
         }
       } else {
         const float gv = (a < p.tk) ? p.gate[valid ? a : 0] : 1.0f;
-        float *yrow = reinterpret_cast<float *>(p.out) + static_cast<size_t>(a) * p.out_ld + c.n0;
+        uint16_t *yrow = reinterpret_cast<uint16_t *>(p.out) + static_cast<size_t>(a) * p.out_ld + c.n0;
 #pragma unroll 1
         for (int ch = 0; ch < BN / 32; ++ch) {
           uint32_t r[32];
           tmem_ld32(taddr + ch * 32, r);
           tmem_ld_wait();
           if (valid) {
-            float4 *dst = reinterpret_cast<float4 *>(yrow + ch * 32);
+            uint32_t packed[16];
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(gv * __uint_as_float(r[4 * v]), gv * __uint_as_float(r[4 * v + 1]),
-                                   gv * __uint_as_float(r[4 * v + 2]), gv * __uint_as_float(r[4 * v + 3]));
+            for (int j = 0; j < 16; ++j)
+              packed[j] = pack_f16x2_sat(gv * __uint_as_float(r[2 * j]), gv * __uint_as_float(r[2 * j + 1]), sat);
+            uint4 *dst = reinterpret_cast<uint4 *>(yrow + ch * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
+                                  packed[4 * v + 3]);
           }
         }
       }
+      if (sat) record_error(p.err, MOE_ERR_RANGE);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {

@@ -16,7 +16,7 @@ struct GemmArgs {
   const int32_t *offsets;  // [groups + 1] first expert-sorted row of each group
   const int32_t *sorted;   // expert-sorted row ids (t*K + slot, or T*K + t for the shared expert)
   const float *gate;       // [T*K] routing gates (kDown)
-  void *out;               // kUp: h bf16 [rows][I];  kDown: Y fp32 [n_rows_y][H]
+  void *out;               // kUp: h fp16 [rows][I];  kDown: Y fp16 [n_rows_y][H]
   int *err;                // device error word
   int T;
   int K;
@@ -60,7 +60,7 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *sorted, int T, 
                                int has_shared, int32_t *pos, uint16_t *xs, int *err, int num_sms,
                                cudaStream_t stream);
 
-cudaError_t launch_combine(const float *Y, uint16_t *y, int T, int H, int K, int has_shared,
+cudaError_t launch_combine(const uint16_t *Y, uint16_t *y, int T, int H, int K, int has_shared,
                            int num_sms, cudaStream_t stream);
 
 cudaError_t launch_pack(const uint16_t *w1, const uint16_t *w3, const uint16_t *w2,

@@ -60,9 +60,10 @@ __global__ void __launch_bounds__(256)
     // bf16 -> fp16: exact for |w| in [2^-17, 65504]; smaller magnitudes keep
     // fp16's subnormal spacing 2^-24, larger ones saturate
     uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    bool sat = false;  // bf16 weights beyond the fp16 range saturate
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-      w[k] = pack_f16x2_sat(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u));
+      w[k] = pack_f16x2_sat(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u), sat);
     *reinterpret_cast<uint4 *>(out + r * I + col) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }

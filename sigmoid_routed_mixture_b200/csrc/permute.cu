@@ -22,13 +22,14 @@ constexpr int CHUNK = 1024;  // assignments per chunk
 constexpr int THREADS = 256;
 constexpr int WARPS = THREADS / 32;
 constexpr int MAX_E = 256;
+constexpr int SCAN_THREADS = 4 * MAX_E;
 }  // namespace pm
 
 int permute_num_chunks(int64_t n_assign) {
   return static_cast<int>((n_assign + pm::CHUNK - 1) / pm::CHUNK);
 }
 
-// 1) chunk histograms: scratch[e * nchunks + c] = entries of chunk c equal to e
+// 1) chunk histograms: scratch[c * E + e] = entries of chunk c equal to e
 __global__ void __launch_bounds__(pm::THREADS)
     permute_hist_kernel(const int32_t *__restrict__ idx, int n, int E, int nchunks,
                         int32_t *__restrict__ scratch, int *err) {
@@ -45,41 +46,62 @@ __global__ void __launch_bounds__(pm::THREADS)
       atomicAdd(&hist[e], 1);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += pm::THREADS) scratch[e * nchunks + c] = hist[e];
+  for (int e = threadIdx.x; e < E; e += pm::THREADS) scratch[c * E + e] = hist[e];
 }
 
 // 2) one CTA: per-expert running sums over the chunks (turning the scratch
-// into each chunk's first destination), counts, and the group offsets.
-__global__ void __launch_bounds__(pm::THREADS)
+// into each chunk's first destination), counts, and the group offsets.  Four
+// threads share an expert, each scanning a quarter of the chunks; for a fixed
+// chunk consecutive threads read consecutive experts (coalesced).
+__global__ void __launch_bounds__(pm::SCAN_THREADS)
     permute_scan_kernel(int32_t *__restrict__ scratch, int E, int nchunks, int T, int has_shared,
                         int32_t *__restrict__ counts, int32_t *__restrict__ offsets) {
-  __shared__ int tot[pm::MAX_E];
+  __shared__ int part_sum[4][pm::MAX_E];
   __shared__ int scan[pm::MAX_E];
-  const int e = threadIdx.x;
+  const int e = threadIdx.x % pm::MAX_E;
+  const int q = threadIdx.x / pm::MAX_E;  // quarter of the chunk range
+  const int per = (nchunks + 3) / 4;
+  const int c0 = q * per, c1 = min(nchunks, c0 + per);
   int run = 0;
   if (e < E) {
-    for (int c = 0; c < nchunks; ++c) {
-      const int v = scratch[e * nchunks + c];
-      scratch[e * nchunks + c] = run;
+    int c = c0;
+    for (; c + 4 <= c1; c += 4) {  // four independent loads in flight
+      const int v0 = scratch[(c + 0) * E + e], v1 = scratch[(c + 1) * E + e];
+      const int v2 = scratch[(c + 2) * E + e], v3 = scratch[(c + 3) * E + e];
+      scratch[(c + 0) * E + e] = run;
+      scratch[(c + 1) * E + e] = run + v0;
+      scratch[(c + 2) * E + e] = run + v0 + v1;
+      scratch[(c + 3) * E + e] = run + v0 + v1 + v2;
+      run += v0 + v1 + v2 + v3;
+    }
+    for (; c < c1; ++c) {
+      const int v = scratch[c * E + e];
+      scratch[c * E + e] = run;
       run += v;
     }
   }
-  tot[e] = e < E ? run : 0;
-  scan[e] = tot[e];
+  part_sum[q][e] = e < E ? run : 0;
   __syncthreads();
-  for (int d = 1; d < pm::MAX_E; d <<= 1) {  // inclusive Hillis-Steele scan
-    const int v = e >= d ? scan[e - d] : 0;
+  if (q == 0) scan[e] = part_sum[0][e] + part_sum[1][e] + part_sum[2][e] + part_sum[3][e];
+  __syncthreads();
+  const int tot = scan[e];
+  for (int d = 1; d < pm::MAX_E; d <<= 1) {  // inclusive Hillis-Steele scan over experts
+    const int v = (q == 0 && e >= d) ? scan[e - d] : 0;
     __syncthreads();
-    scan[e] += v;
+    if (q == 0) scan[e] += v;
     __syncthreads();
   }
-  const int excl = scan[e] - tot[e];
+  const int excl = scan[e] - tot;
   if (e < E) {
-    counts[e] = tot[e];
-    offsets[e] = excl;
-    for (int c = 0; c < nchunks; ++c) scratch[e * nchunks + c] += excl;
+    int before = excl;  // first destination of this quarter
+    for (int qq = 0; qq < q; ++qq) before += part_sum[qq][e];
+    for (int c = c0; c < c1; ++c) scratch[c * E + e] += before;
+    if (q == 0) {
+      counts[e] = tot;
+      offsets[e] = excl;
+    }
   }
-  if (e == 0) {
+  if (threadIdx.x == 0) {
     const int routed = scan[pm::MAX_E - 1];
     counts[E] = has_shared ? T : 0;
     offsets[E] = routed;
@@ -96,7 +118,7 @@ __global__ void __launch_bounds__(pm::THREADS)
   __shared__ int wcnt[pm::WARPS][pm::MAX_E];
   const int c = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < E; e += pm::THREADS) cursor[e] = scratch[e * nchunks + c];
+  for (int e = tid; e < E; e += pm::THREADS) cursor[e] = scratch[c * E + e];
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int r = 0; r < pm::CHUNK / pm::THREADS; ++r) {
     for (int k = tid; k < pm::WARPS * pm::MAX_E; k += pm::THREADS) (&wcnt[0][0])[k] = 0;
@@ -135,8 +157,8 @@ cudaError_t launch_permute(const int32_t *idx, int T, int E, int K, int has_shar
   const int n = T * K;
   const int nchunks = permute_num_chunks(n);
   permute_hist_kernel<<<nchunks, pm::THREADS, 0, stream>>>(idx, n, E, nchunks, scratch, err);
-  permute_scan_kernel<<<1, pm::THREADS, 0, stream>>>(scratch, E, nchunks, T, has_shared, counts,
-                                                     offsets);
+  permute_scan_kernel<<<1, pm::SCAN_THREADS, 0, stream>>>(scratch, E, nchunks, T, has_shared, counts,
+                                                          offsets);
   permute_scatter_kernel<<<nchunks, pm::THREADS, 0, stream>>>(idx, n, E, nchunks, scratch, T,
                                                               has_shared, offsets, sorted);
   return cudaGetLastError();

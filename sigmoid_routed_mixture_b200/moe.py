@@ -46,6 +46,7 @@ STATUS = {
     5: "MOE_ERR_BAD_INDEX",
     6: "MOE_ERR_TIMEOUT",
     7: "MOE_ERR_CUDA",
+    8: "MOE_ERR_RANGE",
 }
 
 

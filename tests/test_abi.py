@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in range(8):
+    for code in range(9):
         s = L.moe_status_string(code)
         assert isinstance(s, bytes) and len(s) > 0
     assert L.moe_status_string(0) == b"ok"

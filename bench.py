@@ -35,7 +35,7 @@ from sigmoid_routed_mixture_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-block tokens/s (GLM-5 shape, bf16, 1 B200)"
 UNIT = "tokens/s"
-KERNELS_PER_STEP = 11  # route 3 + permute 3 + row gather 2 + up 1 + down 1 + combine 1
+KERNELS_PER_STEP = 11  # route 3 + permute 3 + token gather 2 + up 1 + down 1 + combine 1
 
 
 def peaks():
@@ -264,15 +264,18 @@ def main():
         moe.permute(cfg, blk.idx, blk.ws, out=(blk.counts, blk.offsets, blk.sorted))
         if ev is not None:
             ev[2].record(stream)
-        moe.expert_up(cfg, blk.weights, x_dev, blk.offsets, blk.sorted, blk.ws)
+        moe.gather_tokens(cfg, x_dev, blk.sorted, blk.ws)
         if ev is not None:
             ev[3].record(stream)
-        moe.expert_down(cfg, blk.weights, blk.gate, blk.offsets, blk.sorted, blk.ws)
+        moe.expert_up(cfg, blk.weights, blk.offsets, blk.sorted, blk.ws)
         if ev is not None:
             ev[4].record(stream)
-        moe.combine(cfg, blk.ws, blk.y)
+        moe.expert_down(cfg, blk.weights, blk.gate, blk.offsets, blk.sorted, blk.ws)
         if ev is not None:
             ev[5].record(stream)
+        moe.combine(cfg, blk.ws, blk.y)
+        if ev is not None:
+            ev[6].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -280,7 +283,7 @@ def main():
     if moe.device_error(blk.ws) != 0:
         raise RuntimeError("device error during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(torch.cuda.current_device())
@@ -298,7 +301,7 @@ def main():
     if dist is not None:
         dist.barrier()
     total_ms = e_start.elapsed_time(e_end)
-    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)]
+    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(6)]
                          for i in range(args.steps)])
     t_max = total_ms
     if dist is not None:
@@ -345,16 +348,20 @@ def main():
     f_router = 2.0 * w.T * H * w.E
     f_up = 2.0 * rows * H * 2 * I
     f_down = 2.0 * rows * I * H
+    # algorithmic bytes: weights of the touched groups plus the block's own
+    # input (x) or output (y); intermediates (gathered rows, h, slot outputs)
+    # are implementation choices and are not counted
     b_up = touched * 2 * I * H * 2 + w.T * H * 2
     b_down = touched * H * I * 2 + w.T * H * 2
     pk = peaks()
     mean_stage = stage_ms.mean(axis=0)
-    names = ["route", "permute", "expert_up", "expert_down", "combine"]
+    names = ["route", "permute", "gather_tokens", "expert_up", "expert_down", "combine"]
     dom = int(np.argmax(mean_stage))
     ridge = pk["tflops"] * 1e12 / (pk["hbm"] * 1e9)
     work = {"expert_up": (f_up, b_up), "expert_down": (f_down, b_down),
             "route": (f_router, w.T * H * 2 + w.E * H * 4 + w.T * w.K * 8),
             "permute": (0.0, w.T * w.K * 4 * 3 + rows * 4),
+            "gather_tokens": (0.0, w.T * H * 2 + rows * H * 2),
             "combine": (0.0, rows * H * 2 + w.T * H * 2)}
     f, by = work[names[dom]]
     dur_s = mean_stage[dom] / 1e3

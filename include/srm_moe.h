@@ -145,18 +145,23 @@ moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *weights, con
                          const float *topk_gate, const int32_t *offsets, const int32_t *sorted,
                          void *y, void *ws, size_t ws_bytes, void *stream);
 
-/* The three stages moe_forward runs, in this order, exposed separately so a
+/* The four stages moe_forward runs, in this order, exposed separately so a
  * caller can time or overlap them.  They communicate through the workspace
- * (intermediate h and the per-slot outputs), so the same ws, cfg, offsets and
- * sorted must be used for all three.
+ * (token rows in expert-sorted order, the intermediate h and the per-slot
+ * outputs), so the same ws, cfg, offsets and sorted must be used for all four.
  *
- * moe_expert_up: for every group g and its rows (expert-sorted: the token rows
- *   are first copied into that order in the workspace, each row of x read
- *   once), h = silu(x W1_g) (.) (x W3_g)  ("GLM-5 . MoE
- *   transformer block", Mixture of experts: g = x W1, u = x W3,
- *   a = g sigmoid(g), h = a (.) u); h is kept in fp16 in the workspace
- *   (magnitudes above 65504 saturate). */
-moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights, const void *x,
+ * moe_gather_tokens: copies the token rows of x into expert-sorted order in
+ *   the workspace (row p = x of the token of sorted[p]; each row of x is read
+ *   once and written to its K + 1 positions).  x: bf16 [T][H]. */
+moe_status_t moe_gather_tokens(const moe_cfg_t *cfg, const void *x, const int32_t *sorted, void *ws,
+                               size_t ws_bytes, void *stream);
+
+/* moe_expert_up: for every group g and its rows (the gathered token rows),
+ *   h = silu(x W1_g) (.) (x W3_g)  ("GLM-5 . MoE transformer block", Mixture
+ *   of experts: g = x W1, u = x W3, a = g sigmoid(g), h = a (.) u); h is kept
+ *   in fp16 in the workspace (magnitudes above 65504 saturate and are flagged
+ *   MOE_ERR_RANGE).  Needs moe_gather_tokens first. */
+moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights,
                            const int32_t *offsets, const int32_t *sorted, void *ws, size_t ws_bytes,
                            void *stream);
 

@@ -245,16 +245,31 @@ GemmArgs gemm_args(const moe_cfg_t &c, const int32_t *offsets, const int32_t *so
 
 }  // namespace
 
-moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights, const void *x,
+moe_status_t moe_gather_tokens(const moe_cfg_t *cfg, const void *x, const int32_t *sorted, void *ws,
+                               size_t ws_bytes, void *stream) {
+  WsLayout L;
+  moe_status_t st = check_stage(cfg, ws, ws_bytes, &L);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !sorted) return MOE_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(sorted, 4)) return MOE_ERR_ALIGN;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  return cuda_status(srm::launch_gather_rows(
+      static_cast<const uint16_t *>(x), sorted, static_cast<int>(cfg->T), cfg->H, cfg->K,
+      cfg->has_shared, reinterpret_cast<int32_t *>(wsb + L.pos),
+      reinterpret_cast<uint16_t *>(wsb + L.xs), reinterpret_cast<int *>(wsb + L.err), num_sms(),
+      static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights,
                            const int32_t *offsets, const int32_t *sorted, void *ws, size_t ws_bytes,
                            void *stream) {
   WsLayout L;
   moe_status_t st = check_stage(cfg, ws, ws_bytes, &L);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
-  if (!weights || !weights->w13 || !x || !offsets || !sorted) return MOE_ERR_ARG;
-  if (!aligned(weights->w13, 16) || !aligned(x, 16) || !aligned(offsets, 4) || !aligned(sorted, 4))
-    return MOE_ERR_ALIGN;
+  if (!weights || !weights->w13 || !offsets || !sorted) return MOE_ERR_ARG;
+  if (!aligned(weights->w13, 16) || !aligned(offsets, 4) || !aligned(sorted, 4)) return MOE_ERR_ALIGN;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   const int H = cfg->H, I = cfg->I, E = cfg->E;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -263,11 +278,6 @@ moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights, c
   if (!make_tmap(&tm_x, wsb + L.xs, H, static_cast<uint64_t>(rows_y(*cfg)), 64, 128) ||
       !make_tmap(&tm_w13, weights->w13, H, static_cast<uint64_t>(E + 1) * 2 * I, 64,
                  static_cast<uint32_t>(srm::gemm_b_box_rows(pair))))
-    return MOE_ERR_CUDA;
-  if (srm::launch_gather_rows(static_cast<const uint16_t *>(x), sorted, static_cast<int>(cfg->T), H,
-                              cfg->K, cfg->has_shared, reinterpret_cast<int32_t *>(wsb + L.pos),
-                              reinterpret_cast<uint16_t *>(wsb + L.xs),
-                              reinterpret_cast<int *>(wsb + L.err), num_sms(), s) != cudaSuccess)
     return MOE_ERR_CUDA;
   GemmArgs p = gemm_args(*cfg, offsets, sorted, nullptr, wsb, L);
   p.out = wsb + L.h;
@@ -329,7 +339,9 @@ moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *weights, con
   if (!weights || !weights->w13 || !weights->w2 || !x || !topk_gate || !offsets || !sorted || !y ||
       !ws)
     return MOE_ERR_ARG;
-  st = moe_expert_up(cfg, weights, x, offsets, sorted, ws, ws_bytes, stream);
+  st = moe_gather_tokens(cfg, x, sorted, ws, ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  st = moe_expert_up(cfg, weights, offsets, sorted, ws, ws_bytes, stream);
   if (st != MOE_OK) return st;
   st = moe_expert_down(cfg, weights, topk_gate, offsets, sorted, ws, ws_bytes, stream);
   if (st != MOE_OK) return st;

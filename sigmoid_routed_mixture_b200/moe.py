@@ -29,6 +29,7 @@ SYMBOLS = (
     "moe_route",
     "moe_permute",
     "moe_forward",
+    "moe_gather_tokens",
     "moe_expert_up",
     "moe_expert_down",
     "moe_combine",
@@ -115,8 +116,10 @@ def lib():
         L.moe_permute.argtypes = [P(_Cfg), vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.moe_forward.restype = ctypes.c_int
         L.moe_forward.argtypes = [P(_Cfg), P(_Weights), vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.moe_gather_tokens.restype = ctypes.c_int
+        L.moe_gather_tokens.argtypes = [P(_Cfg), vp, vp, vp, ctypes.c_size_t, vp]
         L.moe_expert_up.restype = ctypes.c_int
-        L.moe_expert_up.argtypes = [P(_Cfg), P(_Weights), vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.moe_expert_up.argtypes = [P(_Cfg), P(_Weights), vp, vp, vp, ctypes.c_size_t, vp]
         L.moe_expert_down.restype = ctypes.c_int
         L.moe_expert_down.argtypes = [P(_Cfg), P(_Weights), vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.moe_combine.restype = ctypes.c_int
@@ -272,15 +275,22 @@ def _weights_struct(cfg, weights):
     return _Weights(w13.data_ptr(), w2p.data_ptr())
 
 
-def expert_up(cfg: Config, weights, x, offsets, sorted_, ws, stream=None):
-    """Stage 1 of forward: h = silu(x W1) * (x W3) per expert-sorted row, into ws."""
+def gather_tokens(cfg: Config, x, sorted_, ws, stream=None):
+    """Stage 1 of forward: token rows of x in expert-sorted order, into ws."""
+    _req(x, torch.bfloat16, (cfg.T, cfg.H), "x")
+    _check(lib().moe_gather_tokens(ctypes.byref(cfg.c()), _ptr(x), _ptr(sorted_), _ptr(ws), ws.numel(),
+                                   _stream(stream)), "moe_gather_tokens")
+
+
+def expert_up(cfg: Config, weights, offsets, sorted_, ws, stream=None):
+    """Stage 2 of forward: h = silu(x W1) * (x W3) per expert-sorted row, into ws."""
     W_ = _weights_struct(cfg, weights)
-    _check(lib().moe_expert_up(ctypes.byref(cfg.c()), ctypes.byref(W_), _ptr(x), _ptr(offsets),
-                               _ptr(sorted_), _ptr(ws), ws.numel(), _stream(stream)), "moe_expert_up")
+    _check(lib().moe_expert_up(ctypes.byref(cfg.c()), ctypes.byref(W_), _ptr(offsets), _ptr(sorted_),
+                               _ptr(ws), ws.numel(), _stream(stream)), "moe_expert_up")
 
 
 def expert_down(cfg: Config, weights, topk_gate, offsets, sorted_, ws, stream=None):
-    """Stage 2 of forward: gate * (h W2) per row, into its (token, slot) place in ws."""
+    """Stage 3 of forward: gate * (h W2) per row, into its (token, slot) place in ws."""
     W_ = _weights_struct(cfg, weights)
     _check(lib().moe_expert_down(ctypes.byref(cfg.c()), ctypes.byref(W_), _ptr(topk_gate),
                                  _ptr(offsets), _ptr(sorted_), _ptr(ws), ws.numel(), _stream(stream)),
@@ -288,7 +298,7 @@ def expert_down(cfg: Config, weights, topk_gate, offsets, sorted_, ws, stream=No
 
 
 def combine(cfg: Config, ws, y, stream=None):
-    """Stage 3 of forward: y = sum of slot outputs + shared output (bf16 [T, H])."""
+    """Stage 4 of forward: y = sum of slot outputs + shared output (bf16 [T, H])."""
     _check(lib().moe_combine(ctypes.byref(cfg.c()), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_combine")
     return y

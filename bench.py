@@ -67,7 +67,7 @@ class ClockSampler:
             gpu = ids.split(",")[self.dev] if ids else str(self.dev)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "--query-gpu=" + CLOCK_FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", gpu], stdout=self.tmp, stderr=subprocess.DEVNULL)
+                 "-lms", "100", "-i", gpu], stdout=self.tmp, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
@@ -206,7 +206,7 @@ def workload_config(w, args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="glm5_prefill", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -58,6 +58,8 @@ WORKLOADS = {
     # GLM-5 expert shapes with 32 experts: 2.5 GB of weights, small enough for
     # multi-pass profiler captures, still far larger than the 126 MB L2
     "glm5_e32": Workload("glm5_e32", T=8192, H=6144, I=2048, E=32, K=8, scale=2.5, seed=1005),
+    "glm5_decode_e32": Workload("glm5_decode_e32", T=64, H=6144, I=2048, E=32, K=8, scale=2.5,
+                                seed=1006),
 }
 
 

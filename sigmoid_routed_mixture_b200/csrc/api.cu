@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -240,6 +241,7 @@ GemmArgs gemm_args(const moe_cfg_t &c, const int32_t *offsets, const int32_t *so
   p.tk = static_cast<int>(c.T * c.K);
   p.n_rows_y = static_cast<int>(rows_y(c));
   p.groups = c.E + c.has_shared;
+  p.stall = 0;
   return p;
 }
 
@@ -280,6 +282,11 @@ moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights,
                  static_cast<uint32_t>(srm::gemm_b_box_rows(pair))))
     return MOE_ERR_CUDA;
   GemmArgs p = gemm_args(*cfg, offsets, sorted, nullptr, wsb, L);
+  // Failure-detection tests set SRM_MOE_INJECT_STALL=1: the up projection's
+  // producer then loads nothing, its MMA warp's bounded wait runs out, and the
+  // call reports MOE_ERR_TIMEOUT through the workspace error word.
+  const char *inject = getenv("SRM_MOE_INJECT_STALL");
+  p.stall = (inject && inject[0] == '1') ? 1 : 0;
   p.out = wsb + L.h;
   p.n_total = 2 * I;
   p.k_total = H;

@@ -34,10 +34,9 @@
 //   warp 0: TMA producer (one lane issues the CTA's A and B tile loads)
 //   warp 1: tensor-memory allocation; in the leader also single-thread MMA issue
 //   warps 2-5: epilogue (tensor memory -> registers -> global)
-// Work tiles are (group, 256-row block, 256-column block), column block
-// fastest, dealt round-robin over the persistent CTA pairs; the per-group
-// row-block counts come from the group offsets on the device, so the host
-// never synchronises.
+// Work tiles are (group, 256-column block, row block), row block fastest,
+// dealt round-robin over the persistent units; the per-group row-block counts
+// come from the group offsets on the device, so the host never synchronises.
 //
 // Barrier protocol of a pair (no TMA multicast anywhere):
 //   full[s]   (leader's)  producer of the leader arms it with both CTAs' bytes;
@@ -104,22 +103,30 @@ struct TileCoord {
   int n0;         // first output column
 };
 
+// Tiles of group g occupy [tile_start[g] * n_tiles, tile_start[g+1] * n_tiles)
+// and inside a group the row block runs fastest: the units working at the same
+// moment share each 256-column weight tile (one DRAM read serves all the
+// group's row blocks) instead of spreading over many weight tiles that evict
+// one another from L2.
 template <bool kPair>
 __device__ __forceinline__ TileCoord decode_tile(const gg::Smem &s, int groups, int n_tiles,
                                                  int tile, int rank) {
-  const int mt = tile / n_tiles;
-  const int nt = tile - mt * n_tiles;
-  int lo = 0, hi = groups - 1;  // last g with tile_start[g] <= mt
+  const int mt_flat = tile / n_tiles;
+  int lo = 0, hi = groups - 1;  // last g with tile_start[g] <= mt_flat
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (s.tile_start[mid] <= mt)
+    if (s.tile_start[mid] <= mt_flat)
       lo = mid;
     else
       hi = mid - 1;
   }
+  const int mblocks = s.tile_start[lo + 1] - s.tile_start[lo];
+  const int local = tile - s.tile_start[lo] * n_tiles;
+  const int nt = local / mblocks;
+  const int mt = local - nt * mblocks;
   TileCoord c;
   c.g = lo;
-  c.row_base = s.grp_off[lo] + (mt - s.tile_start[lo]) * gg::Cfg<kPair>::TILE_M + rank * gg::BM;
+  c.row_base = s.grp_off[lo] + mt * gg::Cfg<kPair>::TILE_M + rank * gg::BM;
   c.rows = max(0, min(gg::BM, s.grp_off[lo + 1] - c.row_base));
   c.n0 = nt * gg::BN;
   return c;
@@ -222,7 +229,7 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     uint32_t stage = 0, phase = 0;
-    for (int tile = pair; tile < total_tiles; tile += num_pairs) {
+    for (int tile = pair; tile < total_tiles && !p.stall; tile += num_pairs) {
       const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, tile, rank);
       const int b_row = c.g * p.n_total + c.n0 + rank * C::B_ROWS;
       bool ok = true;

@@ -167,3 +167,24 @@ def test_out_of_range_expert_id_is_flagged():
     moe.permute(cfg, idx, ws)
     assert moe.device_error(ws) == 5
     assert moe.device_error(ws) == 0  # read clears it
+
+
+def test_timeout_is_reported_and_context_survives(monkeypatch):
+    """Failure detection without a GPU fault: with SRM_MOE_INJECT_STALL=1 the up
+    projection's producer issues no loads, so the MMA warp waits on a barrier
+    nothing arms; the wait gives up after its 2 s limit, the kernel returns and
+    the host reads MOE_ERR_TIMEOUT.  The next call on the same context is normal."""
+    w = W.WORKLOADS["tiny"].replace(T=200, seed=2800)
+    case = MH.Case(w)
+    blk = case.block()
+    moe.route(case.cfg, case.x_dev, blk.w_router, blk.bias, blk.ws, out=(blk.idx, blk.gate, blk.margin))
+    moe.permute(case.cfg, blk.idx, blk.ws, out=(blk.counts, blk.offsets, blk.sorted))
+    moe.gather_tokens(case.cfg, case.x_dev, blk.sorted, blk.ws)
+    monkeypatch.setenv("SRM_MOE_INJECT_STALL", "1")
+    moe.expert_up(case.cfg, blk.weights, blk.offsets, blk.sorted, blk.ws)
+    torch.cuda.synchronize()
+    assert moe.device_error(blk.ws) == 6  # MOE_ERR_TIMEOUT
+    monkeypatch.delenv("SRM_MOE_INJECT_STALL")
+    res = case.run()
+    assert res["err"] == 0
+    MH.check_forward(case, res, np.arange(w.T))

@@ -241,6 +241,7 @@ GemmArgs gemm_args(const moe_cfg_t &c, const int32_t *offsets, const int32_t *so
   p.tk = static_cast<int>(c.T * c.K);
   p.n_rows_y = static_cast<int>(rows_y(c));
   p.groups = c.E + c.has_shared;
+  p.tile_counter = reinterpret_cast<int *>(wsb + L.err + 128);
   p.stall = 0;
   return p;
 }
@@ -291,6 +292,7 @@ moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights,
   p.n_total = 2 * I;
   p.k_total = H;
   p.out_ld = I;
+  if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
   return cuda_status(srm::launch_grouped_gemm(srm::kUp, pair, tm_x, tm_w13, p, num_sms(), s));
 }
 
@@ -319,6 +321,8 @@ moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
   p.n_total = H;
   p.k_total = I;
   p.out_ld = H;
+  if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return cuda_status(srm::launch_grouped_gemm(srm::kDown, pair, tm_h, tm_w2, p, num_sms(),
                                               static_cast<cudaStream_t>(stream)));
 }

@@ -92,17 +92,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
   return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity of `bar` has completed.
 // Returns false (and stops waiting) when the CTA's abort flag is raised or the
 // time limit runs out; in the latter case records MOE_ERR_TIMEOUT and raises
 // the abort flag.
+// With cluster_scope the wait also acquires what other CTAs of the cluster
+// released before arriving (stores into this CTA's shared memory).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          int *err) {
+                                          int *err, bool cluster_scope = false) {
   const uint32_t a = smem_addr(bar);
-  if (mbar_try_wait(a, parity)) return true;
+  auto poll = [&]() {
+    return cluster_scope ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity);
+  };
+  if (poll()) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(a, parity)) return true;
+    if (poll()) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
@@ -235,6 +252,11 @@ __device__ __forceinline__ uint32_t cluster_map(const void *p, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
+}
+
+// Store a 32-bit value into another CTA's shared memory (shared::cluster address).
+__device__ __forceinline__ void st_shared_remote(uint32_t cluster_addr, int32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 // Arrive on an mbarrier in another CTA of the cluster (shared::cluster address).

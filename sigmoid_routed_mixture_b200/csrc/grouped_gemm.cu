@@ -34,9 +34,11 @@
 //   warp 0: TMA producer (one lane issues the CTA's A and B tile loads)
 //   warp 1: tensor-memory allocation; in the leader also single-thread MMA issue
 //   warps 2-5: epilogue (tensor memory -> registers -> global)
-// Work tiles are (group, 256-column block, row block), row block fastest,
-// dealt round-robin over the persistent units; the per-group row-block counts
-// come from the group offsets on the device, so the host never synchronises.
+// Work tiles are (group, 256-column block, row block), row block fastest; a
+// unit (CTA pair or single CTA) takes its next tile from a global atomic
+// counter when it is ready for one, so tiles that share a weight tile start
+// together; the per-group row-block counts come from the group offsets on the
+// device, so the host never synchronises.
 //
 // Barrier protocol of a pair (no TMA multicast anywhere):
 //   full[s]   (leader's)  producer of the leader arms it with both CTAs' bytes;
@@ -47,6 +49,9 @@
 //                         accumulator a is complete
 //   tempty[a] (leader's)  the 4 epilogue warps of each CTA arrive (8 in all)
 //                         when they have drained accumulator a
+//   tile_full[i] (each)   the leader's producer publishes tile id i (ring of 4)
+//                         into both CTAs' shared memory and arrives on both
+//   tile_empty[i] (leader's) the epilogue warps of both CTAs release ring slot i
 #include <cuda.h>
 
 #include "common.cuh"
@@ -62,6 +67,7 @@ constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
 constexpr int MAX_GROUPS = 257;
 constexpr int MAX_STAGES = 6;
+constexpr int TILE_RING = 4;  // tile ids in flight between the scheduler and the roles
 
 // kPair: a CTA pair shares each 256-row tile (M = 256, each CTA loads half of
 // B); solo: one CTA per 128-row tile (M = 128, the CTA loads all of B).
@@ -80,6 +86,9 @@ struct Cfg {
 struct Smem {
   uint64_t full[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
+  uint64_t tile_full[TILE_RING];
+  uint64_t tile_empty[TILE_RING];
+  int tile_ring[TILE_RING];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -152,9 +161,6 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
   const int lane = threadIdx.x & 31;
   const uint32_t rank = kPair ? cluster_ctarank() : 0;
   const bool leader = rank == 0;
-  // a "unit" is a CTA pair (kPair) or a single CTA
-  const int pair = kPair ? (blockIdx.x >> 1) : blockIdx.x;
-  const int num_pairs = kPair ? (gridDim.x >> 1) : gridDim.x;
   const int groups = p.groups;
   const int n_tiles = p.n_total / BN;
   const int kblocks = p.k_total / BK;
@@ -170,6 +176,10 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.tfull[i], 1);
       mbar_init(&s.tempty[i], C::EPI_ARRIVALS);
+    }
+    for (int i = 0; i < TILE_RING; ++i) {
+      mbar_init(&s.tile_full[i], 1);
+      mbar_init(&s.tile_empty[i], C::EPI_ARRIVALS);
     }
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
@@ -228,8 +238,34 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    uint32_t stage = 0, phase = 0;
-    for (int tile = pair; tile < total_tiles && !p.stall; tile += num_pairs) {
+    // The leader's producer is also the tile scheduler: it takes the next
+    // tile from the global counter, so tiles sharing a weight tile (one
+    // group's row blocks) start at nearly the same moment on whichever units
+    // are free, and publishes the id to its own CTA and to the peer through
+    // the tile ring.
+    uint32_t stage = 0, phase = 0, ts = 0, tph = 0;
+    while (true) {
+      if (leader) {
+        if (!mbar_wait(&s.tile_empty[ts], tph ^ 1u, abort_flag, p.err)) break;
+        if (lane == 0) {
+          int t = atomicAdd(p.tile_counter, 1);
+          if (t >= total_tiles) t = -1;
+          s.tile_ring[ts] = t;
+          mbar_arrive(&s.tile_full[ts]);
+          if (kPair) {
+            st_shared_remote(cluster_map(&s.tile_ring[ts], 1), t);
+            mbar_arrive_remote(cluster_map(&s.tile_full[ts], 1));
+          }
+        }
+        __syncwarp();
+      }
+      if (!mbar_wait(&s.tile_full[ts], tph, abort_flag, p.err, kPair)) break;
+      const int tile = *reinterpret_cast<volatile int *>(&s.tile_ring[ts]);
+      if (++ts == TILE_RING) {
+        ts = 0;
+        tph ^= 1u;
+      }
+      if (tile < 0 || p.stall) break;
       const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, tile, rank);
       const int b_row = c.g * p.n_total + c.n0 + rank * C::B_ROWS;
       bool ok = true;
@@ -261,9 +297,16 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
     if (leader) {
-      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0, ts = 0, tph = 0;
       int consumed = 0;
-      for (int tile = pair; tile < total_tiles; tile += num_pairs) {
+      while (true) {
+        if (!mbar_wait(&s.tile_full[ts], tph, abort_flag, p.err)) break;
+        const int tile = *reinterpret_cast<volatile int *>(&s.tile_ring[ts]);
+        if (++ts == TILE_RING) {
+          ts = 0;
+          tph ^= 1u;
+        }
+        if (tile < 0) break;
         if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag, p.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
@@ -315,8 +358,16 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // tensor-memory lane quarter this warp may access
     const int row = q * 32 + lane;
-    uint32_t acc = 0, acc_phase = 0;
-    for (int tile = pair; tile < total_tiles; tile += num_pairs) {
+    uint32_t acc = 0, acc_phase = 0, ts = 0, tph = 0;
+    while (true) {
+      if (!mbar_wait(&s.tile_full[ts], tph, abort_flag, p.err, kPair)) break;
+      const int tile = *reinterpret_cast<volatile int *>(&s.tile_ring[ts]);
+      const uint32_t slot = ts;
+      if (++ts == TILE_RING) {
+        ts = 0;
+        tph ^= 1u;
+      }
+      if (tile < 0) break;
       const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, tile, rank);
       if (!mbar_wait(&s.tfull[acc], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
@@ -378,10 +429,15 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (leader)
+        // the accumulator is drained and, past tfull, every reader of this tile
+        // id (both producers, the MMA warp) has read it: free both
+        if (leader) {
           mbar_arrive(&s.tempty[acc]);
-        else
+          mbar_arrive(&s.tile_empty[slot]);
+        } else {
           mbar_arrive_remote(cluster_map(&s.tempty[acc], 0));
+          mbar_arrive_remote(cluster_map(&s.tile_empty[slot], 0));
+        }
       }
       acc ^= 1u;
       if (acc == 0) acc_phase ^= 1u;

@@ -26,6 +26,7 @@ struct GemmArgs {
   int n_total;             // output columns per group (2I for kUp, H for kDown)
   int k_total;             // reduction length (H for kUp, I for kDown)
   int out_ld;              // elements per output row (I for kUp, H for kDown)
+  int *tile_counter;       // zeroed before the launch; units take their next tile from it
   int stall;               // failure-detection tests only: the producer issues no loads, so
                            // the MMA warp's bounded wait runs out (MOE_ERR_TIMEOUT)
 };

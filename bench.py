@@ -144,6 +144,25 @@ def cores():
     return len(os.sched_getaffinity(0))
 
 
+def measured_traffic(workload, kernel):
+    """DRAM bytes per launch from a committed ncu capture (profiles/dram_traffic_glm5.md),
+    or None when the GEMM sources changed since it was taken."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "dram_traffic_glm5.md")
+    if not os.path.exists(path):
+        return None
+    h = hashlib.md5()
+    for f in ("grouped_gemm.cu", "common.cuh", "kernels.h"):
+        h.update(open(os.path.join(ROOT, "sigmoid_routed_mixture_b200", "csrc", f), "rb").read())
+    for line in open(path):
+        parts = line.split()
+        if len(parts) == 5 and parts[0] == "traffic" and parts[1] == workload and parts[2] == kernel:
+            if parts[4] == "src=" + h.hexdigest():
+                return float(parts[3])
+    return None
+
+
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, rank):
@@ -372,7 +391,7 @@ def main():
         roof = {"kernel": names[dom], "bound": "hbm", "achieved": by / dur_s / 1e9, "peak": pk["hbm"],
                 "unit": "GB/s", "peak_kind": "copy bandwidth, " + pk["source"]}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = measured_traffic(w.name, names[dom])
     roof["algorithmic_per_launch"] = f if roof["bound"] == "tensor" else by
     f_alg = f_router + f_up + f_down
     b_alg = touched * 3 * H * I * 2 + w.E * H * 4 + w.E * 4 + 2 * w.T * H * 2

@@ -211,6 +211,36 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ replicas (N > 1)
+
+def replica_tokens(w, rank):
+    """Token batch of replica `rank`: the workload's own x on rank 0, an
+    independently seeded batch of the same shape on the others."""
+    x, w_r, b = W.router_inputs(w)
+    if rank > 0:
+        rng = np.random.default_rng([w.seed, rank])
+        x = W.f32_to_bf16_bits(rng.standard_normal(x.shape, dtype=np.float32))
+        if w.skew:
+            x[:, 0] = W.f32_to_bf16_bits(np.ones((w.T,), dtype=np.float32))
+    return x, w_r, b
+
+
+def max_over_ranks(ms, dist, device):
+    """The slowest replica's device time (every rank takes the same collective)."""
+    if dist is None:
+        return ms
+    import torch
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tokens_per_s(tokens_per_rank, world, steps, t_max_ms):
+    """Whole-job throughput: tokens of all replicas over the slowest replica's time."""
+    return tokens_per_rank * world * steps / (t_max_ms / 1e3)
+
+
 def workload_config(w, args):
     return {"workload": w.name, "tokens": w.T, "hidden": w.H, "expert_intermediate": w.I,
             "routed_experts": w.E, "top_k": w.K, "shared_experts": int(w.has_shared),
@@ -260,12 +290,7 @@ def main():
     w = W.WORKLOADS[args.workload]
     dev = torch.device("cuda", torch.cuda.current_device())
     # each replica draws its own token batch; weights are the workload's
-    x, w_r, b = W.router_inputs(w)
-    if rank > 0:
-        rng = np.random.default_rng([w.seed, rank])
-        x = W.f32_to_bf16_bits(rng.standard_normal(x.shape, dtype=np.float32))
-        if w.skew:
-            x[:, 0] = W.f32_to_bf16_bits(np.ones((w.T,), dtype=np.float32))
+    x, w_r, b = replica_tokens(w, rank)
     weights = W.expert_weights(w, dev)
     cfg = moe.Config.of(w)
     blk = moe.MoeBlock(cfg, torch.from_numpy(w_r).to(dev), torch.from_numpy(b).to(dev), **weights)
@@ -322,12 +347,8 @@ def main():
     total_ms = e_start.elapsed_time(e_end)
     stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(6)]
                          for i in range(args.steps)])
-    t_max = total_ms
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
-    value = w.T * world * args.steps / (t_max / 1e3)
+    t_max = max_over_ranks(total_ms, dist, dev)
+    value = aggregate_tokens_per_s(w.T, world, args.steps, t_max)
 
     # ---- end to end: pinned host x in, result out, every step
     x_host = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -350,12 +371,8 @@ def main():
         e2e_step()
     z.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(z)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = w.T * world * args.e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(a.elapsed_time(z), dist, dev)
+    e2e_value = aggregate_tokens_per_s(w.T, world, args.e2e_steps, e2e_ms)
     if moe.device_error(blk.ws) != 0:
         raise RuntimeError("device error during the timed steps")
 

@@ -1,0 +1,65 @@
+"""The N > 1 path of bench.py (independent replicas, no data-path collective)
+on CPU: two gloo ranks check the per-replica inputs, the max over ranks and
+the whole-job throughput; the reference arm under torchrun prints one line
+from rank 0 only."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    sys.path.insert(0, ROOT)
+    import bench
+    from sigmoid_routed_mixture_b200 import workloads as W
+
+    w = W.WORKLOADS["tiny"]
+    x, w_r, b = bench.replica_tokens(w, rank)
+    ms = 10.0 + 5.0 * rank  # rank 1 is the slower replica
+    t_max = bench.max_over_ranks(ms, dist, "cpu")
+    value = bench.aggregate_tokens_per_s(w.T, world, 7, t_max)
+    digest = torch.tensor([float(x.astype(np.float64).sum())])
+    gathered = [torch.zeros(1) for _ in range(world)]
+    dist.all_gather(gathered, digest)
+    out[rank] = (t_max, value, [float(g) for g in gathered], float(w_r.sum()))
+    dist.destroy_process_group()
+
+
+def test_two_replicas_with_gloo():
+    world = 2
+    out = mp.Manager().dict()
+    mp.spawn(_rank_main, args=(world, free_port(), out), nprocs=world, join=True)
+    (t0, v0, d0, r0), (t1, v1, d1, r1) = out[0], out[1]
+    assert t0 == t1 == 15.0                      # every rank sees the slowest replica
+    assert v0 == v1 == pytest.approx(64 * 2 * 7 / 0.015)
+    assert d0[0] != d0[1]                        # replicas draw different token batches
+    assert r0 == r1                              # ... with the same router weights
+
+
+def test_reference_arm_under_torchrun_prints_one_line():
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--workload", "tiny", "--gpus", "2", "--steps", "1", "--warmup", "3",
+           "--ref-tokens", "4"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2 and lines[0]["value"] > 0

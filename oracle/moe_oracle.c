@@ -59,6 +59,28 @@ static double bf16_to_double(uint16_t v)
 
 static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
 
+/* Pre-FFN RMSNorm of the decoder block ("GLM-5 . MoE transformer block",
+ * "All 43 steps": x_ffn = RMSNorm(x'_n); rms_norm_eps from the config):
+ *   out[t,h] = x[t,h] * gamma[h] / sqrt(mean_h x[t,h]^2 + eps)
+ * in double from the exact bf16 inputs (x and gamma bf16 bit patterns). */
+int oracle_rmsnorm(int64_t T, int64_t H, const uint16_t *x, const uint16_t *gamma, double eps,
+                   double *out)
+{
+    if (T < 0 || H <= 0 || eps < 0 || (T > 0 && (!x || !gamma || !out))) return ORACLE_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double ss = 0.0;
+        for (int64_t h = 0; h < H; ++h) {
+            double v = bf16_to_double(x[t * H + h]);
+            ss += v * v;
+        }
+        double inv = 1.0 / sqrt(ss / (double)H + eps);
+        for (int64_t h = 0; h < H; ++h)
+            out[t * H + h] = bf16_to_double(x[t * H + h]) * inv * bf16_to_double(gamma[h]);
+    }
+    return ORACLE_OK;
+}
+
 /* Parameter count of one MoE block: router matrix E*H, selection bias E,
  * and (E + n_shared) SwiGLU experts of three H*I matrices each.
  * ("Parameters" table of the GLM-5 MoE transformer block page.) */

@@ -51,6 +51,8 @@ def _load():
         lib = ctypes.CDLL(build())
         lib.oracle_param_count.restype = _i64
         lib.oracle_param_count.argtypes = [_i64, _i64, _i64, _i64]
+        lib.oracle_rmsnorm.restype = _int
+        lib.oracle_rmsnorm.argtypes = [_i64, _i64, _vp, _vp, _dbl, _vp]
         lib.oracle_logits.restype = _int
         lib.oracle_logits.argtypes = [_i64, _i64, _i64, _vp, _vp, _vp]
         lib.oracle_select.restype = _int
@@ -86,6 +88,17 @@ def _bf16(a):
 def param_count(H: int, I: int, E: int, n_shared: int = 1) -> int:
     """Parameters of one MoE block: router E*H, bias E, (E+n_shared) experts of 3*H*I."""
     return int(_load().oracle_param_count(H, I, E, n_shared))
+
+
+def rmsnorm(x, gamma, eps: float):
+    """x_ffn = x * gamma / sqrt(mean(x^2) + eps) per row, in double (x, gamma bf16 bits)."""
+    x = _bf16(x)
+    gamma = _bf16(gamma)
+    T, H = x.shape
+    assert gamma.shape == (H,)
+    out = np.empty((T, H), dtype=np.float64)
+    _check(_load().oracle_rmsnorm(T, H, _p(x), _p(gamma), float(eps), _p(out)), "rmsnorm")
+    return out
 
 
 def logits(x, w_r):

@@ -323,3 +323,29 @@ def test_empty_token_batch():
     assert counts.sum() == 0 and srt.shape == (0,)
     y = O.forward(c["x"], c["w1"], c["w3"], c["w2"], c["ws1"], c["ws3"], c["ws2"], idx, gate)
     assert y.shape == (0, c["x"].shape[1])
+
+
+# ---------------------------------------------------------------- pre-FFN RMSNorm
+
+def test_rmsnorm_closed_forms():
+    """A row of one repeated value c has RMS |c|: out = sign(c) * gamma / sqrt(1 + eps / c^2).
+    A row (3, 4) has mean square 12.5."""
+    H = 8
+    gamma = bf([0.5, 1.0, 2.0, -1.0, 0.25, 4.0, 1.5, -0.75])
+    g = W.bf16_bits_to_f32(gamma).astype(np.float64)
+    x = bf([[3.0] * H, [-0.5] * H])
+    out = O.rmsnorm(x, gamma, 1e-5)
+    np.testing.assert_allclose(out[0], g / math.sqrt(1 + 1e-5 / 9.0), rtol=1e-15, atol=0)
+    np.testing.assert_allclose(out[1], -g / math.sqrt(1 + 1e-5 / 0.25), rtol=1e-15, atol=0)
+    out = O.rmsnorm(bf([[3.0, 4.0]]), bf([1.0, 1.0]), 0.0)
+    np.testing.assert_allclose(out[0], [3 / math.sqrt(12.5), 4 / math.sqrt(12.5)], rtol=1e-15)
+
+
+def test_rmsnorm_scale_invariance_and_unit_rms():
+    rng = np.random.default_rng(9)
+    x = W.f32_to_bf16_bits(rng.standard_normal((6, 64), dtype=np.float32))
+    ones = bf([1.0] * 64)
+    out = O.rmsnorm(x, ones, 0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(out ** 2, axis=1)), 1.0, rtol=1e-14)
+    x4 = W.f32_to_bf16_bits(W.bf16_bits_to_f32(x) * np.float32(4.0))  # exact: power of two
+    np.testing.assert_allclose(O.rmsnorm(x4, ones, 0.0), out, rtol=1e-14, atol=0)

@@ -202,6 +202,22 @@ moe_status_t moe_combine(const moe_cfg_t *cfg, void *y, void *ws, size_t ws_byte
 moe_status_t moe_permute_noalloc(const moe_cfg_t *cfg, const int32_t *topk_idx, int32_t *counts,
                                  int32_t *offsets, int32_t *sorted, void *stream);
 
+/* moe_combine followed by the block's residual add in the same pass
+ * ("GLM-5 . MoE transformer block", All 43 steps: x_{n+1} = x'_n + Delta_ffn):
+ *   y[t] = residual[t] + (sum of the K slot outputs, in order) + shared output,
+ * in fp32, rounded once to bf16.  residual: bf16 [T][H] (x'_n, the stream the
+ * pre-FFN RMSNorm read); NULL gives moe_combine. */
+moe_status_t moe_combine_residual(const moe_cfg_t *cfg, const void *residual, void *y, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/* The decoder block's pre-FFN RMSNorm (All 43 steps: x_ffn = RMSNorm(x'_n)):
+ *   x_ffn[t][h] = x[t][h] * gamma[h] / sqrt(mean_h x[t][h]^2 + eps)
+ * in fp32, rounded once to bf16.  x, x_ffn: bf16 [T][H]; gamma: bf16 [H] (the
+ * norm's weight); eps = rms_norm_eps (1e-5 in the GLM configs).  Only cfg->T
+ * and cfg->H are used (cfg must still be valid). */
+moe_status_t moe_rmsnorm(const moe_cfg_t *cfg, const void *x, const void *gamma, float eps,
+                         void *x_ffn, void *stream);
+
 /* Read (and clear) the device error word of a workspace.  Synchronises
  * `stream`.  *device_status receives MOE_OK or the first device-side error
  * recorded since the last read.  Returns MOE_ERR_CUDA if the copy fails. */

@@ -328,16 +328,37 @@ moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
 }
 
 moe_status_t moe_combine(const moe_cfg_t *cfg, void *y, void *ws, size_t ws_bytes, void *stream) {
+  return moe_combine_residual(cfg, nullptr, y, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_combine_residual(const moe_cfg_t *cfg, const void *residual, void *y, void *ws,
+                                  size_t ws_bytes, void *stream) {
   WsLayout L;
   moe_status_t st = check_stage(cfg, ws, ws_bytes, &L);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
   if (!y) return MOE_ERR_ARG;
-  if (!aligned(y, 16)) return MOE_ERR_ALIGN;
+  if (!aligned(y, 16) || (residual && !aligned(residual, 16))) return MOE_ERR_ALIGN;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   return cuda_status(srm::launch_combine(reinterpret_cast<const uint16_t *>(wsb + L.ybuf),
+                                         static_cast<const uint16_t *>(residual),
                                          static_cast<uint16_t *>(y), static_cast<int>(cfg->T),
                                          cfg->H, cfg->K, cfg->has_shared, num_sms(),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_rmsnorm(const moe_cfg_t *cfg, const void *x, const void *gamma, float eps,
+                         void *x_ffn, void *stream) {
+  moe_status_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!(eps >= 0.f) || !isfinite(eps)) return MOE_ERR_ARG;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !gamma || !x_ffn) return MOE_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(x_ffn, 16)) return MOE_ERR_ALIGN;
+  return cuda_status(srm::launch_rmsnorm(static_cast<const uint16_t *>(x),
+                                         static_cast<const uint16_t *>(gamma), eps,
+                                         static_cast<int>(cfg->T), cfg->H,
+                                         static_cast<uint16_t *>(x_ffn), num_sms(),
                                          static_cast<cudaStream_t>(stream)));
 }
 

@@ -5,7 +5,9 @@
 // T*K routed rows, the shared expert's output; "the shared expert runs after
 // the routed ones" (nnterp GLM-5 page, section 03) fixes the order of the
 // final addition, and Delta_ffn = y_routed + y_shared ("GLM-5 . MoE
-// transformer block", "All 43 steps").
+// transformer block", "All 43 steps").  With a residual row the kernel also
+// performs the block's x_{n+1} = x'_n + Delta_ffn in the same pass (one
+// rounding of the sum).
 //
 // Pure streaming: each thread owns 8 consecutive columns of one token, loads
 // K+1 16-byte vectors of fp16 and stores 16 bytes of bf16.
@@ -27,8 +29,8 @@ __device__ __forceinline__ void add8(float (&acc)[8], const uint16_t *src) {
 }
 
 __global__ void __launch_bounds__(256)
-    combine_kernel(const uint16_t *__restrict__ Y, uint16_t *__restrict__ y, int T, int H, int K,
-                   int has_shared) {
+    combine_kernel(const uint16_t *__restrict__ Y, const uint16_t *__restrict__ residual,
+                   uint16_t *__restrict__ y, int T, int H, int K, int has_shared) {
   const int vecs = H / 8;
   const int64_t total = static_cast<int64_t>(T) * vecs;
   const int64_t tk = static_cast<int64_t>(T) * K;
@@ -39,6 +41,15 @@ __global__ void __launch_bounds__(256)
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int k = 0; k < K; ++k) add8(acc, Y + (t * K + k) * H + col);
     if (has_shared) add8(acc, Y + (tk + t) * H + col);
+    if (residual) {  // x_{n+1} = x'_n + Delta_ffn: the block output added to the residual stream
+      const uint4 r = *reinterpret_cast<const uint4 *>(residual + t * H + col);
+      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc[2 * k] = __uint_as_float(w[k] << 16) + acc[2 * k];
+        acc[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u) + acc[2 * k + 1];
+      }
+    }
     uint4 o;
     o.x = pack_bf16x2(acc[0], acc[1]);
     o.y = pack_bf16x2(acc[2], acc[3]);
@@ -48,13 +59,13 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-cudaError_t launch_combine(const uint16_t *Y, uint16_t *y, int T, int H, int K, int has_shared,
-                           int num_sms, cudaStream_t stream) {
+cudaError_t launch_combine(const uint16_t *Y, const uint16_t *residual, uint16_t *y, int T, int H,
+                           int K, int has_shared, int num_sms, cudaStream_t stream) {
   const int64_t total = static_cast<int64_t>(T) * (H / 8);
   int64_t blocks = (total + 255) / 256;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   if (blocks > cap) blocks = cap;
-  combine_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(Y, y, T, H, K, has_shared);
+  combine_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(Y, residual, y, T, H, K, has_shared);
   return cudaGetLastError();
 }
 

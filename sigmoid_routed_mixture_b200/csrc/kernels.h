@@ -63,8 +63,12 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *sorted, int T, 
                                int has_shared, int32_t *pos, uint16_t *xs, int *err, int num_sms,
                                cudaStream_t stream);
 
-cudaError_t launch_combine(const uint16_t *Y, uint16_t *y, int T, int H, int K, int has_shared,
-                           int num_sms, cudaStream_t stream);
+// y = (residual +) sum of slot outputs + shared output; residual may be NULL
+cudaError_t launch_combine(const uint16_t *Y, const uint16_t *residual, uint16_t *y, int T, int H,
+                           int K, int has_shared, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_rmsnorm(const uint16_t *x, const uint16_t *gamma, float eps, int T, int H,
+                           uint16_t *out, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_pack(const uint16_t *w1, const uint16_t *w3, const uint16_t *w2,
                         const uint16_t *ws1, const uint16_t *ws3, const uint16_t *ws2, int H, int I,

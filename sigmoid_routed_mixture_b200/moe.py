@@ -33,6 +33,8 @@ SYMBOLS = (
     "moe_expert_up",
     "moe_expert_down",
     "moe_combine",
+    "moe_combine_residual",
+    "moe_rmsnorm",
     "moe_get_device_error",
     "moe_status_string",
     "moe_permute_noalloc",
@@ -124,6 +126,10 @@ def lib():
         L.moe_expert_down.argtypes = [P(_Cfg), P(_Weights), vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.moe_combine.restype = ctypes.c_int
         L.moe_combine.argtypes = [P(_Cfg), vp, vp, ctypes.c_size_t, vp]
+        L.moe_combine_residual.restype = ctypes.c_int
+        L.moe_combine_residual.argtypes = [P(_Cfg), vp, vp, vp, ctypes.c_size_t, vp]
+        L.moe_rmsnorm.restype = ctypes.c_int
+        L.moe_rmsnorm.argtypes = [P(_Cfg), vp, vp, ctypes.c_float, vp, vp]
         L.moe_get_device_error.restype = ctypes.c_int
         L.moe_get_device_error.argtypes = [vp, P(ctypes.c_int), vp]
         L.moe_permute_noalloc.restype = ctypes.c_int
@@ -304,6 +310,25 @@ def combine(cfg: Config, ws, y, stream=None):
     return y
 
 
+def combine_residual(cfg: Config, ws, residual, y, stream=None):
+    """Stage 4 with the residual add: y = residual + slot outputs + shared output."""
+    _req(residual, torch.bfloat16, (cfg.T, cfg.H), "residual")
+    _check(lib().moe_combine_residual(ctypes.byref(cfg.c()), _ptr(residual), _ptr(y), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "moe_combine_residual")
+    return y
+
+
+def rmsnorm(cfg: Config, x, gamma, eps=1e-5, out=None, stream=None):
+    """Pre-FFN RMSNorm: x * gamma / sqrt(mean(x^2) + eps) per row (bf16 in and out)."""
+    _req(x, torch.bfloat16, (cfg.T, cfg.H), "x")
+    _req(gamma, torch.bfloat16, (cfg.H,), "gamma")
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().moe_rmsnorm(ctypes.byref(cfg.c()), _ptr(x), _ptr(gamma), float(eps), _ptr(out),
+                             _stream(stream)), "moe_rmsnorm")
+    return out
+
+
 def device_error(ws, stream=None) -> int:
     """Read and clear the workspace's device error word (synchronises the stream)."""
     st = ctypes.c_int(0)
@@ -330,6 +355,19 @@ class MoeBlock:
         self.offsets = torch.empty((E + 2,), dtype=torch.int32, device=dev)
         self.sorted = torch.empty((cfg.rows,), dtype=torch.int32, device=dev)
         self.y = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
+
+    def sublayer(self, x_resid, gamma, eps=1e-5, stream=None, logits=None):
+        """The decoder block's FFN sublayer: x' + MoE(RMSNorm(x')) (bf16 [T, H])."""
+        cfg = self.cfg
+        x_ffn = rmsnorm(cfg, x_resid, gamma, eps, stream=stream)
+        route(cfg, x_ffn, self.w_router, self.bias, self.ws, out=(self.idx, self.gate, self.margin),
+              logits=logits, stream=stream)
+        permute(cfg, self.idx, self.ws, out=(self.counts, self.offsets, self.sorted), stream=stream)
+        gather_tokens(cfg, x_ffn, self.sorted, self.ws, stream=stream)
+        expert_up(cfg, self.weights, self.offsets, self.sorted, self.ws, stream=stream)
+        expert_down(cfg, self.weights, self.gate, self.offsets, self.sorted, self.ws, stream=stream)
+        combine_residual(cfg, self.ws, x_resid, self.y, stream=stream)
+        return self.y, x_ffn
 
     def __call__(self, x, stream=None, logits=None):
         route(self.cfg, x, self.w_router, self.bias, self.ws, out=(self.idx, self.gate, self.margin),

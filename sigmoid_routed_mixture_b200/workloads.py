@@ -89,6 +89,12 @@ def router_inputs(w: Workload):
     return x, w_r, b
 
 
+def norm_weight(w: Workload):
+    """Pre-FFN RMSNorm weight gamma [H] (bf16 bits): 1 + N(0, 0.1), seeded by (seed, 7)."""
+    rng = np.random.default_rng([w.seed, 7])
+    return f32_to_bf16_bits(1.0 + 0.1 * rng.standard_normal((w.H,), dtype=np.float32))
+
+
 def expert_weights(w: Workload, device="cpu"):
     """Expert weights as torch bf16 tensors on ``device``:
     dict(w1 [E,I,H], w3 [E,I,H], w2 [E,H,I], ws1 [I,H], ws3 [I,H], ws2 [H,I])."""

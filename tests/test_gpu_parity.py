@@ -188,3 +188,38 @@ def test_timeout_is_reported_and_context_survives(monkeypatch):
     res = case.run()
     assert res["err"] == 0
     MH.check_forward(case, res, np.arange(w.T))
+
+
+@pytest.mark.parametrize("name", ["tiny", "glm47flash"])
+def test_rmsnorm_and_residual_sublayer(name):
+    """The decoder block's FFN sublayer x' + MoE(RMSNorm(x')) ("All 43 steps"):
+    the norm against the oracle's double RMSNorm (within half a bf16 ulp of the
+    exact value plus fp32 rounding), the block output with the residual added
+    in the combine against x' + the oracle's MoE of the same normalised rows."""
+    w = W.WORKLOADS[name]
+    if name == "glm47flash":
+        w = w.replace(T=1024, seed=2900)
+    x_res, w_r, b = W.router_inputs(w)
+    gamma = W.norm_weight(w)
+    case = MH.Case(w, x_res, w_r, b)
+    blk = case.block()
+    logits = torch.empty((w.T, w.E), dtype=torch.float32, device="cuda")
+    y, x_ffn = blk.sublayer(case.x_dev, MH.to_dev_bf16(gamma), 1e-5, logits=logits)
+    torch.cuda.synchronize()
+    assert moe.device_error(blk.ws) == 0
+    xf_bits = W.torch_bf16_to_bits(x_ffn)
+    exact = O.rmsnorm(x_res, gamma, 1e-5)
+    got = W.bf16_bits_to_f32(xf_bits).astype(np.float64)
+    assert np.all(np.abs(got - exact) <= MH.half_ulp_bf16(exact) * 1.001 + 1e-6 * np.abs(exact))
+    # the MoE on the GPU's normalised rows, selection from the GPU, gates in double
+    idx = blk.idx.cpu().numpy()
+    tokens = np.arange(w.T) if w.T <= 256 else np.sort(np.random.default_rng(3).choice(w.T, 128, replace=False))
+    z = O.logits(xf_bits[tokens], w_r)
+    gate = np.zeros(idx.shape)
+    gate[tokens] = O.gates_for(z, idx[tokens], w.scale)
+    norm_case = MH.Case(w, xf_bits, w_r, b, weights=case.weights)
+    delta = norm_case.oracle_forward(tokens, idx, gate)
+    y_o = W.bf16_bits_to_f32(x_res[tokens]).astype(np.float64) + delta
+    y_g = MH.bf16_to_f64(y)[tokens]
+    rms = float(np.sqrt(np.mean(delta ** 2)))
+    assert np.all(np.abs(y_g - y_o) <= MH.Y_TOL * rms + MH.half_ulp_bf16(y_o))

@@ -36,6 +36,7 @@ from sigmoid_routed_mixture_b200 import workloads as W  # noqa: E402
 METRIC = "MoE-block tokens/s (GLM-5 shape, bf16, 1 B200)"
 UNIT = "tokens/s"
 KERNELS_PER_STEP = 11  # route 3 + permute 3 + token gather 2 + up 1 + down 1 + combine 1
+KERNELS_PER_DENSE_STEP = 4  # identity rows 1 + up 1 + down 1 + combine 1
 
 
 def peaks():
@@ -241,6 +242,26 @@ def aggregate_tokens_per_s(tokens_per_rank, world, steps, t_max_ms):
     return tokens_per_rank * world * steps / (t_max_ms / 1e3)
 
 
+class DenseBlock:
+    """The dense SwiGLU MLP of the first blocks with its buffers (bench only)."""
+
+    def __init__(self, cfg, weights, dev):
+        import torch
+        from sigmoid_routed_mixture_b200 import moe
+
+        self.cfg = cfg
+        self.weights = weights
+        self.ws = moe.workspace(cfg, device=dev)
+        self.y = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
+        self.counts = torch.zeros((1,), dtype=torch.int32, device=dev)
+        self.margin = torch.ones((cfg.T,), dtype=torch.float32, device=dev)
+
+    def __call__(self, x):
+        from sigmoid_routed_mixture_b200 import moe
+
+        return moe.dense_mlp(self.cfg, self.weights, x, self.ws, y=self.y)
+
+
 def workload_config(w, args):
     return {"workload": w.name, "tokens": w.T, "hidden": w.H, "expert_intermediate": w.I,
             "routed_experts": w.E, "top_k": w.K, "shared_experts": int(w.has_shared),
@@ -292,14 +313,30 @@ def main():
     # each replica draws its own token batch; weights are the workload's
     x, w_r, b = replica_tokens(w, rank)
     weights = W.expert_weights(w, dev)
-    cfg = moe.Config.of(w)
-    blk = moe.MoeBlock(cfg, torch.from_numpy(w_r).to(dev), torch.from_numpy(b).to(dev), **weights)
-    del weights["w1"], weights["w3"], weights["w2"]
+    dense = w.E == 0
+    if dense:
+        cfg = moe.Config.dense(w.T, w.H, w.I)
+        blk = DenseBlock(cfg, moe.pack_weights(cfg, None, None, None, weights["ws1"], weights["ws3"],
+                                               weights["ws2"]), dev)
+    else:
+        cfg = moe.Config.of(w)
+        blk = moe.MoeBlock(cfg, torch.from_numpy(w_r).to(dev), torch.from_numpy(b).to(dev), **weights)
+    del weights
     torch.cuda.empty_cache()
     x_dev = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
+        if dense:
+            # one stage: the dense MLP (identity rows, up, down, combine)
+            if ev is not None:
+                for j in range(4):
+                    ev[j].record(stream)
+            moe.dense_mlp(cfg, blk.weights, x_dev, blk.ws, y=blk.y)
+            if ev is not None:
+                for j in range(4, 7):
+                    ev[j].record(stream)
+            return
         if ev is not None:
             ev[0].record(stream)
         moe.route(cfg, x_dev, blk.w_router, blk.bias, blk.ws, out=(blk.idx, blk.gate, blk.margin))
@@ -378,7 +415,7 @@ def main():
 
     # ---- algorithmic work and the roofline of the dominant kernel
     counts = blk.counts.cpu().numpy()
-    touched = int((counts[: w.E] > 0).sum()) + int(w.has_shared)
+    touched = (int((counts[: w.E] > 0).sum()) if not dense else 0) + int(w.has_shared)
     rows = cfg.rows
     H, I = w.H, w.I
     f_router = 2.0 * w.T * H * w.E
@@ -392,13 +429,16 @@ def main():
     pk = peaks()
     mean_stage = stage_ms.mean(axis=0)
     names = ["route", "permute", "gather_tokens", "expert_up", "expert_down", "combine"]
+    if dense:
+        names[3] = "dense_mlp"
     dom = int(np.argmax(mean_stage))
     ridge = pk["tflops"] * 1e12 / (pk["hbm"] * 1e9)
     work = {"expert_up": (f_up, b_up), "expert_down": (f_down, b_down),
             "route": (f_router, w.T * H * 2 + w.E * H * 4 + w.T * w.K * 8),
             "permute": (0.0, w.T * w.K * 4 * 3 + rows * 4),
             "gather_tokens": (0.0, w.T * H * 2 + rows * H * 2),
-            "combine": (0.0, rows * H * 2 + w.T * H * 2)}
+            "combine": (0.0, rows * H * 2 + w.T * H * 2),
+            "dense_mlp": (f_up + f_down, 3 * H * I * 2 + 2 * w.T * H * 2)}
     f, by = work[names[dom]]
     dur_s = mean_stage[dom] / 1e3
     if f > 0 and f / by > ridge:
@@ -425,17 +465,18 @@ def main():
         "block_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof / step_s,
                            "f_alg_tflop": f_alg / 1e12, "b_alg_gb": b_alg / 1e9},
         "stage_ms": {n: float(v) for n, v in zip(names, mean_stage)},
-        "routing": {"touched_groups": touched, "zero_count_experts": int((counts[: w.E] == 0).sum()),
-                    "max_count": int(counts[: w.E].max()), "min_count": int(counts[: w.E].min()),
-                    "near_ties": int((blk.margin <= 1e-4).sum().item())},
+        "routing": None if dense else {
+            "touched_groups": touched, "zero_count_experts": int((counts[: w.E] == 0).sum()),
+            "max_count": int(counts[: w.E].max()), "min_count": int(counts[: w.E].min()),
+            "near_ties": int((blk.margin <= 1e-4).sum().item())},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(w.T * H * 2),
                 "d2h_bytes_per_step": int(w.T * H * 2), "steps": args.e2e_steps},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (KERNELS_PER_DENSE_STEP if dense else KERNELS_PER_STEP) * args.steps,
         "clocks": clocks,
     }
 
     # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N = 1 only
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not dense:
         os.environ.setdefault("OMP_NUM_THREADS", str(cores()))
         from oracle import oracle as O
 

@@ -218,6 +218,18 @@ moe_status_t moe_combine_residual(const moe_cfg_t *cfg, const void *residual, vo
 moe_status_t moe_rmsnorm(const moe_cfg_t *cfg, const void *x, const void *gamma, float eps,
                          void *x_ffn, void *stream);
 
+/* The dense SwiGLU MLP of the first decoder blocks (GLM-5: blocks 0-2, 6144 ->
+ * intermediate_size 12288; GLM-4.7-Flash: block 0, 2048 -> 10240; nnterp
+ * Config sections and printouts), run through the same tensor-core kernels as
+ * one group: y[t] = (residual[t] +) W2 (silu(W1 x_t) (.) W3 x_t).
+ *   cfg:      E = 0, K = 0, has_shared = 1, I = the MLP's intermediate size
+ *             (moe_workspace_size and moe_pack_weights accept this form; pack
+ *             the MLP's gate/up/down weights as the shared expert ws1/ws3/ws2,
+ *             w1/w3/w2 may be NULL)
+ *   x:        bf16 [T][H];  residual: bf16 [T][H] or NULL;  y: bf16 [T][H]. */
+moe_status_t moe_dense_mlp(const moe_cfg_t *cfg, const moe_weights_t *weights, const void *x,
+                           const void *residual, void *y, void *ws, size_t ws_bytes, void *stream);
+
 /* Read (and clear) the device error word of a workspace.  Synchronises
  * `stream`.  *device_status receives MOE_OK or the first device-side error
  * recorded since the last read.  Returns MOE_ERR_CUDA if the copy fails. */

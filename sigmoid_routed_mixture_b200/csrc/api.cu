@@ -27,9 +27,14 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 int64_t rows_y(const moe_cfg_t &c) { return c.T * c.K + (c.has_shared ? c.T : 0); }
 
-moe_status_t check_cfg(const moe_cfg_t *c) {
+// A dense-MLP configuration (the first decoder blocks): E == 0, K == 0 and
+// has_shared == 1, the shared-expert slot holding the MLP's weights.
+bool is_dense(const moe_cfg_t *c) { return c && c->E == 0 && c->K == 0 && c->has_shared == 1; }
+
+moe_status_t check_cfg(const moe_cfg_t *c, bool allow_dense = false) {
   if (!c) return MOE_ERR_ARG;
-  if (c->T < 0 || c->H <= 0 || c->I <= 0 || c->E <= 0 || c->K <= 0 || c->K > c->E)
+  const bool dense = allow_dense && is_dense(c);
+  if (c->T < 0 || c->H <= 0 || c->I <= 0 || (!dense && (c->E <= 0 || c->K <= 0 || c->K > c->E)))
     return MOE_ERR_ARG;
   if (!isfinite(c->routed_scale)) return MOE_ERR_ARG;
   if (c->has_shared != 0 && c->has_shared != 1) return MOE_ERR_ARG;
@@ -126,7 +131,7 @@ bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, u
 extern "C" {
 
 size_t moe_workspace_size(const moe_cfg_t *cfg) {
-  if (check_cfg(cfg) != MOE_OK) return 0;
+  if (check_cfg(cfg, true) != MOE_OK) return 0;
   return layout(*cfg).total;
 }
 
@@ -148,13 +153,13 @@ const char *moe_status_string(moe_status_t s) {
 moe_status_t moe_pack_weights(const moe_cfg_t *cfg, const void *w1, const void *w3, const void *w2,
                               const void *ws1, const void *ws3, const void *ws2, void *w13_out,
                               void *w2_out, void *stream) {
-  moe_status_t st = check_cfg(cfg);
+  moe_status_t st = check_cfg(cfg, true);
   if (st != MOE_OK) return st;
-  if (!w1 || !w3 || !w2 || !w13_out || !w2_out) return MOE_ERR_ARG;
+  if (!w13_out || !w2_out || (cfg->E > 0 && (!w1 || !w3 || !w2))) return MOE_ERR_ARG;
   if (cfg->has_shared && (!ws1 || !ws3 || !ws2)) return MOE_ERR_ARG;
   const void *ptrs[] = {w1, w3, w2, w13_out, w2_out};
   for (const void *p : ptrs)
-    if (!aligned(p, 16)) return MOE_ERR_ALIGN;
+    if (p && !aligned(p, 16)) return MOE_ERR_ALIGN;
   if (cfg->has_shared && (!aligned(ws1, 16) || !aligned(ws3, 16) || !aligned(ws2, 16)))
     return MOE_ERR_ALIGN;
   return cuda_status(srm::launch_pack(
@@ -378,6 +383,57 @@ moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *weights, con
   st = moe_expert_down(cfg, weights, topk_gate, offsets, sorted, ws, ws_bytes, stream);
   if (st != MOE_OK) return st;
   return moe_combine(cfg, y, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_dense_mlp(const moe_cfg_t *cfg, const moe_weights_t *weights, const void *x,
+                           const void *residual, void *y, void *ws, size_t ws_bytes, void *stream) {
+  moe_status_t st = check_cfg(cfg, true);
+  if (st != MOE_OK) return st;
+  if (!is_dense(cfg)) return MOE_ERR_ARG;
+  if (cfg->T == 0) return MOE_OK;
+  if (!weights || !weights->w13 || !weights->w2 || !x || !y || !ws) return MOE_ERR_ARG;
+  if (!aligned(weights->w13, 16) || !aligned(weights->w2, 16) || !aligned(x, 16) || !aligned(y, 16) ||
+      (residual && !aligned(residual, 16)) || !aligned(ws, 256))
+    return MOE_ERR_ALIGN;
+  const WsLayout L = layout(*cfg);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  const int T = static_cast<int>(cfg->T), H = cfg->H, I = cfg->I;
+  // one group holding every token in order: offsets {0, T}, sorted = identity
+  int32_t *offsets = reinterpret_cast<int32_t *>(wsb + L.err + 192);
+  int32_t *sorted = reinterpret_cast<int32_t *>(wsb + L.pos);
+  if (cudaMemsetAsync(wsb + L.err, 0, sizeof(int32_t), s) != cudaSuccess ||
+      srm::launch_identity_rows(offsets, sorted, T, num_sms(), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const bool pair = cfg->T >= 512;
+  CUtensorMap tm_x, tm_w13, tm_h, tm_w2;
+  if (!make_tmap(&tm_x, x, H, static_cast<uint64_t>(T), 64, 128) ||
+      !make_tmap(&tm_w13, weights->w13, H, 2ull * I, 64,
+                 static_cast<uint32_t>(srm::gemm_b_box_rows(pair))) ||
+      !make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(T), 64, 128,
+                 CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(H), 64,
+                 static_cast<uint32_t>(srm::gemm_b_box_rows(pair)), CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    return MOE_ERR_CUDA;
+  GemmArgs p = gemm_args(*cfg, offsets, sorted, nullptr, wsb, L);
+  p.out = wsb + L.h;
+  p.n_total = 2 * I;
+  p.k_total = H;
+  p.out_ld = I;
+  if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s) != cudaSuccess ||
+      srm::launch_grouped_gemm(srm::kUp, pair, tm_x, tm_w13, p, num_sms(), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  p.out = wsb + L.ybuf;
+  p.n_total = H;
+  p.k_total = I;
+  p.out_ld = H;
+  if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s) != cudaSuccess ||
+      srm::launch_grouped_gemm(srm::kDown, pair, tm_h, tm_w2, p, num_sms(), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cuda_status(srm::launch_combine(reinterpret_cast<const uint16_t *>(wsb + L.ybuf),
+                                         static_cast<const uint16_t *>(residual),
+                                         static_cast<uint16_t *>(y), T, H, 0, 1, num_sms(), s));
 }
 
 moe_status_t moe_get_device_error(void *ws, moe_status_t *device_status, void *stream) {

@@ -67,6 +67,10 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *sorted, int T, 
 cudaError_t launch_combine(const uint16_t *Y, const uint16_t *residual, uint16_t *y, int T, int H,
                            int K, int has_shared, int num_sms, cudaStream_t stream);
 
+// offsets = {0, T}, sorted[t] = t: every token in one group, in order
+cudaError_t launch_identity_rows(int32_t *offsets, int32_t *sorted, int T, int num_sms,
+                                 cudaStream_t stream);
+
 cudaError_t launch_rmsnorm(const uint16_t *x, const uint16_t *gamma, float eps, int T, int H,
                            uint16_t *out, int num_sms, cudaStream_t stream);
 

@@ -35,6 +35,7 @@ SYMBOLS = (
     "moe_combine",
     "moe_combine_residual",
     "moe_rmsnorm",
+    "moe_dense_mlp",
     "moe_get_device_error",
     "moe_status_string",
     "moe_permute_noalloc",
@@ -90,6 +91,11 @@ class Config:
     def c(self) -> _Cfg:
         return _Cfg(self.T, self.H, self.I, self.E, self.K, self.routed_scale, int(bool(self.has_shared)))
 
+    @classmethod
+    def dense(cls, T: int, H: int, I: int) -> "Config":
+        """A dense-MLP configuration (E = K = 0, the MLP in the shared-expert slot)."""
+        return cls(T, H, I, 0, 0, 1.0, True)
+
     @property
     def rows(self) -> int:
         """Expert-sorted rows: T*K routed plus T shared."""
@@ -130,6 +136,8 @@ def lib():
         L.moe_combine_residual.argtypes = [P(_Cfg), vp, vp, vp, ctypes.c_size_t, vp]
         L.moe_rmsnorm.restype = ctypes.c_int
         L.moe_rmsnorm.argtypes = [P(_Cfg), vp, vp, ctypes.c_float, vp, vp]
+        L.moe_dense_mlp.restype = ctypes.c_int
+        L.moe_dense_mlp.argtypes = [P(_Cfg), P(_Weights), vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.moe_get_device_error.restype = ctypes.c_int
         L.moe_get_device_error.argtypes = [vp, P(ctypes.c_int), vp]
         L.moe_permute_noalloc.restype = ctypes.c_int
@@ -192,15 +200,17 @@ def pack_weights(cfg: Config, w1, w3, w2, ws1=None, ws3=None, ws2=None, stream=N
     """Returns (w13 bf16 [(E+1)*2I, H], w2p fp16 [(E+1)*H, I]) in the kernels' layout."""
     E, I, H = cfg.E, cfg.I, cfg.H
     bf = torch.bfloat16
-    _req(w1, bf, (E, I, H), "w1")
-    _req(w3, bf, (E, I, H), "w3")
-    _req(w2, bf, (E, H, I), "w2")
+    if E > 0 or w1 is not None:
+        _req(w1, bf, (E, I, H), "w1")
+        _req(w3, bf, (E, I, H), "w3")
+        _req(w2, bf, (E, H, I), "w2")
     if cfg.has_shared:
         _req(ws1, bf, (I, H), "ws1")
         _req(ws3, bf, (I, H), "ws3")
         _req(ws2, bf, (H, I), "ws2")
-    w13 = torch.empty(((E + 1) * 2 * I, H), dtype=bf, device=w1.device)
-    w2p = torch.empty(((E + 1) * H, I), dtype=torch.float16, device=w1.device)
+    dev = (w1 if w1 is not None else ws1).device
+    w13 = torch.empty(((E + 1) * 2 * I, H), dtype=bf, device=dev)
+    w2p = torch.empty(((E + 1) * H, I), dtype=torch.float16, device=dev)
     _check(lib().moe_pack_weights(ctypes.byref(cfg.c()), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(ws1),
                                   _ptr(ws3), _ptr(ws2), _ptr(w13), _ptr(w2p), _stream(stream)),
            "moe_pack_weights")
@@ -327,6 +337,19 @@ def rmsnorm(cfg: Config, x, gamma, eps=1e-5, out=None, stream=None):
     _check(lib().moe_rmsnorm(ctypes.byref(cfg.c()), _ptr(x), _ptr(gamma), float(eps), _ptr(out),
                              _stream(stream)), "moe_rmsnorm")
     return out
+
+
+def dense_mlp(cfg: Config, weights, x, ws, residual=None, y=None, stream=None):
+    """Dense SwiGLU MLP (cfg from Config.dense): y = (residual +) W2 (silu(W1 x) * W3 x)."""
+    _req(x, torch.bfloat16, (cfg.T, cfg.H), "x")
+    if residual is not None:
+        _req(residual, torch.bfloat16, (cfg.T, cfg.H), "residual")
+    if y is None:
+        y = torch.empty_like(x)
+    W_ = _weights_struct(cfg, weights)
+    _check(lib().moe_dense_mlp(ctypes.byref(cfg.c()), ctypes.byref(W_), _ptr(x), _ptr(residual), _ptr(y),
+                               _ptr(ws), ws.numel(), _stream(stream)), "moe_dense_mlp")
+    return y
 
 
 def device_error(ws, stream=None) -> int:

@@ -58,6 +58,10 @@ WORKLOADS = {
     # GLM-5 expert shapes with 32 experts: 2.5 GB of weights, small enough for
     # multi-pass profiler captures, still far larger than the 126 MB L2
     "glm5_e32": Workload("glm5_e32", T=8192, H=6144, I=2048, E=32, K=8, scale=2.5, seed=1005),
+    # dense SwiGLU MLP of the first blocks (E = K = 0; I = intermediate_size)
+    "glm5_dense": Workload("glm5_dense", T=16384, H=6144, I=12288, E=0, K=0, scale=1.0, seed=1007),
+    "glm47flash_dense": Workload("glm47flash_dense", T=4096, H=2048, I=10240, E=0, K=0, scale=1.0,
+                                 seed=1008),
     "glm5_decode_e32": Workload("glm5_decode_e32", T=64, H=6144, I=2048, E=32, K=8, scale=2.5,
                                 seed=1006),
 }

@@ -223,3 +223,38 @@ def test_rmsnorm_and_residual_sublayer(name):
     y_g = MH.bf16_to_f64(y)[tokens]
     rms = float(np.sqrt(np.mean(delta ** 2)))
     assert np.all(np.abs(y_g - y_o) <= MH.Y_TOL * rms + MH.half_ulp_bf16(y_o))
+
+
+@pytest.mark.parametrize("name,T", [("tiny_dense", 300), ("tiny_dense", 1500), ("glm47flash_dense", 4096),
+                                    ("glm5_dense", 16384)])
+def test_dense_mlp(name, T):
+    """The dense SwiGLU MLP of the first blocks through the same kernels as one
+    group (E = K = 0): against the oracle's shared-expert SwiGLU (a single dummy
+    routed expert at gate 0 leaves exactly the shared term), with the residual
+    added in the combine."""
+    if name == "tiny_dense":
+        w = W.WORKLOADS["tiny"].replace(name="tiny_dense", T=T, I=512, E=0, K=0, seed=3000 + T)
+    else:
+        w = W.WORKLOADS[name]
+    rng = np.random.default_rng(w.seed)
+    x = W.f32_to_bf16_bits(rng.standard_normal((w.T, w.H), dtype=np.float32))
+    res = W.f32_to_bf16_bits(rng.standard_normal((w.T, w.H), dtype=np.float32))
+    wt = W.expert_weights(w, "cuda")
+    cfg = moe.Config.dense(w.T, w.H, w.I)
+    weights = moe.pack_weights(cfg, None, None, None, wt["ws1"], wt["ws3"], wt["ws2"])
+    ws = moe.workspace(cfg)
+    y = moe.dense_mlp(cfg, weights, MH.to_dev_bf16(x), ws, residual=MH.to_dev_bf16(res))
+    torch.cuda.synchronize()
+    assert moe.device_error(ws) == 0
+    tokens = np.arange(w.T) if w.T <= 1500 else np.sort(rng.choice(w.T, 24, replace=False))
+    sh = [W.torch_bf16_to_bits(wt[n]) for n in ("ws1", "ws3", "ws2")]
+    dummy1 = [np.zeros((w.I, w.H), np.uint16)]
+    dummy2 = [np.zeros((w.H, w.I), np.uint16)]
+    idx = np.zeros((w.T, 1), np.int32)
+    mlp = O.forward(x, dummy1, dummy1, dummy2, sh[0], sh[1], sh[2], idx, np.zeros((w.T, 1)), tokens=tokens)
+    y_o = W.bf16_bits_to_f32(res[tokens]).astype(np.float64) + mlp
+    y_g = MH.bf16_to_f64(y)[tokens]
+    rms = float(np.sqrt(np.mean(mlp ** 2)))
+    assert np.all(np.abs(y_g - y_o) <= MH.Y_TOL * rms + MH.half_ulp_bf16(y_o))
+    del wt, weights, ws
+    free()

@@ -284,6 +284,9 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--tokens", type=int, default=0, help="run the workload at this many tokens")
+    ap.add_argument("--cublas", action="store_true",
+                    help="dense workloads: also time torch.matmul (cuBLAS) on the same two GEMMs")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -309,15 +312,21 @@ def main():
     from sigmoid_routed_mixture_b200 import moe
 
     w = W.WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.replace(T=args.tokens)
     dev = torch.device("cuda", torch.cuda.current_device())
     # each replica draws its own token batch; weights are the workload's
     x, w_r, b = replica_tokens(w, rank)
     weights = W.expert_weights(w, dev)
     dense = w.E == 0
+    cublas = None
     if dense:
         cfg = moe.Config.dense(w.T, w.H, w.I)
         blk = DenseBlock(cfg, moe.pack_weights(cfg, None, None, None, weights["ws1"], weights["ws3"],
                                                weights["ws2"]), dev)
+        if args.cublas:  # the same two GEMMs through torch.matmul, for comparison only
+            cublas = (torch.cat([weights["ws1"], weights["ws3"]], 0), weights["ws2"].clone(),
+                      torch.randn((w.T, w.I), device=dev).to(torch.bfloat16))
     else:
         cfg = moe.Config.of(w)
         blk = moe.MoeBlock(cfg, torch.from_numpy(w_r).to(dev), torch.from_numpy(b).to(dev), **weights)
@@ -413,6 +422,25 @@ def main():
     if moe.device_error(blk.ws) != 0:
         raise RuntimeError("device error during the timed steps")
 
+    cublas_ms = None
+    if cublas is not None:
+        w13_t, w2_t, h_t = cublas
+
+        def loop(fn):
+            fn()
+            torch.cuda.synchronize()
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            return a0.elapsed_time(a1) / args.steps
+
+        cublas_ms = {"up": loop(lambda: torch.matmul(x_dev, w13_t.t())),
+                     "down": loop(lambda: torch.matmul(h_t, w2_t.t()))}
+
     # ---- algorithmic work and the roofline of the dominant kernel
     counts = blk.counts.cpu().numpy()
     touched = (int((counts[: w.E] > 0).sum()) if not dense else 0) + int(w.has_shared)
@@ -472,6 +500,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(w.T * H * 2),
                 "d2h_bytes_per_step": int(w.T * H * 2), "steps": args.e2e_steps},
         "gpu_launches": (KERNELS_PER_DENSE_STEP if dense else KERNELS_PER_STEP) * args.steps,
+        "cublas_same_gemms_ms": cublas_ms,
         "clocks": clocks,
     }
 

@@ -25,14 +25,21 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// One warp per token; the row moves in chunks of 8 x 16 bytes per lane.
+// WPT warps per token (each moves a contiguous part of the row, 8 x 16 bytes
+// per lane at a time): one warp per token for large batches, more when there
+// are few tokens so that enough bytes are in flight.
 __global__ void __launch_bounds__(256)
     scatter_rows_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ pos, int T,
-                        int H, int K, int has_shared, int rows, uint16_t *__restrict__ xs) {
+                        int H, int K, int has_shared, int rows, int wpt, uint16_t *__restrict__ xs) {
   const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // global warp
   const int warps = gridDim.x * (blockDim.x >> 5);
   const int vecs = H / 8;  // 16-byte vectors per row
-  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+  const int part = (vecs + wpt - 1) / wpt;
+  for (int job = gw; job < T * wpt; job += warps) {
+    const int t = job / wpt;
+    const int v_begin = (job - t * wpt) * part;
+    const int v_end = min(vecs, v_begin + part);
     int dst[17];
     const int n_dst = K + has_shared;
 #pragma unroll
@@ -45,12 +52,12 @@ __global__ void __launch_bounds__(256)
       dst[k] = (d >= 0 && d < rows) ? d : -1;
     }
     const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t) * H);
-    for (int v0 = 0; v0 < vecs; v0 += 32 * 8) {
+    for (int v0 = v_begin; v0 < v_end; v0 += 32 * 8) {
       uint4 buf[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int v = v0 + j * 32 + lane;
-        if (v < vecs) buf[j] = __ldcs(src + v);
+        if (v < v_end) buf[j] = __ldcs(src + v);
       }
 #pragma unroll
       for (int k = 0; k < 17; ++k) {
@@ -60,7 +67,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int v = v0 + j * 32 + lane;
-          if (v < vecs) out[v] = buf[j];
+          if (v < v_end) out[v] = buf[j];
         }
       }
     }
@@ -94,9 +101,11 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *sorted, int T, 
   int blocks = (rows + 255) / 256;
   if (blocks > num_sms * 8) blocks = num_sms * 8;
   invert_rows_kernel<<<blocks, 256, 0, stream>>>(sorted, rows, n_rows_y, pos, err);
-  int tb = (T + 7) / 8;
+  int wpt = 1;  // warps per token: aim for at least ~4 warps per SM in flight
+  while (wpt < 8 && T * wpt < num_sms * 32) wpt *= 2;
+  int tb = (T * wpt + 7) / 8;
   if (tb > num_sms * 16) tb = num_sms * 16;
-  scatter_rows_kernel<<<tb, 256, 0, stream>>>(x, pos, T, H, K, has_shared, rows, xs);
+  scatter_rows_kernel<<<tb, 256, 0, stream>>>(x, pos, T, H, K, has_shared, rows, wpt, xs);
   return cudaGetLastError();
 }
 

@@ -151,10 +151,92 @@ __global__ void __launch_bounds__(pm::THREADS)
   }
 }
 
+// Small batches (n <= SMALL_N assignments, e.g. decode): the same histogram ->
+// scan -> stable scatter in ONE CTA, so the permutation costs one launch.
+namespace pm {
+constexpr int SMALL_THREADS = 1024;
+constexpr int SMALL_WARPS = SMALL_THREADS / 32;
+constexpr int SMALL_N = 8192;
+}  // namespace pm
+
+__global__ void __launch_bounds__(pm::SMALL_THREADS)
+    permute_small_kernel(const int32_t *__restrict__ idx, int n, int E, int T, int has_shared,
+                         int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                         int32_t *__restrict__ sorted, int *err) {
+  __shared__ int hist[pm::MAX_E];
+  __shared__ int scan[pm::MAX_E];
+  __shared__ int cursor[pm::MAX_E];
+  __shared__ int wcnt[pm::SMALL_WARPS][pm::MAX_E];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < pm::MAX_E; e += pm::SMALL_THREADS) hist[e] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += pm::SMALL_THREADS) {
+    const int e = idx[i];
+    if (e < 0 || e >= E)
+      record_error(err, MOE_ERR_BAD_INDEX);
+    else
+      atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  if (tid < pm::MAX_E) scan[tid] = hist[tid];
+  __syncthreads();
+  for (int d = 1; d < pm::MAX_E; d <<= 1) {  // inclusive Hillis-Steele scan
+    const int v = (tid < pm::MAX_E && tid >= d) ? scan[tid - d] : 0;
+    __syncthreads();
+    if (tid < pm::MAX_E) scan[tid] += v;
+    __syncthreads();
+  }
+  if (tid < E) {
+    const int excl = scan[tid] - hist[tid];
+    counts[tid] = hist[tid];
+    offsets[tid] = excl;
+    cursor[tid] = excl;
+  }
+  if (tid == 0) {
+    const int routed = scan[pm::MAX_E - 1];
+    counts[E] = has_shared ? T : 0;
+    offsets[E] = routed;
+    offsets[E + 1] = routed + (has_shared ? T : 0);
+  }
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < n; base += pm::SMALL_THREADS) {
+    for (int k = tid; k < pm::SMALL_WARPS * pm::MAX_E; k += pm::SMALL_THREADS) (&wcnt[0][0])[k] = 0;
+    __syncthreads();
+    const int i = base + tid;
+    int e = i < n ? idx[i] : -1;
+    if (e >= E) e = -1;
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(same & lt_mask);
+    if (e >= 0 && rank == 0) wcnt[warp][e] = __popc(same);
+    __syncthreads();
+    if (e >= 0) {
+      int before = 0;
+      for (int w = 0; w < warp; ++w) before += wcnt[w][e];
+      sorted[cursor[e] + before + rank] = i;
+    }
+    __syncthreads();
+    if (tid < E) {
+      int add = 0;
+      for (int w = 0; w < pm::SMALL_WARPS; ++w) add += wcnt[w][tid];
+      cursor[tid] += add;
+    }
+    __syncthreads();
+  }
+  if (has_shared) {
+    const int sbase = scan[pm::MAX_E - 1];
+    for (int t = tid; t < T; t += pm::SMALL_THREADS) sorted[sbase + t] = n + t;
+  }
+}
+
 cudaError_t launch_permute(const int32_t *idx, int T, int E, int K, int has_shared, int32_t *counts,
                            int32_t *offsets, int32_t *sorted, int32_t *scratch, int *err,
                            cudaStream_t stream) {
   const int n = T * K;
+  if (n <= pm::SMALL_N) {
+    permute_small_kernel<<<1, pm::SMALL_THREADS, 0, stream>>>(idx, n, E, T, has_shared, counts,
+                                                              offsets, sorted, err);
+    return cudaGetLastError();
+  }
   const int nchunks = permute_num_chunks(n);
   permute_hist_kernel<<<nchunks, pm::THREADS, 0, stream>>>(idx, n, E, nchunks, scratch, err);
   permute_scan_kernel<<<1, pm::SCAN_THREADS, 0, stream>>>(scratch, E, nchunks, T, has_shared, counts,

@@ -22,9 +22,11 @@
 //      chains promoted to fp32 registers (see below); the H range may be split
 //      over S CTAs (S > 1 when there are few 128-token tiles) and each CTA
 //      writes fp32 partial logits zp[s][t][e].
-//   3) router_select_kernel: one warp per token sums the S partials in order
-//      (deterministic), then s, keys, K rounds of a warp arg-max (key
-//      descending, index ascending), one more round for the margin, gates.
+//   2b) router_reduce_kernel (S > 1): one thread per (token, expert) sums the
+//      S partials in a fixed order (deterministic).
+//   3) router_select_kernel: one warp per token: s, keys, K rounds of a warp
+//      arg-max (key descending, index ascending), one more round for the
+//      margin, gates.
 #include <cuda.h>
 #include <math.h>
 
@@ -67,22 +69,40 @@ __device__ __forceinline__ uint16_t bf16_rn_bits(float v) {
   return *reinterpret_cast<uint16_t *>(&b);
 }
 
+// Eight consecutive weights per thread: two 16-byte loads, three 16-byte stores.
 __global__ void __launch_bounds__(256)
     router_split_kernel(const float *__restrict__ w_r, int E, int e_pad, int H,
                         uint16_t *__restrict__ wsplit) {
   const int64_t n = static_cast<int64_t>(e_pad) * H;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+  const int64_t n8 = n / 8;  // H is a multiple of 256
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t e = i / H;
-    const float w = e < E ? w_r[i] : 0.f;
-    const uint16_t hi = bf16_rn_bits(w);
-    const float r1 = w - bf16_bits_to_float(hi);
-    const uint16_t mid = bf16_rn_bits(r1);
-    const float r2 = r1 - bf16_bits_to_float(mid);
-    const uint16_t lo = bf16_rn_bits(r2);
-    wsplit[i] = hi;
-    wsplit[n + i] = mid;
-    wsplit[2 * n + i] = lo;
+    const int64_t e = (i * 8) / H;
+    float w[8];
+    if (e < E) {
+      const float4 a = reinterpret_cast<const float4 *>(w_r)[2 * i];
+      const float4 b = reinterpret_cast<const float4 *>(w_r)[2 * i + 1];
+      w[0] = a.x, w[1] = a.y, w[2] = a.z, w[3] = a.w, w[4] = b.x, w[5] = b.y, w[6] = b.z, w[7] = b.w;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w[k] = 0.f;
+    }
+    uint16_t hi[8], mid[8], lo[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      hi[k] = bf16_rn_bits(w[k]);
+      const float r1 = w[k] - bf16_bits_to_float(hi[k]);
+      mid[k] = bf16_rn_bits(r1);
+      const float r2 = r1 - bf16_bits_to_float(mid[k]);
+      lo[k] = bf16_rn_bits(r2);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(wsplit);
+    dst[i] = make_uint4(hi[0] | (uint32_t(hi[1]) << 16), hi[2] | (uint32_t(hi[3]) << 16),
+                        hi[4] | (uint32_t(hi[5]) << 16), hi[6] | (uint32_t(hi[7]) << 16));
+    dst[n8 + i] = make_uint4(mid[0] | (uint32_t(mid[1]) << 16), mid[2] | (uint32_t(mid[3]) << 16),
+                             mid[4] | (uint32_t(mid[5]) << 16), mid[6] | (uint32_t(mid[7]) << 16));
+    dst[2 * n8 + i] = make_uint4(lo[0] | (uint32_t(lo[1]) << 16), lo[2] | (uint32_t(lo[3]) << 16),
+                                 lo[4] | (uint32_t(lo[5]) << 16), lo[6] | (uint32_t(lo[7]) << 16));
   }
 }
 
@@ -291,6 +311,27 @@ int router_stages(int e_pad) {
   return s > 4 ? 4 : s;
 }
 
+// ---------------------------------------------------------------- 2b) split-K sum
+
+// z[t][e] = sum over the S partials, written over partial 0.  One thread per
+// (token, expert); eight independent accumulators (split s goes to s mod 8)
+// added in a fixed order at the end: deterministic, and eight loads in flight.
+__global__ void __launch_bounds__(256)
+    router_reduce_kernel(float *__restrict__ zp, int splits, int T, int e_pad) {
+  const int64_t n = static_cast<int64_t>(T) * e_pad;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int sp = 0;
+    for (; sp + 8 <= splits; sp += 8) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc[u] += zp[(sp + u) * n + i];
+    }
+    for (int u = 0; sp < splits; ++sp, ++u) acc[u] += zp[sp * n + i];
+    zp[i] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+  }
+}
+
 // ---------------------------------------------------------------- 3) select
 
 template <int NE>
@@ -308,17 +349,7 @@ __global__ void __launch_bounds__(256)
     const int e = lane + 32 * j;
     float z = 0.f;
     if (e < E) {
-      // partial sums of the H splits, eight loads in flight, added in a fixed order
-      const float *zc = zp + static_cast<size_t>(t) * e_pad + e;
-      const size_t stride = static_cast<size_t>(T) * e_pad;
-      int sp = 0;
-      for (; sp + 8 <= splits; sp += 8) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = zc[(sp + u) * stride];
-        z += ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
-      }
-      for (; sp < splits; ++sp) z += zc[sp * stride];
+      z = zp[static_cast<size_t>(t) * e_pad + e];
       if (logits) logits[static_cast<size_t>(t) * E + e] = z;
     }
     const float sj = sigmoidf_(z);
@@ -415,18 +446,24 @@ cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, c
   }
   if (e != cudaSuccess) return e;
   const int used_splits = static_cast<int>(grid.y);
+  if (used_splits > 1) {
+    const int64_t n = static_cast<int64_t>(T) * e_pad;
+    int rb = static_cast<int>((n + 255) / 256);
+    if (rb > num_sms * 8) rb = num_sms * 8;
+    router_reduce_kernel<<<rb, 256, 0, stream>>>(zp, used_splits, T, e_pad);
+  }
   const int blocks = (T + 7) / 8;
   if (E <= 32)
-    router_select_kernel<1><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
+    router_select_kernel<1><<<blocks, 256, 0, stream>>>(zp, 1, bias, T, E, e_pad, K, scale,
                                                         idx, gate, margin, logits);
   else if (E <= 64)
-    router_select_kernel<2><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
+    router_select_kernel<2><<<blocks, 256, 0, stream>>>(zp, 1, bias, T, E, e_pad, K, scale,
                                                         idx, gate, margin, logits);
   else if (E <= 128)
-    router_select_kernel<4><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
+    router_select_kernel<4><<<blocks, 256, 0, stream>>>(zp, 1, bias, T, E, e_pad, K, scale,
                                                         idx, gate, margin, logits);
   else
-    router_select_kernel<8><<<blocks, 256, 0, stream>>>(zp, used_splits, bias, T, E, e_pad, K, scale,
+    router_select_kernel<8><<<blocks, 256, 0, stream>>>(zp, 1, bias, T, E, e_pad, K, scale,
                                                         idx, gate, margin, logits);
   return cudaGetLastError();
 }

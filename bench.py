@@ -35,8 +35,21 @@ from sigmoid_routed_mixture_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-block tokens/s (GLM-5 shape, bf16, 1 B200)"
 UNIT = "tokens/s"
-KERNELS_PER_STEP = 11  # route 3 + permute 3 + token gather 2 + up 1 + down 1 + combine 1
 KERNELS_PER_DENSE_STEP = 4  # identity rows 1 + up 1 + down 1 + combine 1
+
+
+def kernels_per_step(w, num_sms=148):
+    """Kernel launches of one routed step: router split + logits (+ split-K
+    reduction when the H range is split) + select; permutation (one CTA for
+    small batches, else histogram + scan + scatter); token gather (invert +
+    scatter); up GEMM; down GEMM; combine."""
+    m_tiles = -(-w.T // 128)
+    kblocks = w.H // 64
+    splits = max(1, min(num_sms // max(1, m_tiles), max(1, kblocks // 2)))
+    kb_per = -(-kblocks // splits)
+    route = 3 + (1 if -(-kblocks // kb_per) > 1 else 0)
+    permute = 1 if w.T * w.K <= 8192 else 3
+    return route + permute + 2 + 1 + 1 + 1
 
 
 def peaks():
@@ -499,7 +512,7 @@ def main():
             "near_ties": int((blk.margin <= 1e-4).sum().item())},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(w.T * H * 2),
                 "d2h_bytes_per_step": int(w.T * H * 2), "steps": args.e2e_steps},
-        "gpu_launches": (KERNELS_PER_DENSE_STEP if dense else KERNELS_PER_STEP) * args.steps,
+        "gpu_launches": (KERNELS_PER_DENSE_STEP if dense else kernels_per_step(w)) * args.steps,
         "cublas_same_gemms_ms": cublas_ms,
         "clocks": clocks,
     }

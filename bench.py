@@ -48,7 +48,7 @@ def kernels_per_step(w, num_sms=148):
     splits = max(1, min(num_sms // max(1, m_tiles), max(1, kblocks // 2)))
     kb_per = -(-kblocks // splits)
     route = 3 + (1 if -(-kblocks // kb_per) > 1 else 0)
-    permute = 1 if w.T * w.K <= 8192 else 3
+    permute = 1 if w.T * w.K <= 16384 else 3
     return route + permute + 2 + 1 + 1 + 1
 
 
@@ -298,6 +298,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--tokens", type=int, default=0, help="run the workload at this many tokens")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every step from the host instead of replaying a CUDA graph of it")
     ap.add_argument("--cublas", action="store_true",
                     help="dense workloads: also time torch.matmul (cuBLAS) on the same two GEMMs")
     args = ap.parse_args()
@@ -400,10 +402,29 @@ def main():
         step(evs[i])
     e_end.record(stream)
     torch.cuda.synchronize()
+    eager_ms = e_start.elapsed_time(e_end)
+    total_ms = eager_ms
+    graph = None
+    if not args.eager:
+        # the same step captured once as a CUDA graph and replayed: every kernel of
+        # every step still runs; only the host launch gaps go away
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e_start.record(stream)
+        for i in range(args.steps):
+            graph.replay()
+        e_end.record(stream)
+        torch.cuda.synchronize()
+        total_ms = e_start.elapsed_time(e_end)
     clocks = sampler.stop()
     if dist is not None:
         dist.barrier()
-    total_ms = e_start.elapsed_time(e_end)
     stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(6)]
                          for i in range(args.steps)])
     t_max = max_over_ranks(total_ms, dist, dev)
@@ -415,8 +436,12 @@ def main():
     x_in = torch.empty_like(x_dev)
 
     def e2e_step():
-        x_in.copy_(x_host, non_blocking=True)
-        blk(x_in)
+        if graph is not None:
+            x_dev.copy_(x_host, non_blocking=True)  # into the buffer the graph reads
+            graph.replay()
+        else:
+            x_in.copy_(x_host, non_blocking=True)
+            blk(x_in)
         y_host.copy_(blk.y, non_blocking=True)
 
     e2e_step()
@@ -506,6 +531,8 @@ def main():
         "block_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof / step_s,
                            "f_alg_tflop": f_alg / 1e12, "b_alg_gb": b_alg / 1e9},
         "stage_ms": {n: float(v) for n, v in zip(names, mean_stage)},
+        "launch": "cuda graph replay" if graph is not None else "eager",
+        "eager_ms_per_step": eager_ms / args.steps,
         "routing": None if dense else {
             "touched_groups": touched, "zero_count_experts": int((counts[: w.E] == 0).sum()),
             "max_count": int(counts[: w.E].max()), "min_count": int(counts[: w.E].min()),

@@ -151,12 +151,12 @@ __global__ void __launch_bounds__(pm::THREADS)
   }
 }
 
-// Small batches (n <= SMALL_N assignments, e.g. decode): the same histogram ->
+// Small batches (n <= SMALL_N assignments: decode, 4096 tokens at top-4): the same histogram ->
 // scan -> stable scatter in ONE CTA, so the permutation costs one launch.
 namespace pm {
 constexpr int SMALL_THREADS = 1024;
 constexpr int SMALL_WARPS = SMALL_THREADS / 32;
-constexpr int SMALL_N = 8192;
+constexpr int SMALL_N = 16384;
 }  // namespace pm
 
 __global__ void __launch_bounds__(pm::SMALL_THREADS)

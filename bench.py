@@ -321,7 +321,7 @@ def main():
         import torch.distributed as dist
 
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     else:
         torch.cuda.set_device(0)
     from sigmoid_routed_mixture_b200 import moe
@@ -392,39 +392,43 @@ def main():
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(torch.cuda.current_device())
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.3)
-    e_start.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
-    e_end.record(stream)
-    torch.cuda.synchronize()
-    eager_ms = e_start.elapsed_time(e_end)
-    total_ms = eager_ms
     graph = None
     if not args.eager:
-        # the same step captured once as a CUDA graph and replayed: every kernel of
+        # the step captured once as a CUDA graph and replayed: every kernel of
         # every step still runs; only the host launch gaps go away
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             step()
         for _ in range(args.warmup):
             graph.replay()
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        e_start.record(stream)
-        for i in range(args.steps):
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    # the timed steps (value): graph replays, or host launches with --eager
+    e_start.record(stream)
+    for i in range(args.steps):
+        if graph is not None:
             graph.replay()
-        e_end.record(stream)
-        torch.cuda.synchronize()
-        total_ms = e_start.elapsed_time(e_end)
+        else:
+            step(evs[i])
+    e_end.record(stream)
+    torch.cuda.synchronize()
     clocks = sampler.stop()
     if dist is not None:
         dist.barrier()
+    total_ms = e_start.elapsed_time(e_end)
+    eager_ms = total_ms
+    if graph is not None:
+        # per-stage breakdown from the same number of host-launched steps, after
+        # the timed ones (it only feeds the stage shares and the kernel roofline)
+        e_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        e_end.record(stream)
+        torch.cuda.synchronize()
+        eager_ms = e_start.elapsed_time(e_end)
     stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(6)]
                          for i in range(args.steps)])
     t_max = max_over_ranks(total_ms, dist, dev)

@@ -57,6 +57,21 @@ def test_cta_pair_tiles(T):
     full_check(w, lambda res: MH.sample_tokens(res, w.T, 400))
 
 
+@pytest.mark.parametrize("E,K", [(2, 1), (1, 1), (3, 2)])
+def test_degenerate_expert_counts(E, K):
+    """One expert per token (gate = scale), a single expert in all (every token on it)."""
+    w = W.WORKLOADS["tiny"].replace(E=E, K=K, T=150, seed=3100 + 10 * E + K)
+    case, res, _ = full_check(w)
+    if K == 1:
+        assert np.allclose(res["gate"], w.scale, rtol=0, atol=2e-6)
+
+
+def test_cta_pair_tiles_without_shared_expert():
+    w = W.WORKLOADS["tiny"].replace(T=2500, has_shared=False, seed=3200)
+    assert w.T * w.K >= 512 * w.E
+    full_check(w, lambda res: MH.sample_tokens(res, w.T, 300))
+
+
 def test_without_shared_expert():
     full_check(W.WORKLOADS["tiny"].replace(has_shared=False, T=200, seed=2200))
 

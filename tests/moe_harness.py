@@ -175,16 +175,36 @@ def check_forward(case: Case, res, tokens):
 
 
 def sample_tokens(res, T, n_random, seed=0):
-    """A seeded token sample that always includes the first and last token and
-    the tokens sitting in the ragged last row of several expert groups."""
+    """A seeded token sample that always includes the first and last token, the
+    tokens in the ragged last row of the largest expert groups, and the tokens
+    on either side of each group's last 256-row boundary."""
     rng = np.random.default_rng(seed)
     picks = {0, T - 1}
     picks.update(rng.choice(T, size=min(n_random, T), replace=False).tolist())
     offsets, srt = res["offsets"], res["sorted"]
     K = res["idx"].shape[1]
     counts = np.diff(offsets)[:-1]
+    rows = []
     for g in np.argsort(-counts)[:4]:
         if counts[g] > 0:
-            a = int(srt[offsets[g + 1] - 1])
-            picks.add(a // K if a < T * K else a - T * K)
+            rows.append(offsets[g + 1] - 1)
+    # Both ways a group can end in 256-row CTA-pair tiling: a last partial
+    # block of <= 128 rows (its own 128-row tile) or of 129..255 rows (a
+    # partial pair tile).  Take the rows on either side of each boundary, for
+    # up to 16 groups of each kind.
+    n_groups = len(offsets) - 1  # routed experts and the shared expert
+    kinds = {True: 0, False: 0}
+    for g in range(n_groups):
+        c = int(offsets[g + 1] - offsets[g])
+        if c % 256 == 0:
+            continue
+        small = c % 256 <= 128
+        if kinds[small] >= 16:
+            continue
+        kinds[small] += 1
+        start = int(offsets[g]) + c // 256 * 256
+        rows += [start, int(offsets[g + 1]) - 1] + ([start - 1] if c >= 256 else [])
+    for r in rows:
+        a = int(srt[r])
+        picks.add(a // K if a < T * K else a - T * K)
     return np.array(sorted(picks), dtype=np.int64)

@@ -54,7 +54,10 @@ def test_cta_pair_tiles(T):
     256 rows; 3001 tokens leave ragged 256-row and 128-row tails."""
     w = W.WORKLOADS["tiny"].replace(T=T, seed=2700 + T)
     assert T * w.K >= 512 * w.E
-    full_check(w, lambda res: MH.sample_tokens(res, w.T, 400))
+    _, res, _ = full_check(w, lambda res: MH.sample_tokens(res, w.T, 400))
+    if T == 3001:  # both kinds of group end: a 128-row tail tile and a partial pair tile
+        rem = np.diff(res["offsets"]) % 256
+        assert np.any((rem > 0) & (rem <= 128)) and np.any(rem > 128)
 
 
 @pytest.mark.parametrize("E,K", [(2, 1), (1, 1), (3, 2)])

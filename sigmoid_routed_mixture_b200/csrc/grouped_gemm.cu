@@ -116,10 +116,14 @@ struct TileCoord {
 // and inside a group the row block runs fastest: the units working at the same
 // moment share each 256-column weight tile (one DRAM read serves all the
 // group's row blocks) instead of spreading over many weight tiles that evict
-// one another from L2.
+// one another from L2.  A group with more than m_chunk row blocks (the shared
+// expert at large batches) is walked in chunks of m_chunk row blocks, each
+// chunk through all column blocks, so that the chunk's rows stay in L2 while
+// every column block reads them (a whole 16384-token group would not fit and
+// would be re-read from DRAM once per column block).
 template <bool kPair>
 __device__ __forceinline__ TileCoord decode_tile(const gg::Smem &s, int groups, int n_tiles,
-                                                 int tile, int rank) {
+                                                 int m_chunk, int tile, int rank) {
   const int mt_flat = tile / n_tiles;
   int lo = 0, hi = groups - 1;  // last g with tile_start[g] <= mt_flat
   while (lo < hi) {
@@ -131,8 +135,12 @@ __device__ __forceinline__ TileCoord decode_tile(const gg::Smem &s, int groups, 
   }
   const int mblocks = s.tile_start[lo + 1] - s.tile_start[lo];
   const int local = tile - s.tile_start[lo] * n_tiles;
-  const int nt = local / mblocks;
-  const int mt = local - nt * mblocks;
+  const int chunk = local / (m_chunk * n_tiles);
+  const int m0 = chunk * m_chunk;
+  const int cm = min(m_chunk, mblocks - m0);  // row blocks in this chunk
+  const int r = local - m0 * n_tiles;
+  const int nt = r / cm;
+  const int mt = m0 + (r - nt * cm);
   TileCoord c;
   c.g = lo;
   c.row_base = s.grp_off[lo] + mt * gg::Cfg<kPair>::TILE_M + rank * gg::BM;
@@ -164,6 +172,8 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
   const int groups = p.groups;
   const int n_tiles = p.n_total / BN;
   const int kblocks = p.k_total / BK;
+  // row blocks per chunk: about 48 MB of A rows (16-bit operands)
+  const int m_chunk = max(1, (48 << 20) / (TILE_M * p.k_total * 2));
   // up: bf16 x times bf16 W13; down: fp16 h times fp16 W2
   constexpr uint32_t IDESC = umma_idesc_f32acc(TILE_M, BN, kMode == kUp ? 1u : 0u);
 
@@ -266,7 +276,7 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
         tph ^= 1u;
       }
       if (tile < 0 || p.stall) break;
-      const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, tile, rank);
+      const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, m_chunk, tile, rank);
       const int b_row = c.g * p.n_total + c.n0 + rank * C::B_ROWS;
       bool ok = true;
       for (int kb = 0; kb < kblocks; ++kb) {
@@ -368,7 +378,7 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
         tph ^= 1u;
       }
       if (tile < 0) break;
-      const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, tile, rank);
+      const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, m_chunk, tile, rank);
       if (!mbar_wait(&s.tfull[acc], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
       bool valid = row < c.rows;

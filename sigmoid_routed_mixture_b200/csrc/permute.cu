@@ -151,81 +151,105 @@ __global__ void __launch_bounds__(pm::THREADS)
   }
 }
 
-// Small batches (n <= SMALL_N assignments: decode, 4096 tokens at top-4): the same histogram ->
-// scan -> stable scatter in ONE CTA, so the permutation costs one launch.
+// Small batches (n <= SMALL_N assignments: decode, 4096 tokens at top-4): the same
+// histogram -> scan -> stable scatter in ONE CTA, so the permutation costs one
+// launch.  Warp w owns the contiguous assignments [w*S*32, (w+1)*S*32) (S steps
+// of 32) and keeps them in registers:
+//   1) each warp counts its segment per expert (warp matches; one writer per
+//      expert per step, so no atomics);
+//   2) per expert, an exclusive scan over the warps in order, offset by the
+//      expert's first row (exclusive scan of the totals over the experts);
+//   3) each warp walks its segment again and writes every entry to its
+//      expert's running position: ascending entries keep ascending positions.
 namespace pm {
 constexpr int SMALL_THREADS = 1024;
 constexpr int SMALL_WARPS = SMALL_THREADS / 32;
 constexpr int SMALL_N = 16384;
+constexpr int SMALL_STEPS = SMALL_N / SMALL_THREADS;  // 32-entry steps per warp
 }  // namespace pm
 
 __global__ void __launch_bounds__(pm::SMALL_THREADS)
     permute_small_kernel(const int32_t *__restrict__ idx, int n, int E, int T, int has_shared,
                          int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                          int32_t *__restrict__ sorted, int *err) {
-  __shared__ int hist[pm::MAX_E];
-  __shared__ int scan[pm::MAX_E];
-  __shared__ int cursor[pm::MAX_E];
-  __shared__ int wcnt[pm::SMALL_WARPS][pm::MAX_E];
+  __shared__ int whist[pm::SMALL_WARPS][pm::MAX_E];  // counts, then running positions
+  __shared__ int wsum[pm::MAX_E / 32];
+  __shared__ int routed_total;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < pm::MAX_E; e += pm::SMALL_THREADS) hist[e] = 0;
-  __syncthreads();
-  for (int i = tid; i < n; i += pm::SMALL_THREADS) {
-    const int e = idx[i];
-    if (e < 0 || e >= E)
-      record_error(err, MOE_ERR_BAD_INDEX);
-    else
-      atomicAdd(&hist[e], 1);
+  for (int k = tid; k < pm::SMALL_WARPS * pm::MAX_E; k += pm::SMALL_THREADS) (&whist[0][0])[k] = 0;
+  const int steps = (n + pm::SMALL_THREADS - 1) / pm::SMALL_THREADS;
+  const int seg0 = warp * steps * 32;
+  int e_reg[pm::SMALL_STEPS];
+#pragma unroll
+  for (int j = 0; j < pm::SMALL_STEPS; ++j) {
+    const int i = seg0 + j * 32 + lane;
+    int e = -1;
+    if (j < steps && i < n) {
+      e = idx[i];
+      if (e < 0 || e >= E) {
+        record_error(err, MOE_ERR_BAD_INDEX);
+        e = -1;
+      }
+    }
+    e_reg[j] = e;
   }
   __syncthreads();
-  if (tid < pm::MAX_E) scan[tid] = hist[tid];
+  const unsigned lt_mask = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < pm::SMALL_STEPS; ++j) {
+    if (j >= steps) break;
+    const int e = e_reg[j];
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && __popc(same & lt_mask) == 0) whist[warp][e] += __popc(same);
+    __syncwarp();
+  }
   __syncthreads();
-  for (int d = 1; d < pm::MAX_E; d <<= 1) {  // inclusive Hillis-Steele scan
-    const int v = (tid < pm::MAX_E && tid >= d) ? scan[tid - d] : 0;
-    __syncthreads();
-    if (tid < pm::MAX_E) scan[tid] += v;
-    __syncthreads();
+  if (tid < pm::MAX_E) {  // 8 warps: one expert per thread
+    const int e = tid;
+    int run = 0;
+    for (int w = 0; w < pm::SMALL_WARPS; ++w) {
+      const int v = whist[w][e];
+      whist[w][e] = run;
+      run += v;
+    }
+    int incl = run;  // inclusive scan of the expert totals: within the warp, then across
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    asm volatile("bar.sync 1, %0;" ::"n"(pm::MAX_E));
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    const int excl = before + incl - run;
+    if (e < E) {
+      counts[e] = run;
+      offsets[e] = excl;
+      for (int w = 0; w < pm::SMALL_WARPS; ++w) whist[w][e] += excl;
+    }
+    if (e == pm::MAX_E - 1) routed_total = before + incl;
   }
-  if (tid < E) {
-    const int excl = scan[tid] - hist[tid];
-    counts[tid] = hist[tid];
-    offsets[tid] = excl;
-    cursor[tid] = excl;
-  }
+  __syncthreads();
+  const int routed = routed_total;
   if (tid == 0) {
-    const int routed = scan[pm::MAX_E - 1];
     counts[E] = has_shared ? T : 0;
     offsets[E] = routed;
     offsets[E + 1] = routed + (has_shared ? T : 0);
   }
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = 0; base < n; base += pm::SMALL_THREADS) {
-    for (int k = tid; k < pm::SMALL_WARPS * pm::MAX_E; k += pm::SMALL_THREADS) (&wcnt[0][0])[k] = 0;
-    __syncthreads();
-    const int i = base + tid;
-    int e = i < n ? idx[i] : -1;
-    if (e >= E) e = -1;
+#pragma unroll
+  for (int j = 0; j < pm::SMALL_STEPS; ++j) {
+    if (j >= steps) break;
+    const int e = e_reg[j];
     const unsigned same = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(same & lt_mask);
-    if (e >= 0 && rank == 0) wcnt[warp][e] = __popc(same);
-    __syncthreads();
-    if (e >= 0) {
-      int before = 0;
-      for (int w = 0; w < warp; ++w) before += wcnt[w][e];
-      sorted[cursor[e] + before + rank] = i;
-    }
-    __syncthreads();
-    if (tid < E) {
-      int add = 0;
-      for (int w = 0; w < pm::SMALL_WARPS; ++w) add += wcnt[w][tid];
-      cursor[tid] += add;
-    }
-    __syncthreads();
+    if (e >= 0) sorted[whist[warp][e] + rank] = seg0 + j * 32 + lane;
+    __syncwarp();
+    if (e >= 0 && rank == 0) whist[warp][e] += __popc(same);
+    __syncwarp();
   }
-  if (has_shared) {
-    const int sbase = scan[pm::MAX_E - 1];
-    for (int t = tid; t < T; t += pm::SMALL_THREADS) sorted[sbase + t] = n + t;
-  }
+  if (has_shared)
+    for (int t = tid; t < T; t += pm::SMALL_THREADS) sorted[routed + t] = n + t;
 }
 
 cudaError_t launch_permute(const int32_t *idx, int T, int E, int K, int has_shared, int32_t *counts,

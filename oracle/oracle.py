@@ -12,6 +12,12 @@ selection-bias and renormalisation rules of the nnterp GLM-4.7-Flash / GLM-5
 pages (note "The mixture: sigmoid scores, a selection bias, renormalized
 weights").  Every function below names the equation it computes.
 
+The second part, ``dsa_oracle.c``, states the sparse attention's key selection:
+the indexer score of the same page's "All 43 steps" (S_I = sum_h w ReLU(q.k) /
+(sqrt(32) sqrt(128)), causal mask) and the top-k key selection of the nnterp
+glm_moe_dsa page ("Up to 2048 tokens the sparse attention is plain causal
+attention"), pinned in ``tests/test_dsa_oracle_pins.py``.
+
 Parity status: every function here is pinned by the not-gpu tests in
 ``tests/test_oracle_pins.py`` (closed forms, brute force, invariants, the
 page's parameter count and a hand-derived worked example); none is "parity
@@ -26,7 +32,7 @@ import subprocess
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "moe_oracle.c")
+_SRCS = [os.path.join(_HERE, "moe_oracle.c"), os.path.join(_HERE, "dsa_oracle.c")]
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
@@ -37,10 +43,12 @@ _vp = ctypes.c_void_p
 
 
 def build(force: bool = False) -> str:
-    """Compile moe_oracle.c into liboracle.so next to it (gcc, OpenMP)."""
-    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+    """Compile moe_oracle.c and dsa_oracle.c into liboracle.so next to them (gcc, OpenMP)."""
+    stale = not os.path.exists(_LIB_PATH) or any(
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(src) for src in _SRCS)
+    if force or stale:
         tmp = _LIB_PATH + ".tmp.%d" % os.getpid()
-        subprocess.check_call(["gcc", "-O3", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        subprocess.check_call(["gcc", "-O3", "-fopenmp", "-fPIC", "-shared", "-o", tmp] + _SRCS + ["-lm"])
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
@@ -64,6 +72,10 @@ def _load():
         lib.oracle_forward.restype = _int
         lib.oracle_forward.argtypes = [_i64, _i64, _i64, _i64, _i64, _int, _vp, _vp, _vp, _vp,
                                        _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp]
+        lib.oracle_dsa_scores.restype = _int
+        lib.oracle_dsa_scores.argtypes = [_i64, _i64, _i64, _i64, _i64, _vp, _vp, _vp, _vp]
+        lib.oracle_dsa_select.restype = _int
+        lib.oracle_dsa_select.argtypes = [_i64, _i64, _i64, _vp, _vp, _vp, _vp]
         _lib = lib
     return _lib
 
@@ -212,3 +224,43 @@ def forward(x, w1, w3, w2, ws1, ws3, ws2, idx, gate, tokens=None, has_shared=Tru
     if want_parts:
         return y, yr, ys, yk
     return y
+
+
+# ---------------------------------------------------------------- sparse-attention key selection
+# dsa_oracle.c: the indexer score of the "GLM-5 . MoE transformer block" page
+# (section "All 43 steps") and the top-k key selection of the nnterp glm_moe_dsa
+# page (section "Up to 2048 tokens the sparse attention is plain causal attention").
+
+def dsa_scores(q, k, w):
+    """Indexer scores in double: S[b,t,s] = sum_h w[b,t,h] ReLU(q[b,t,h].k[b,s]) / sqrt(NH*D)
+    for s <= S-T+t, -inf for the keys the causal mask hides.
+
+    q bf16 bits [B,T,NH,D], k bf16 bits [B,S,D], w float32 [B,T,NH] -> float64 [B,T,S]."""
+    q = _bf16(q)
+    k = _bf16(k)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    B, T, NH, D = q.shape
+    S = k.shape[1]
+    assert k.shape == (B, S, D) and w.shape == (B, T, NH)
+    out = np.empty((B, T, S), dtype=np.float64)
+    _check(_load().oracle_dsa_scores(B, T, S, NH, D, _p(q), _p(k), _p(w), _p(out)), "dsa_scores")
+    return out
+
+
+def dsa_select(scores, topk: int):
+    """The first min(topk, S) keys of each row in (score descending, index ascending)
+    order, listed in ascending key index.
+
+    scores float64 [..., S] -> (sel int32 [..., n_sel], kth float64 [...], next float64 [...]):
+    kth is the last taken key's score, next the first left out (-inf when all are taken)."""
+    scores = np.ascontiguousarray(scores, dtype=np.float64)
+    lead = scores.shape[:-1]
+    S = scores.shape[-1]
+    R = int(np.prod(lead)) if lead else 1
+    n_sel = min(int(topk), S)
+    sel = np.empty((R, n_sel), dtype=np.int32)
+    kth = np.empty((R,), dtype=np.float64)
+    nxt = np.empty((R,), dtype=np.float64)
+    _check(_load().oracle_dsa_select(R, S, int(topk), _p(scores), _p(sel), _p(kth), _p(nxt)),
+           "dsa_select")
+    return sel.reshape(lead + (n_sel,)), kth.reshape(lead), nxt.reshape(lead)

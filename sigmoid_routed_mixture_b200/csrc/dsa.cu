@@ -1,0 +1,580 @@
+// dsa.cu -- the sparse attention's key selection ("lightning indexer"):
+// indexer scores on the tensor cores, then a per-query top-k.
+//
+// Definition ("GLM-5 . MoE transformer block", open model atlas, section "All
+// 43 steps", indexer equations):
+//     S[t,s] = 1/(sqrt(NH) sqrt(D)) * sum_h w[t,h] * ReLU(q[t,h,:] . k[s,:]),
+// causal (query t of a sequence sits at position S - T + t), and each query
+// keeps the min(topk, S) best keys (nnterp glm_moe_dsa page, section "Up to 2048
+// tokens the sparse attention is plain causal attention").
+//
+// 1) dsa_plan_kernel: lists the work units (query block, chunk of key tiles)
+//    that the causal mask leaves, largest first.
+// 2) dsa_score_kernel: persistent, warp-specialised.  One tcgen05.mma tile is
+//    128 keys (M, the A operand) x 256 (query, head) rows (N, the B operand):
+//    QB = 256 / NH queries of all their heads, so every head's dot product of
+//    a key lands in that key's TMEM lane and the head sum happens inside one
+//    thread (no cross-lane reduction).  The query block stays in shared memory
+//    for a unit of up to KCH key tiles that stream through a TMA ring; two TMEM
+//    accumulators let the epilogue (ReLU, weight, head sum, store) overlap the
+//    next tile's MMAs.  Roles: warp 0 TMA producer and unit fetch, warp 1 TMEM
+//    allocation and single-thread MMA issue, warps 2-9 epilogue.
+// 3) dsa_topk_kernel: one CTA per query row: radix select of the topk-th score
+//    (4 passes of 8 bits over order-preserving integer keys, values cached in
+//    registers), then an ordered compaction that lists the selection in
+//    ascending key index (equal scores: lower index first).
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace srm {
+
+namespace dsa {
+constexpr int KT = 128;            // keys per tile (MMA M)
+constexpr int QN = 256;            // (query, head) rows per tile (MMA N)
+constexpr int KCH = 16;            // key tiles per work unit
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr int RING = 4;            // unit ring entries
+constexpr int MAX_SMEM = 232448;   // 227 KB dynamic shared memory per CTA
+
+template <int D>
+struct Cfg {
+  static constexpr int KB = D / 64;                  // 64-element k-blocks
+  static constexpr int Q_BYTES = QN * D * 2;         // one query block
+  static constexpr int K_BYTES = KT * D * 2;         // one key tile
+  static constexpr int K_STAGES = D == 128 ? 3 : 6;
+  static constexpr int DATA_BYTES = 2 * Q_BYTES + K_STAGES * K_BYTES;
+};
+
+struct Smem {
+  uint64_t kfull[6], kempty[6];
+  uint64_t qfull[2], qempty[2];
+  uint64_t tfull[2], tempty[2];
+  uint64_t ufull[RING], uempty[RING];
+  uint64_t drain;
+  int4 ring[RING];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+constexpr size_t smem_bytes() {
+  return 1024 + Cfg<D>::DATA_BYTES + sizeof(Smem);
+}
+static_assert(smem_bytes<128>() <= MAX_SMEM, "score kernel shared memory");
+static_assert(smem_bytes<64>() <= MAX_SMEM, "score kernel shared memory");
+}  // namespace dsa
+
+// key tiles query block qb needs (its last query sees keys 0 .. S - T + t_last)
+__host__ __device__ __forceinline__ int dsa_key_tiles(int qb, int qbs, int T, int S) {
+  const int t_last = min(T, (qb + 1) * qbs) - 1;
+  return (S - T + t_last) / dsa::KT + 1;
+}
+
+int dsa_units_bound(int T, int S, int n_heads) {
+  const int qbs = dsa::QN / n_heads;
+  const int nqb = (T + qbs - 1) / qbs;
+  const int nkt = (S + dsa::KT - 1) / dsa::KT;
+  return nqb * ((nkt + dsa::KCH - 1) / dsa::KCH);
+}
+
+// ---------------------------------------------------------------- 1) plan
+
+// units[i] = (qb, kc): query blocks in descending order (the most keys
+// first), each split into ceil(tiles / KCH) chunks.  ctl[0] = 0 (the unit
+// counter of the score kernel), ctl[1] = number of (qb, kc) entries.
+__global__ void __launch_bounds__(1024)
+    dsa_plan_kernel(int T, int S, int qbs, int2 *__restrict__ units, int *ctl) {
+  __shared__ int wsum[32];
+  __shared__ int base_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nqb = (T + qbs - 1) / qbs;
+  if (tid == 0) base_s = 0;
+  __syncthreads();
+  for (int i0 = 0; i0 < nqb; i0 += 1024) {
+    const int i = i0 + tid;
+    const int qb = nqb - 1 - i;
+    const int n = i < nqb ? (dsa_key_tiles(qb, qbs, T, S) + dsa::KCH - 1) / dsa::KCH : 0;
+    int incl = n;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int before = base_s;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    const int off = before + incl - n;
+    for (int kc = 0; kc < n; ++kc) units[off + kc] = make_int2(qb, kc);
+    __syncthreads();
+    if (tid == 1023) base_s = off + n;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    ctl[0] = 0;
+    ctl[1] = base_s;
+  }
+}
+
+// ---------------------------------------------------------------- 2) scores
+
+template <int NH, int D>
+__global__ void __launch_bounds__(dsa::THREADS, 1)
+    dsa_score_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                     const __grid_constant__ CUtensorMap tmap_k, const float *__restrict__ w,
+                     float *__restrict__ scores, const int2 *__restrict__ units, int *ctl, int B,
+                     int T, int S, float scale, int *err) {
+  using namespace dsa;
+  using C = Cfg<D>;
+  constexpr int QB = QN / NH;          // queries per tile
+  constexpr int QW = QB / 2;           // queries per epilogue warp
+  constexpr int CPQ = NH / 32;         // 32-column TMEM loads per query
+  constexpr uint32_t IDESC = umma_idesc_f32acc(KT, QN, 1u);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  uint8_t *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t *sQ = base;                       // 2 query blocks
+  uint8_t *sK = base + 2 * C::Q_BYTES;      // K_STAGES key tiles
+  Smem &s = *reinterpret_cast<Smem *>(base + C::DATA_BYTES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int *counter = ctl;
+  const int64_t n_units = static_cast<int64_t>(ctl[1]) * B;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::K_STAGES; ++i) {
+      mbar_init(&s.kfull[i], 1);
+      mbar_init(&s.kempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.qfull[i], 1);
+      mbar_init(&s.qempty[i], 1);
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], EPI_WARPS);
+    }
+    for (int i = 0; i < RING; ++i) {
+      mbar_init(&s.ufull[i], 1);
+      mbar_init(&s.uempty[i], 1 + EPI_WARPS);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_k);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, 2 * QN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  volatile int *abort_flag = &s.abort_flag;
+
+  // loads in flight at an abort: the last issued phase of every key stage and
+  // query buffer (a slot is refilled only after its previous load was consumed)
+  int k_last[6], q_last[2];
+#pragma unroll
+  for (int i = 0; i < 6; ++i) k_last[i] = -1;
+  q_last[0] = q_last[1] = -1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t kstage = 0, kphase = 0;
+    int n_unit = 0;
+    for (;;) {
+      const int slot = n_unit % RING;
+      if (!mbar_wait(&s.uempty[slot], ((n_unit / RING) & 1) ^ 1u, abort_flag, err)) break;
+      int64_t u = -1;
+      if (lane == 0) u = atomicAdd(counter, 1);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      int4 e = make_int4(-1, 0, 0, 0);
+      if (u < n_units) {
+        const int2 ent = units[u / B];
+        const int b = static_cast<int>(u % B);
+        const int kt0 = ent.y * KCH;
+        const int kt1 = min(dsa_key_tiles(ent.x, QB, T, S), kt0 + KCH);
+        e = make_int4(b, ent.x, kt0, kt1);
+      }
+      if (lane == 0) {
+        s.ring[slot] = e;
+        mbar_arrive(&s.ufull[slot]);
+      }
+      __syncwarp();
+      ++n_unit;
+      if (e.x < 0) break;
+      // the unit's query block
+      const int qbuf = (n_unit - 1) & 1;
+      if (!mbar_wait(&s.qempty[qbuf], (((n_unit - 1) >> 1) & 1) ^ 1u, abort_flag, err)) break;
+      if (lane == 0) {
+        uint8_t *dst = sQ + qbuf * C::Q_BYTES;
+        mbar_arrive_expect_tx(&s.qfull[qbuf], C::Q_BYTES);
+        const int row0 = (e.x * T + e.y * QB) * NH;
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_2d(dst + kb * (QN * 128), &tmap_q, &s.qfull[qbuf], kb * 64, row0);
+      }
+      q_last[qbuf] = ((n_unit - 1) >> 1) & 1;
+      __syncwarp();
+      // its key tiles
+      bool ok = true;
+      for (int kt = e.z; kt < e.w; ++kt) {
+        if (!mbar_wait(&s.kempty[kstage], kphase ^ 1u, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          uint8_t *dst = sK + kstage * C::K_BYTES;
+          mbar_arrive_expect_tx(&s.kfull[kstage], C::K_BYTES);
+          const int row0 = e.x * S + kt * KT;
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_2d(dst + kb * (KT * 128), &tmap_k, &s.kfull[kstage], kb * 64, row0);
+        }
+        k_last[kstage] = static_cast<int>(kphase);
+        __syncwarp();
+        if (++kstage == static_cast<uint32_t>(C::K_STAGES)) {
+          kstage = 0;
+          kphase ^= 1u;
+        }
+      }
+      if (!ok) break;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t kstage = 0, kphase = 0;
+    int n_unit = 0, n_tile = 0;
+    bool ok = true;
+    while (ok) {
+      const int slot = n_unit % RING;
+      if (!mbar_wait(&s.ufull[slot], (n_unit / RING) & 1, abort_flag, err)) break;
+      const int4 e = s.ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.uempty[slot]);
+      const int qbuf = n_unit & 1;
+      const uint32_t qphase = (n_unit >> 1) & 1;
+      ++n_unit;
+      if (e.x < 0) break;
+      if (!mbar_wait(&s.qfull[qbuf], qphase, abort_flag, err)) break;
+      tc_fence_after();
+      const uint32_t q_addr = smem_addr(sQ + qbuf * C::Q_BYTES);
+      for (int kt = e.z; kt < e.w; ++kt, ++n_tile) {
+        const uint32_t acc = n_tile & 1;
+        if (!mbar_wait(&s.tempty[acc], ((n_tile >> 1) & 1) ^ 1u, abort_flag, err) ||
+            !mbar_wait(&s.kfull[kstage], kphase, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t k_addr = smem_addr(sK + kstage * C::K_BYTES);
+          const uint32_t d = tmem + acc * QN;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // k-step kk: 64-element k-block kk / 4 (its own swizzled region),
+            // 16 elements (32 bytes) in
+            const uint32_t off = (kk & 3) * 32;
+            umma_bf16(d, umma_desc_sw128(k_addr + (kk >> 2) * (KT * 128) + off),
+                      umma_desc_sw128(q_addr + (kk >> 2) * (QN * 128) + off), IDESC,
+                      kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s.kempty[kstage]);
+          umma_commit(&s.tfull[acc]);
+        }
+        __syncwarp();
+        if (++kstage == static_cast<uint32_t>(C::K_STAGES)) {
+          kstage = 0;
+          kphase ^= 1u;
+        }
+      }
+      if (ok && lane == 0) umma_commit(&s.qempty[qbuf]);
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // warp -> TMEM lane quarter q (keys q*32 .. q*32+31 of the tile) and query
+    // half hf (queries hf*QW .. hf*QW+QW-1 of the block)
+    const int q = warp & 3;
+    const int hf = (warp - 2) >> 2;
+    int n_unit = 0, n_tile = 0;
+    float wr[QW * NH];  // this warp's queries' head weights (the same in every lane)
+    for (;;) {
+      const int slot = n_unit % RING;
+      if (!mbar_wait(&s.ufull[slot], (n_unit / RING) & 1, abort_flag, err)) break;
+      const int4 e = s.ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.uempty[slot]);
+      ++n_unit;
+      if (e.x < 0) break;
+      const int t0 = e.y * QB + hf * QW;  // first query of this warp
+#pragma unroll
+      for (int j = 0; j < QW; ++j) {
+        const int t = t0 + j;
+        const float4 *src =
+            reinterpret_cast<const float4 *>(w + (static_cast<int64_t>(e.x) * T + min(t, T - 1)) * NH);
+#pragma unroll
+        for (int h4 = 0; h4 < NH / 4; ++h4) {
+          const float4 v = t < T ? __ldg(src + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          wr[j * NH + 4 * h4 + 0] = v.x;
+          wr[j * NH + 4 * h4 + 1] = v.y;
+          wr[j * NH + 4 * h4 + 2] = v.z;
+          wr[j * NH + 4 * h4 + 3] = v.w;
+        }
+      }
+      bool ok = true;
+      for (int kt = e.z; kt < e.w; ++kt, ++n_tile) {
+        const uint32_t acc = n_tile & 1;
+        if (!mbar_wait(&s.tfull[acc], (n_tile >> 1) & 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int key = kt * KT + q * 32 + lane;
+        const uint32_t taddr = tmem + acc * QN + (static_cast<uint32_t>(q * 32) << 16);
+        float res[QW];
+#pragma unroll
+        for (int j = 0; j < QW; ++j) {
+          float a = 0.f;
+#pragma unroll
+          for (int c = 0; c < CPQ; ++c) {
+            uint32_t r[32];
+            tmem_ld32(taddr + (hf * QW + j) * NH + c * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              a = fmaf(wr[j * NH + c * 32 + i], fmaxf(__uint_as_float(r[i]), 0.f), a);
+          }
+          res[j] = a * scale;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.tempty[acc]);
+#pragma unroll
+        for (int j = 0; j < QW; ++j) {
+          const int t = t0 + j;
+          if (t < T && key <= S - T + t)
+            scores[(static_cast<int64_t>(e.x) * T + t) * S + key] = res[j];
+        }
+      }
+      if (!ok) break;
+    }
+  }
+
+  __syncthreads();
+  if (s.abort_flag) {  // error path: let copies and MMAs in flight land first
+    if (warp == 0 && lane == 0) {
+      for (int i = 0; i < C::K_STAGES; ++i)
+        if (k_last[i] >= 0) {
+          const uint32_t a = smem_addr(&s.kfull[i]);
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(a, static_cast<uint32_t>(k_last[i])) &&
+                 global_timer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      for (int i = 0; i < 2; ++i)
+        if (q_last[i] >= 0) {
+          const uint32_t a = smem_addr(&s.qfull[i]);
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(a, static_cast<uint32_t>(q_last[i])) &&
+                 global_timer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+    }
+    if (warp == 1 && lane == 0) {
+      umma_commit(&s.drain);
+      const uint32_t a = smem_addr(&s.drain);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(a, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * QN);
+  }
+}
+
+// ---------------------------------------------------------------- 3) top-k
+
+// Order-preserving integer key of a float: larger float -> larger key.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Block-wide exclusive prefix count of `flag` in thread order; returns the
+// count before this thread and writes the block total to *total.
+template <int NT>
+__device__ __forceinline__ int block_excl_count(bool flag, int *wtot, int *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned m = __ballot_sync(0xffffffffu, flag);
+  if (lane == 0) wtot[warp] = __popc(m);
+  __syncthreads();
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const int v = wtot[w];
+    before += w < warp ? v : 0;
+    all += v;
+  }
+  __syncthreads();
+  *total = all;
+  return before + __popc(m & ((1u << lane) - 1u));
+}
+
+// One CTA per query row.  Thread i holds keys i, i + NT, ... (VPT of them) of
+// the visible part of the row in registers.
+template <int NT, int VPT>
+__global__ void __launch_bounds__(NT)
+    dsa_topk_kernel(const float *__restrict__ scores, int T, int S, int n_sel,
+                    int32_t *__restrict__ sel) {
+  __shared__ int hist[256];
+  __shared__ int wtot[NT / 32];
+  __shared__ int pick[2];  // digit, keys above it
+  const int64_t row = blockIdx.x;
+  const int t = static_cast<int>(row % T);
+  const int n_vis = S - T + t + 1;  // keys this query sees
+  int32_t *out = sel + row * n_sel;
+  const int tid = threadIdx.x;
+  if (n_vis <= n_sel) {  // every visible key, then the lowest-index hidden ones
+    for (int j = tid; j < n_sel; j += NT) out[j] = j;
+    return;
+  }
+  const float *src = scores + row * S;
+  uint32_t v[VPT];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int idx = j * NT + tid;
+    v[j] = idx < n_vis ? order_key(src[idx]) : 0u;  // 0: below every real key
+  }
+  // radix select of the n_sel-th largest key, 8 bits at a time
+  uint32_t prefix = 0, pmask = 0;
+  int k_rem = n_sel;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += NT) hist[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int idx = j * NT + tid;
+      if (idx < n_vis && (v[j] & pmask) == prefix) atomicAdd(&hist[(v[j] >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (tid < 32) {  // digits 255 .. 0, eight per lane: find the one holding the k_rem-th key
+      int c[8], sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        c[i] = hist[255 - (tid * 8 + i)];
+        sum += c[i];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, incl, d);
+        if (tid >= d) incl += x;
+      }
+      int above = incl - sum;  // keys in higher digits than this lane's first
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (above < k_rem && k_rem <= above + c[i]) {
+          pick[0] = 255 - (tid * 8 + i);
+          pick[1] = above;
+        }
+        above += c[i];
+      }
+    }
+    __syncthreads();
+    const int digit = pick[0];
+    k_rem -= pick[1];
+    prefix |= static_cast<uint32_t>(digit) << shift;
+    pmask |= 255u << shift;
+    __syncthreads();
+  }
+  // prefix is the n_sel-th largest key; take every key above it and the first
+  // k_rem keys equal to it, in ascending index
+  int taken_before = 0, eq_before = 0;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    if (j * NT >= n_vis) break;
+    const int idx = j * NT + tid;
+    const bool valid = idx < n_vis;
+    const bool eq = valid && v[j] == prefix;
+    int eq_tot;
+    const int eq_rank = eq_before + block_excl_count<NT>(eq, wtot, &eq_tot);
+    const bool take = valid && (v[j] > prefix || (eq && eq_rank < k_rem));
+    int take_tot;
+    const int pos = taken_before + block_excl_count<NT>(take, wtot, &take_tot);
+    if (take && pos < n_sel) out[pos] = idx;
+    eq_before += eq_tot;
+    taken_before += take_tot;
+  }
+}
+
+// ---------------------------------------------------------------- launches
+
+int dsa_score_smem(int head_dim) {
+  return static_cast<int>(head_dim == 128 ? dsa::smem_bytes<128>() : dsa::smem_bytes<64>());
+}
+
+template <int NH, int D>
+static cudaError_t launch_score(const CUtensorMap &tq, const CUtensorMap &tk, const float *w,
+                                float *scores, const int2 *units, int *ctl, int64_t B, int T,
+                                int S, float scale, int *err, int num_sms, cudaStream_t stream) {
+  auto kern = dsa_score_kernel<NH, D>;
+  constexpr size_t smem = dsa::smem_bytes<D>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<num_sms, dsa::THREADS, smem, stream>>>(tq, tk, w, scores, units, ctl, static_cast<int>(B),
+                                                T, S, scale, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dsa_scores(const CUtensorMap &tq, const CUtensorMap &tk, const float *w,
+                              float *scores, int2 *units, int *ctl, int64_t B, int T, int S,
+                              int n_heads, int head_dim, float scale, int *err, int num_sms,
+                              cudaStream_t stream) {
+  const int qbs = dsa::QN / n_heads;
+  dsa_plan_kernel<<<1, 1024, 0, stream>>>(T, S, qbs, units, ctl);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+#define SRM_DSA_CASE(NH_, D_)                                                                    \
+  if (n_heads == NH_ && head_dim == D_)                                                        \
+    return launch_score<NH_, D_>(tq, tk, w, scores, units, ctl, B, T, S, scale, err, num_sms, \
+                                 stream);
+  SRM_DSA_CASE(32, 128)
+  SRM_DSA_CASE(64, 128)
+  SRM_DSA_CASE(128, 128)
+  SRM_DSA_CASE(32, 64)
+  SRM_DSA_CASE(64, 64)
+  SRM_DSA_CASE(128, 64)
+#undef SRM_DSA_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_dsa_topk(const float *scores, int64_t B, int T, int S, int topk, int32_t *sel,
+                            cudaStream_t stream) {
+  const int n_sel = min(topk, S);
+  const int64_t rows = B * T;
+  if (rows == 0) return cudaSuccess;
+  if (rows > 0x7fffffff) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(rows));
+  if (S <= 256 * 16)
+    dsa_topk_kernel<256, 16><<<grid, 256, 0, stream>>>(scores, T, S, n_sel, sel);
+  else if (S <= 1024 * 16)
+    dsa_topk_kernel<1024, 16><<<grid, 1024, 0, stream>>>(scores, T, S, n_sel, sel);
+  else if (S <= 512 * 64)
+    dsa_topk_kernel<512, 64><<<grid, 512, 0, stream>>>(scores, T, S, n_sel, sel);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace srm

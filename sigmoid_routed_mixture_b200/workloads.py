@@ -130,3 +130,43 @@ def torch_bf16_to_bits(t) -> np.ndarray:
     import torch
 
     return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ------------------------------------------------- sparse-attention key selection
+# Shapes of the GLM-5 indexer (config.json: index_n_heads 32, index_head_dim 128,
+# index_topk 2048).  Recipe (seed as listed): q [B, T, NH, D] and k [B, S, D] bf16
+# N(0, 1) (the keys leave a LayerNorm, the queries a normalised latent's
+# projection), w [B, T, NH] fp32 N(0, 1), drawn in that order from NumPy
+# default_rng(seed), fp32 -> bf16 RNE.  Prefill: T == S (4 sequences of 4096
+# tokens, the block's 16384-token batch); decode: one query per sequence over a
+# 32768-key cache.
+
+@dataclasses.dataclass(frozen=True)
+class DsaWorkload:
+    name: str
+    B: int
+    T: int
+    S: int
+    n_heads: int = 32
+    head_dim: int = 128
+    topk: int = 2048
+    seed: int = 2000
+
+    def replace(self, **kw) -> "DsaWorkload":
+        return dataclasses.replace(self, **kw)
+
+
+DSA_WORKLOADS = {
+    "dsa_tiny": DsaWorkload("dsa_tiny", B=2, T=300, S=300, topk=64, seed=2001),
+    "dsa_prefill": DsaWorkload("dsa_prefill", B=4, T=4096, S=4096, seed=2002),
+    "dsa_decode": DsaWorkload("dsa_decode", B=64, T=1, S=32768, seed=2003),
+}
+
+
+def dsa_inputs(w: DsaWorkload):
+    """(q bf16 bits [B,T,NH,D], k bf16 bits [B,S,D], w fp32 [B,T,NH]) on the host."""
+    rng = np.random.default_rng(w.seed)
+    q = f32_to_bf16_bits(rng.standard_normal((w.B, w.T, w.n_heads, w.head_dim), dtype=np.float32))
+    k = f32_to_bf16_bits(rng.standard_normal((w.B, w.S, w.head_dim), dtype=np.float32))
+    wt = rng.standard_normal((w.B, w.T, w.n_heads), dtype=np.float32)
+    return q, k, wt

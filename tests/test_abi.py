@@ -1,6 +1,6 @@
 """Host-side checks of the C ABI (no GPU needed): the library loads, exports
-every entry point include/srm_moe.h declares, sizes its workspace and rejects
-invalid arguments before any launch."""
+every entry point include/srm_moe.h and include/srm_dsa.h declare, sizes its
+workspaces and rejects invalid arguments before any launch."""
 import ctypes
 import os
 import re
@@ -8,6 +8,7 @@ import re
 import pytest
 
 from sigmoid_routed_mixture_b200 import build as B
+from sigmoid_routed_mixture_b200 import dsa
 from sigmoid_routed_mixture_b200 import moe
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -25,7 +26,7 @@ def declared_functions():
         if fn.endswith(".h"):
             src = open(os.path.join(ROOT, "include", fn)).read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-            names |= set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src))
+            names |= set(re.findall(r"\b((?:moe|dsa)_[a-z0-9_]+)\s*\(", src))
     return names
 
 
@@ -35,6 +36,7 @@ def test_exports_every_declared_symbol(L):
     for name in declared:
         assert hasattr(L, name), name
     assert set(moe.SYMBOLS) <= declared
+    assert set(dsa.SYMBOLS) <= declared and "dsa_select" in declared
 
 
 def test_status_strings(L):
@@ -102,3 +104,52 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(moe, "_lib", None)
     with pytest.raises(RuntimeError, match="not found"):
         moe.lib()
+
+
+# ---------------------------------------------------------------- key selection
+
+def dsa_cfg(**kw):
+    base = dict(B=2, T=64, S=64)
+    base.update(kw)
+    return dsa.Config(**base)
+
+
+def test_dsa_workspace_size(L):
+    dsa.lib()
+    small = dsa.workspace_bytes(dsa_cfg())
+    big = dsa.workspace_bytes(dsa_cfg(T=4096, S=4096, B=4))
+    assert big > small > 0
+    assert big >= 4 * 4096 * 4096 * 4  # room for the fp32 scores
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(n_heads=16), 2), (dict(head_dim=96), 2), (dict(T=0), 1), (dict(T=65, S=64), 1),
+    (dict(topk=0), 1), (dict(topk=70000), 2), (dict(S=40000, T=1), 2), (dict(B=-1), 1),
+])
+def test_dsa_invalid_configs_rejected(L, bad, code):
+    dsa.lib()
+    c = dsa_cfg(**bad).c()
+    assert L.dsa_workspace_size(ctypes.byref(c)) == 0
+    assert L.dsa_select(ctypes.byref(c), None, None, None, None, None, None, 0, None) == code
+
+
+def test_dsa_pointer_checks_before_launch(L):
+    dsa.lib()
+    c = dsa_cfg().c()
+    need = L.dsa_workspace_size(ctypes.byref(c))
+    ws = ctypes.c_void_p(0x100000)
+    p16 = ctypes.c_void_p(0x200000)
+    odd = ctypes.c_void_p(0x200008)  # 8-byte aligned only: q, k, w need 16
+    assert L.dsa_select(ctypes.byref(c), None, p16, p16, p16, None, ws, need, None) == 1
+    assert L.dsa_select(ctypes.byref(c), odd, p16, p16, p16, None, ws, need, None) == 3
+    assert L.dsa_select(ctypes.byref(c), p16, p16, p16, p16, None, ws, need - 1, None) == 4
+    assert L.dsa_scores(ctypes.byref(c), p16, p16, p16, None, ws, need, None) == 1
+    assert L.dsa_topk(ctypes.byref(c), p16, None, ws, need, None) == 1
+    assert L.dsa_select(ctypes.byref(c), p16, p16, p16, p16, None, ctypes.c_void_p(0x100010), need,
+                        None) == 3
+
+
+def test_dsa_no_sequences_is_a_no_op(L):
+    dsa.lib()
+    c = dsa_cfg(B=0).c()
+    assert L.dsa_select(ctypes.byref(c), None, None, None, None, None, None, 0, None) == 0

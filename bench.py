@@ -160,15 +160,20 @@ def cores():
 
 def measured_traffic(workload, kernel):
     """DRAM bytes per launch from a committed ncu capture (profiles/dram_traffic_glm5.md),
-    or None when the GEMM sources changed since it was taken."""
+    or None when the GEMM sources (grouped_gemm.cu, common.cuh, the GemmArgs block
+    of kernels.h) changed since it was taken."""
     import hashlib
 
     path = os.path.join(ROOT, "profiles", "dram_traffic_glm5.md")
     if not os.path.exists(path):
         return None
     h = hashlib.md5()
-    for f in ("grouped_gemm.cu", "common.cuh", "kernels.h"):
-        h.update(open(os.path.join(ROOT, "sigmoid_routed_mixture_b200", "csrc", f), "rb").read())
+    csrc = os.path.join(ROOT, "sigmoid_routed_mixture_b200", "csrc")
+    for f in ("grouped_gemm.cu", "common.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    hdr = open(os.path.join(csrc, "kernels.h"), "rb").read()
+    a = hdr.index(b"struct GemmArgs {")
+    h.update(hdr[a:hdr.index(b"};", a) + 2])  # the GEMM's argument block, not the other declarations
     for line in open(path):
         parts = line.split()
         if len(parts) == 5 and parts[0] == "traffic" and parts[1] == workload and parts[2] == kernel:
@@ -284,6 +289,225 @@ def workload_config(w, args):
                 (w.E + 1) * 3 * w.H * w.I * 2 / 1e9)}
 
 
+# ------------------------------------------------------------------ key selection workloads
+
+DSA_METRIC = "DSA key selections/s (GLM-5 indexer, 32 heads x 128, top-2048, 1 B200)"
+DSA_UNIT = "queries/s"
+DSA_KERNELS_PER_STEP = 3  # plan, scores, top-k
+
+
+def dsa_visible_pairs(w):
+    """(query, key) pairs the causal mask leaves: sum over queries of S - T + t + 1."""
+    return w.B * (w.T * (w.S - w.T) + w.T * (w.T + 1) // 2)
+
+
+def dsa_oracle_sample(w, n, inputs):
+    """A bounded oracle sample: n consecutive queries of sequence 0 around the
+    middle of the prompt (prefill), or the single query of n sequences (decode).
+    Returns (seconds, queries)."""
+    from oracle import oracle as O
+
+    q, k, wt = inputs
+    if w.T == 1:
+        n = min(n, w.B)
+        t0 = time.time()
+        O.dsa_select(O.dsa_scores(q[:n], k[:n], wt[:n]), w.topk)
+        return time.time() - t0, n
+    n = min(n, w.T)
+    p = min(w.T - 1, (w.S - w.T) + w.T // 2 + n // 2)  # position of the last sampled query
+    t_hi = p - (w.S - w.T)
+    qs, ws_ = q[:1, t_hi - n + 1:t_hi + 1], wt[:1, t_hi - n + 1:t_hi + 1]
+    t0 = time.time()
+    O.dsa_select(O.dsa_scores(qs, k[:1, :p + 1], ws_), w.topk)
+    return time.time() - t0, n
+
+
+def dsa_line_config(w, world):
+    return {"workload": w.name, "sequences": w.B, "queries_per_sequence": w.T, "keys_per_sequence": w.S,
+            "index_heads": w.n_heads, "index_head_dim": w.head_dim, "topk": w.topk,
+            "global_batch": w.B * w.T * world, "parallelism": "replicas x%d" % world,
+            "l2": "inputs larger than L2: q %.0f MB, keys %.0f MB and scores %.0f MB per step against 126 MB" % (
+                w.B * w.T * w.n_heads * w.head_dim * 2 / 1e6, w.B * w.S * w.head_dim * 2 / 1e6,
+                dsa_visible_pairs(w) * 4 / 1e6)}
+
+
+def run_dsa_reference(args, rank):
+    if rank != 0:
+        return
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores()))
+    from oracle import oracle as O
+
+    O.build()
+    w = W.DSA_WORKLOADS[args.workload]
+    n = args.ref_tokens or 2 * cores()
+    inputs = W.dsa_inputs(w)
+    for _ in range(args.warmup):
+        dsa_oracle_sample(w, n, inputs)
+    secs, nq = 0.0, 0
+    for _ in range(args.steps):
+        s_, q_ = dsa_oracle_sample(w, n, inputs)
+        secs += s_
+        nq += q_
+    value = nq / secs
+    sample = "scores + top-%d of %d queries per step (double-precision C oracle, OpenMP)" % (w.topk, nq // args.steps)
+    line = {"impl": "reference", "metric": DSA_METRIC, "value": value, "unit": DSA_UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": dsa_line_config(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": DSA_UNIT, "cores": int(os.environ["OMP_NUM_THREADS"]),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": DSA_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_dsa(args, world, rank, dist, dev):
+    import torch
+
+    from sigmoid_routed_mixture_b200 import dsa, moe
+
+    w = W.DSA_WORKLOADS[args.workload]
+    q, k, wt = W.dsa_inputs(w if rank == 0 else w.replace(seed=w.seed + 7919 * rank))
+    cfg = dsa.Config(w.B, w.T, w.S, w.n_heads, w.head_dim, w.topk)
+    ws = dsa.workspace(cfg, device=dev)
+    q_dev = torch.from_numpy(q.view(np.int16)).to(dev).view(torch.bfloat16)
+    k_dev = torch.from_numpy(k.view(np.int16)).to(dev).view(torch.bfloat16)
+    w_dev = torch.from_numpy(wt).to(dev)
+    scores = torch.empty((w.B, w.T, w.S), dtype=torch.float32, device=dev)
+    sel = torch.empty((w.B, w.T, cfg.n_sel), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dsa.scores(cfg, q_dev, k_dev, w_dev, ws, out=scores)
+        if ev is not None:
+            ev[1].record(stream)
+        dsa.topk(cfg, scores, ws, out=sel)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if moe.device_error(ws) != 0:
+        raise RuntimeError("device error during warm-up")
+    graph = None
+    if not args.eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(args.warmup):
+            graph.replay()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(torch.cuda.current_device())
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    e0.record(stream)
+    for i in range(args.steps):
+        if graph is not None:
+            graph.replay()
+        else:
+            step(evs[i])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    total_ms = e0.elapsed_time(e1)
+    if graph is not None:  # stage breakdown from host-launched steps after the timed ones
+        for i in range(args.steps):
+            step(evs[i])
+        torch.cuda.synchronize()
+    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(2)] for i in range(args.steps)])
+    t_max = max_over_ranks(total_ms, dist, dev)
+    value = w.B * w.T * world * args.steps / (t_max / 1e3)
+
+    # end to end: q, k, w from pinned host memory in, the selection out, every step
+    hq = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(k.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hw = torch.from_numpy(wt).pin_memory()
+    hsel = torch.empty(tuple(sel.shape), dtype=torch.int32).pin_memory()
+
+    def e2e_step():
+        q_dev.copy_(hq, non_blocking=True)
+        k_dev.copy_(hk, non_blocking=True)
+        w_dev.copy_(hw, non_blocking=True)
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
+        hsel.copy_(sel, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    if moe.device_error(ws) != 0:
+        raise RuntimeError("device error during the timed steps")
+
+    pk = peaks()
+    pairs = dsa_visible_pairs(w)
+    f_score = 2.0 * pairs * w.n_heads * w.head_dim
+    b_in = w.B * w.T * w.n_heads * w.head_dim * 2 + w.B * w.S * w.head_dim * 2 + w.B * w.T * w.n_heads * 4
+    b_sel = w.B * w.T * cfg.n_sel * 4
+    b_score = b_in + pairs * 4       # inputs + the scores it writes
+    b_topk = pairs * 4 + b_sel       # the visible scores read + the selection written
+    mean = stage.mean(axis=0)
+    ridge = pk["tflops"] * 1e12 / (pk["hbm"] * 1e9)
+    kernels = [("dsa_score_kernel", f_score, b_score, mean[0]), ("dsa_topk_kernel", 0.0, b_topk, mean[1])]
+    name, f, by, ms = max(kernels, key=lambda x: x[3])
+    if f > 0 and f / by > ridge:
+        roof = {"kernel": name, "bound": "tensor", "achieved": f / (ms / 1e3) / 1e12, "peak": pk["tflops"],
+                "unit": "TFLOP/s", "peak_kind": "burst bf16 (cuBLAS), " + pk["source"],
+                "algorithmic_per_launch": f}
+    else:
+        roof = {"kernel": name, "bound": "hbm", "achieved": by / (ms / 1e3) / 1e9, "peak": pk["hbm"],
+                "unit": "GB/s", "peak_kind": "copy bandwidth, " + pk["source"], "algorithmic_per_launch": by}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = measured_traffic(w.name, name)
+    step_s = t_max / 1e3 / args.steps
+    t_roof = max(f_score / (pk["tflops"] * 1e12), (b_in + b_sel) / (pk["hbm"] * 1e9))
+    line = {
+        "metric": DSA_METRIC, "value": value, "unit": DSA_UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded q, k, w of the GLM-5 indexer shapes)",
+        "config": dsa_line_config(w, world), "roofline": roof,
+        "block_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof / step_s, "f_alg_tflop": f_score / 1e12,
+                           "b_alg_gb": (b_in + b_sel) / 1e9},
+        "stage_ms": {"scores": float(mean[0]), "topk": float(mean[1])},
+        "stage_roofline": {
+            "scores": {"bound": "tensor" if f_score / b_score > ridge else "hbm",
+                       "frac": (f_score / (mean[0] / 1e3) / 1e12 / pk["tflops"]) if f_score / b_score > ridge
+                       else (b_score / (mean[0] / 1e3) / 1e9 / pk["hbm"])},
+            "topk": {"bound": "hbm", "frac": b_topk / (mean[1] / 1e3) / 1e9 / pk["hbm"]}},
+        "launch": "cuda graph replay" if graph is not None else "eager",
+        "e2e": {"value": w.B * w.T * world * args.e2e_steps / (e2e_ms / 1e3), "unit": DSA_UNIT,
+                "h2d_bytes_per_step": int(b_in), "d2h_bytes_per_step": int(b_sel), "steps": args.e2e_steps},
+        "gpu_launches": DSA_KERNELS_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        os.environ.setdefault("OMP_NUM_THREADS", str(cores()))
+        from oracle import oracle as O
+
+        O.build()
+        secs, nq = dsa_oracle_sample(w, args.cpu_tokens or 2 * cores(), (q, k, wt))
+        line["cpu_baseline"] = {"value": nq / secs, "unit": DSA_UNIT, "cores": int(os.environ["OMP_NUM_THREADS"]),
+                                "kind": "oracle",
+                                "sample": "scores + top-%d of %d queries (double-precision C oracle, OpenMP), "
+                                          "%.1f s" % (w.topk, nq, secs)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ our arm
 
 def main():
@@ -291,7 +515,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="glm5_prefill", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="glm5_prefill",
+                    choices=sorted(W.WORKLOADS) + sorted(W.DSA_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=0)
     ap.add_argument("--cpu-tokens", type=int, default=0)
@@ -308,8 +533,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    is_dsa = args.workload in W.DSA_WORKLOADS
     if args.impl == "reference":
-        run_reference(args, rank)
+        (run_dsa_reference if is_dsa else run_reference)(args, rank)
         return
 
     import torch
@@ -326,6 +552,11 @@ def main():
         torch.cuda.set_device(0)
     from sigmoid_routed_mixture_b200 import moe
 
+    if is_dsa:
+        run_dsa(args, world, rank, dist, torch.device("cuda", torch.cuda.current_device()))
+        if dist is not None:
+            dist.destroy_process_group()
+        return
     w = W.WORKLOADS[args.workload]
     if args.tokens:
         w = w.replace(T=args.tokens)

@@ -40,17 +40,23 @@ constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int RING = 4;            // unit ring entries
 constexpr int MAX_SMEM = 232448;   // 227 KB dynamic shared memory per CTA
 
+constexpr int KSTAGE_BYTES = KT * 64 * 2;  // one 64-element k-block of a key tile (16 KB)
+constexpr int W_BYTES = QN * 4;            // the head weights of one query block (fp32)
+constexpr int MAX_KSTAGES = 8;
+
 template <int D>
 struct Cfg {
-  static constexpr int KB = D / 64;                  // 64-element k-blocks
-  static constexpr int Q_BYTES = QN * D * 2;         // one query block
-  static constexpr int K_BYTES = KT * D * 2;         // one key tile
-  static constexpr int K_STAGES = D == 128 ? 3 : 6;
-  static constexpr int DATA_BYTES = 2 * Q_BYTES + K_STAGES * K_BYTES;
+  static constexpr int KB = D / 64;             // 64-element k-blocks per key tile
+  static constexpr int Q_BYTES = QN * D * 2;    // one query block
+  static constexpr int K_STAGES =
+      (MAX_SMEM - 2048 - 2 * Q_BYTES - 2 * W_BYTES) / KSTAGE_BYTES < MAX_KSTAGES
+          ? (MAX_SMEM - 2048 - 2 * Q_BYTES - 2 * W_BYTES) / KSTAGE_BYTES
+          : MAX_KSTAGES;
+  static constexpr int DATA_BYTES = 2 * Q_BYTES + K_STAGES * KSTAGE_BYTES + 2 * W_BYTES;
 };
 
 struct Smem {
-  uint64_t kfull[6], kempty[6];
+  uint64_t kfull[MAX_KSTAGES], kempty[MAX_KSTAGES];
   uint64_t qfull[2], qempty[2];
   uint64_t tfull[2], tempty[2];
   uint64_t ufull[RING], uempty[RING];
@@ -66,6 +72,18 @@ constexpr size_t smem_bytes() {
 }
 static_assert(smem_bytes<128>() <= MAX_SMEM, "score kernel shared memory");
 static_assert(smem_bytes<64>() <= MAX_SMEM, "score kernel shared memory");
+static_assert(Cfg<128>::K_STAGES >= 4, "key ring depth");
+
+// Untiled bulk copy of `bytes` contiguous bytes global -> shared, completing on
+// `bar` (both addresses 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load_1d(void *dst, const void *src, uint32_t bytes,
+                                             uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
 }  // namespace dsa
 
 // key tiles query block qb needs (its last query sees keys 0 .. S - T + t_last)
@@ -137,8 +155,9 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   uint8_t *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t *sQ = base;                       // 2 query blocks
-  uint8_t *sK = base + 2 * C::Q_BYTES;      // K_STAGES key tiles
+  uint8_t *sQ = base;                                   // 2 query blocks
+  uint8_t *sK = base + 2 * C::Q_BYTES;                  // K_STAGES key k-blocks
+  float *sW = reinterpret_cast<float *>(sK + C::K_STAGES * KSTAGE_BYTES);  // 2 x [QB][NH]
   Smem &s = *reinterpret_cast<Smem *>(base + C::DATA_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -152,7 +171,7 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.qfull[i], 1);
-      mbar_init(&s.qempty[i], 1);
+      mbar_init(&s.qempty[i], 1 + EPI_WARPS);  // the MMAs and the epilogue warps (weights)
       mbar_init(&s.tfull[i], 1);
       mbar_init(&s.tempty[i], EPI_WARPS);
     }
@@ -178,9 +197,9 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
 
   // loads in flight at an abort: the last issued phase of every key stage and
   // query buffer (a slot is refilled only after its previous load was consumed)
-  int k_last[6], q_last[2];
+  int k_last[MAX_KSTAGES], q_last[2];
 #pragma unroll
-  for (int i = 0; i < 6; ++i) k_last[i] = -1;
+  for (int i = 0; i < MAX_KSTAGES; ++i) k_last[i] = -1;
   q_last[0] = q_last[1] = -1;
 
   if (warp == 0) {
@@ -208,39 +227,42 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
       __syncwarp();
       ++n_unit;
       if (e.x < 0) break;
-      // the unit's query block
+      // the unit's query block and its queries' head weights (valid rows only)
       const int qbuf = (n_unit - 1) & 1;
       if (!mbar_wait(&s.qempty[qbuf], (((n_unit - 1) >> 1) & 1) ^ 1u, abort_flag, err)) break;
       if (lane == 0) {
+        const int t0 = e.y * QB;
+        const uint32_t w_bytes = static_cast<uint32_t>(min(QB, T - t0) * NH * 4);
         uint8_t *dst = sQ + qbuf * C::Q_BYTES;
-        mbar_arrive_expect_tx(&s.qfull[qbuf], C::Q_BYTES);
-        const int row0 = (e.x * T + e.y * QB) * NH;
+        mbar_arrive_expect_tx(&s.qfull[qbuf], C::Q_BYTES + w_bytes);
+        const int row0 = (e.x * T + t0) * NH;
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_2d(dst + kb * (QN * 128), &tmap_q, &s.qfull[qbuf], kb * 64, row0);
+        bulk_load_1d(sW + qbuf * QN, w + static_cast<int64_t>(e.x * T + t0) * NH, w_bytes,
+                     &s.qfull[qbuf]);
       }
       q_last[qbuf] = ((n_unit - 1) >> 1) & 1;
       __syncwarp();
-      // its key tiles
+      // its key tiles, one 64-element k-block per stage
       bool ok = true;
-      for (int kt = e.z; kt < e.w; ++kt) {
-        if (!mbar_wait(&s.kempty[kstage], kphase ^ 1u, abort_flag, err)) {
-          ok = false;
-          break;
-        }
-        if (lane == 0) {
-          uint8_t *dst = sK + kstage * C::K_BYTES;
-          mbar_arrive_expect_tx(&s.kfull[kstage], C::K_BYTES);
-          const int row0 = e.x * S + kt * KT;
+      for (int kt = e.z; kt < e.w && ok; ++kt) {
 #pragma unroll
-          for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_2d(dst + kb * (KT * 128), &tmap_k, &s.kfull[kstage], kb * 64, row0);
-        }
-        k_last[kstage] = static_cast<int>(kphase);
-        __syncwarp();
-        if (++kstage == static_cast<uint32_t>(C::K_STAGES)) {
-          kstage = 0;
-          kphase ^= 1u;
+        for (int kb = 0; kb < C::KB; ++kb) {
+          if (!mbar_wait(&s.kempty[kstage], kphase ^ 1u, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&s.kfull[kstage], KSTAGE_BYTES);
+            tma_load_2d(sK + kstage * KSTAGE_BYTES, &tmap_k, &s.kfull[kstage], kb * 64, e.x * S + kt * KT);
+          }
+          k_last[kstage] = static_cast<int>(kphase);
+          __syncwarp();
+          if (++kstage == static_cast<uint32_t>(C::K_STAGES)) {
+            kstage = 0;
+            kphase ^= 1u;
+          }
         }
       }
       if (!ok) break;
@@ -263,34 +285,38 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
       if (!mbar_wait(&s.qfull[qbuf], qphase, abort_flag, err)) break;
       tc_fence_after();
       const uint32_t q_addr = smem_addr(sQ + qbuf * C::Q_BYTES);
-      for (int kt = e.z; kt < e.w; ++kt, ++n_tile) {
+      for (int kt = e.z; kt < e.w && ok; ++kt, ++n_tile) {
         const uint32_t acc = n_tile & 1;
-        if (!mbar_wait(&s.tempty[acc], ((n_tile >> 1) & 1) ^ 1u, abort_flag, err) ||
-            !mbar_wait(&s.kfull[kstage], kphase, abort_flag, err)) {
+        if (!mbar_wait(&s.tempty[acc], ((n_tile >> 1) & 1) ^ 1u, abort_flag, err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t k_addr = smem_addr(sK + kstage * C::K_BYTES);
-          const uint32_t d = tmem + acc * QN;
+        const uint32_t d = tmem + acc * QN;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            // k-step kk: 64-element k-block kk / 4 (its own swizzled region),
-            // 16 elements (32 bytes) in
-            const uint32_t off = (kk & 3) * 32;
-            umma_bf16(d, umma_desc_sw128(k_addr + (kk >> 2) * (KT * 128) + off),
-                      umma_desc_sw128(q_addr + (kk >> 2) * (QN * 128) + off), IDESC,
-                      kk > 0 ? 1u : 0u);
+        for (int kb = 0; kb < C::KB; ++kb) {
+          if (!mbar_wait(&s.kfull[kstage], kphase, abort_flag, err)) {
+            ok = false;
+            break;
           }
-          umma_commit(&s.kempty[kstage]);
-          umma_commit(&s.tfull[acc]);
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t k_addr = smem_addr(sK + kstage * KSTAGE_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)  // 16 elements (32 bytes) per MMA
+              umma_bf16(d, umma_desc_sw128(k_addr + kk * 32),
+                        umma_desc_sw128(q_addr + kb * (QN * 128) + kk * 32), IDESC,
+                        (kb > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(&s.kempty[kstage]);
+          }
+          __syncwarp();
+          if (++kstage == static_cast<uint32_t>(C::K_STAGES)) {
+            kstage = 0;
+            kphase ^= 1u;
+          }
         }
+        if (ok && lane == 0) umma_commit(&s.tfull[acc]);
         __syncwarp();
-        if (++kstage == static_cast<uint32_t>(C::K_STAGES)) {
-          kstage = 0;
-          kphase ^= 1u;
-        }
       }
       if (ok && lane == 0) umma_commit(&s.qempty[qbuf]);
       __syncwarp();
@@ -301,31 +327,21 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
     // half hf (queries hf*QW .. hf*QW+QW-1 of the block)
     const int q = warp & 3;
     const int hf = (warp - 2) >> 2;
+    constexpr int NL = QW * CPQ;  // 32-column TMEM loads per tile
     int n_unit = 0, n_tile = 0;
-    float wr[QW * NH];  // this warp's queries' head weights (the same in every lane)
     for (;;) {
       const int slot = n_unit % RING;
       if (!mbar_wait(&s.ufull[slot], (n_unit / RING) & 1, abort_flag, err)) break;
       const int4 e = s.ring[slot];
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.uempty[slot]);
+      const int qbuf = n_unit & 1;
+      const uint32_t qphase = (n_unit >> 1) & 1;
       ++n_unit;
       if (e.x < 0) break;
+      if (!mbar_wait(&s.qfull[qbuf], qphase, abort_flag, err)) break;  // the weights landed
+      const float4 *wq = reinterpret_cast<const float4 *>(sW + qbuf * QN + hf * QW * NH);
       const int t0 = e.y * QB + hf * QW;  // first query of this warp
-#pragma unroll
-      for (int j = 0; j < QW; ++j) {
-        const int t = t0 + j;
-        const float4 *src =
-            reinterpret_cast<const float4 *>(w + (static_cast<int64_t>(e.x) * T + min(t, T - 1)) * NH);
-#pragma unroll
-        for (int h4 = 0; h4 < NH / 4; ++h4) {
-          const float4 v = t < T ? __ldg(src + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
-          wr[j * NH + 4 * h4 + 0] = v.x;
-          wr[j * NH + 4 * h4 + 1] = v.y;
-          wr[j * NH + 4 * h4 + 2] = v.z;
-          wr[j * NH + 4 * h4 + 3] = v.w;
-        }
-      }
       bool ok = true;
       for (int kt = e.z; kt < e.w; ++kt, ++n_tile) {
         const uint32_t acc = n_tile & 1;
@@ -335,21 +351,32 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
         }
         tc_fence_after();
         const int key = kt * KT + q * 32 + lane;
-        const uint32_t taddr = tmem + acc * QN + (static_cast<uint32_t>(q * 32) << 16);
+        const uint32_t taddr =
+            tmem + acc * QN + hf * QW * NH + (static_cast<uint32_t>(q * 32) << 16);
         float res[QW];
 #pragma unroll
-        for (int j = 0; j < QW; ++j) {
-          float a = 0.f;
+        for (int j = 0; j < QW; ++j) res[j] = 0.f;
+        // load n + 1 while n is being summed (two register buffers)
+        uint32_t ra[32], rb[32];
+        tmem_ld32(taddr, ra);
+        tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < CPQ; ++c) {
-            uint32_t r[32];
-            tmem_ld32(taddr + (hf * QW + j) * NH + c * 32, r);
-            tmem_ld_wait();
+        for (int n = 0; n < NL; ++n) {
+          uint32_t(&cur)[32] = (n & 1) ? rb : ra;
+          uint32_t(&nxt)[32] = (n & 1) ? ra : rb;
+          if (n + 1 < NL) tmem_ld32(taddr + (n + 1) * 32, nxt);
+          const int j = n / CPQ;
+          float a = res[j];
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              a = fmaf(wr[j * NH + c * 32 + i], fmaxf(__uint_as_float(r[i]), 0.f), a);
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 wv = wq[n * 8 + i4];  // same address in every lane: broadcast
+            a = fmaf(wv.x, fmaxf(__uint_as_float(cur[4 * i4 + 0]), 0.f), a);
+            a = fmaf(wv.y, fmaxf(__uint_as_float(cur[4 * i4 + 1]), 0.f), a);
+            a = fmaf(wv.z, fmaxf(__uint_as_float(cur[4 * i4 + 2]), 0.f), a);
+            a = fmaf(wv.w, fmaxf(__uint_as_float(cur[4 * i4 + 3]), 0.f), a);
           }
-          res[j] = a * scale;
+          res[j] = a;
+          tmem_ld_wait();
         }
         tc_fence_before();
         __syncwarp();
@@ -358,9 +385,12 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
         for (int j = 0; j < QW; ++j) {
           const int t = t0 + j;
           if (t < T && key <= S - T + t)
-            scores[(static_cast<int64_t>(e.x) * T + t) * S + key] = res[j];
+            scores[(static_cast<int64_t>(e.x) * T + t) * S + key] = res[j] * scale;
         }
       }
+      // this warp is done with the unit's weights
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.qempty[qbuf]);
       if (!ok) break;
     }
   }
@@ -403,46 +433,54 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
 
 // ---------------------------------------------------------------- 3) top-k
 
-// Order-preserving integer key of a float: larger float -> larger key.
+// Order-preserving integer key of a float: larger float -> larger key, and
+// -0 and +0 (equal numbers) the same key.
 __device__ __forceinline__ uint32_t order_key(float f) {
-  const uint32_t u = __float_as_uint(f);
+  uint32_t u = __float_as_uint(f);
+  if ((u << 1) == 0u) u = 0u;  // -0 -> +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Block-wide exclusive prefix count of `flag` in thread order; returns the
-// count before this thread and writes the block total to *total.
-template <int NT>
-__device__ __forceinline__ int block_excl_count(bool flag, int *wtot, int *total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned m = __ballot_sync(0xffffffffu, flag);
-  if (lane == 0) wtot[warp] = __popc(m);
-  __syncthreads();
-  int before = 0, all = 0;
+// In place: exclusive prefix sums of cnt[0 .. n) (n a multiple of 32), by one warp;
+// returns the total to every lane.
+__device__ __forceinline__ int warp_exclusive_scan(int *cnt, int n) {
+  const int lane = threadIdx.x & 31;
+  const int per = n / 32;
+  int *c = cnt + lane * per;
+  int sum = 0;
+  for (int i = 0; i < per; ++i) sum += c[i];
+  int incl = sum;
 #pragma unroll
-  for (int w = 0; w < NT / 32; ++w) {
-    const int v = wtot[w];
-    before += w < warp ? v : 0;
-    all += v;
+  for (int d = 1; d < 32; d <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += x;
   }
-  __syncthreads();
-  *total = all;
-  return before + __popc(m & ((1u << lane) - 1u));
+  int run = incl - sum;
+  for (int i = 0; i < per; ++i) {
+    const int v = c[i];
+    c[i] = run;
+    run += v;
+  }
+  return __shfl_sync(0xffffffffu, incl, 31);
 }
 
-// One CTA per query row.  Thread i holds keys i, i + NT, ... (VPT of them) of
-// the visible part of the row in registers.
+// One CTA per query row.  Thread i holds keys j*NT + i (j < VPT) of the
+// visible part of the row in registers (coalesced loads).  Keys are ordered by
+// index as (j, warp, lane), so ranks in index order come from per-(j, warp)
+// counts: ballots, one table, one warp scan.
 template <int NT, int VPT>
 __global__ void __launch_bounds__(NT)
     dsa_topk_kernel(const float *__restrict__ scores, int T, int S, int n_sel,
                     int32_t *__restrict__ sel) {
+  constexpr int NW = NT / 32;
   __shared__ int hist[256];
-  __shared__ int wtot[NT / 32];
-  __shared__ int pick[2];  // digit, keys above it
+  __shared__ int cnt[VPT * NW];
+  __shared__ int pick[3];  // digit, keys above it, keys in it
   const int64_t row = blockIdx.x;
   const int t = static_cast<int>(row % T);
   const int n_vis = S - T + t + 1;  // keys this query sees
   int32_t *out = sel + row * n_sel;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (n_vis <= n_sel) {  // every visible key, then the lowest-index hidden ones
     for (int j = tid; j < n_sel; j += NT) out[j] = j;
     return;
@@ -452,11 +490,11 @@ __global__ void __launch_bounds__(NT)
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const int idx = j * NT + tid;
-    v[j] = idx < n_vis ? order_key(src[idx]) : 0u;  // 0: below every real key
+    v[j] = idx < n_vis ? order_key(__ldg(src + idx)) : 0u;
   }
   // radix select of the n_sel-th largest key, 8 bits at a time
   uint32_t prefix = 0, pmask = 0;
-  int k_rem = n_sel;
+  int k_rem = n_sel, n_eq = 0;
 #pragma unroll 1
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += NT) hist[i] = 0;
@@ -486,6 +524,7 @@ __global__ void __launch_bounds__(NT)
         if (above < k_rem && k_rem <= above + c[i]) {
           pick[0] = 255 - (tid * 8 + i);
           pick[1] = above;
+          pick[2] = c[i];
         }
         above += c[i];
       }
@@ -493,27 +532,49 @@ __global__ void __launch_bounds__(NT)
     __syncthreads();
     const int digit = pick[0];
     k_rem -= pick[1];
+    n_eq = pick[2];
     prefix |= static_cast<uint32_t>(digit) << shift;
     pmask |= 255u << shift;
     __syncthreads();
   }
-  // prefix is the n_sel-th largest key; take every key above it and the first
-  // k_rem keys equal to it, in ascending index
-  int taken_before = 0, eq_before = 0;
+  // prefix is the n_sel-th largest key: take every key above it and the first
+  // k_rem of the n_eq keys equal to it (lowest indices), listed by index
+  const unsigned lt = (1u << lane) - 1u;
+  uint64_t eq_take = ~uint64_t(0);  // bit j: this thread's key j, if equal, is taken
+  if (n_eq > k_rem) {  // ties across the threshold: rank the equal keys by index
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && v[j] == prefix);
+      if (lane == 0) cnt[j * NW + warp] = __popc(m);
+    }
+    __syncthreads();
+    if (warp == 0) warp_exclusive_scan(cnt, VPT * NW);
+    __syncthreads();
+    eq_take = 0;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && v[j] == prefix);
+      if (cnt[j * NW + warp] + __popc(m & lt) < k_rem) eq_take |= uint64_t(1) << j;
+    }
+    __syncthreads();
+  }
+  uint64_t take_bits = 0;
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
-    if (j * NT >= n_vis) break;
-    const int idx = j * NT + tid;
-    const bool valid = idx < n_vis;
-    const bool eq = valid && v[j] == prefix;
-    int eq_tot;
-    const int eq_rank = eq_before + block_excl_count<NT>(eq, wtot, &eq_tot);
-    const bool take = valid && (v[j] > prefix || (eq && eq_rank < k_rem));
-    int take_tot;
-    const int pos = taken_before + block_excl_count<NT>(take, wtot, &take_tot);
-    if (take && pos < n_sel) out[pos] = idx;
-    eq_before += eq_tot;
-    taken_before += take_tot;
+    const bool take = j * NT + tid < n_vis && (v[j] > prefix || (v[j] == prefix && ((eq_take >> j) & 1u)));
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (take) take_bits |= uint64_t(1) << j;
+    if (lane == 0) cnt[j * NW + warp] = __popc(m);
+  }
+  __syncthreads();
+  if (warp == 0) warp_exclusive_scan(cnt, VPT * NW);
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const bool take = (take_bits >> j) & 1u;
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    const int pos = cnt[j * NW + warp] + __popc(m & lt);
+    if (take && pos < n_sel) out[pos] = j * NT + tid;
   }
 }
 

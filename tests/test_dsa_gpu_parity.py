@@ -167,6 +167,8 @@ def test_topk_alone_on_given_scores_is_exact():
     thr = np.sort(vis)[-topk]                  # the row's topk-th score
     sc[0, 5, 100:140] = thr                    # a run of 40 equal scores at the threshold
     sc[1, :, :] = np.round(sc[1] * 4) / 4      # many ties everywhere
+    sc[1, 2, ::3] = -0.0                       # signed zeros: -0 and +0 are equal scores
+    sc[1, 2, 1::3] = 0.0
     cfg = dsa.Config(B, T, S, topk=topk)
     ws = dsa.workspace(cfg)
     got = dsa.topk(cfg, torch.from_numpy(sc).cuda(), ws).cpu().numpy()

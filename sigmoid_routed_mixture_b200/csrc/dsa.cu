@@ -41,18 +41,20 @@ constexpr int RING = 4;            // unit ring entries
 constexpr int MAX_SMEM = 232448;   // 227 KB dynamic shared memory per CTA
 
 constexpr int KSTAGE_BYTES = KT * 64 * 2;  // one 64-element k-block of a key tile (16 KB)
-constexpr int W_BYTES = QN * 4;            // the head weights of one query block (fp32)
 constexpr int MAX_KSTAGES = 8;
 
-template <int D>
+// N (query, head) rows per tile: QB queries of NH heads (QB = 256 / NH, or 1
+// when every sequence has one query: decode reads each key once either way,
+// and N = NH wastes no tensor-core work on empty query rows).
+template <int D, int N>
 struct Cfg {
-  static constexpr int KB = D / 64;             // 64-element k-blocks per key tile
-  static constexpr int Q_BYTES = QN * D * 2;    // one query block
-  static constexpr int K_STAGES =
-      (MAX_SMEM - 2048 - 2 * Q_BYTES - 2 * W_BYTES) / KSTAGE_BYTES < MAX_KSTAGES
-          ? (MAX_SMEM - 2048 - 2 * Q_BYTES - 2 * W_BYTES) / KSTAGE_BYTES
-          : MAX_KSTAGES;
+  static constexpr int KB = D / 64;           // 64-element k-blocks per key tile
+  static constexpr int Q_BYTES = N * D * 2;   // one query block
+  static constexpr int W_BYTES = N * 4;       // its head weights (fp32)
+  static constexpr int FREE = MAX_SMEM - 2048 - 2 * Q_BYTES - 2 * W_BYTES;
+  static constexpr int K_STAGES = FREE / KSTAGE_BYTES < MAX_KSTAGES ? FREE / KSTAGE_BYTES : MAX_KSTAGES;
   static constexpr int DATA_BYTES = 2 * Q_BYTES + K_STAGES * KSTAGE_BYTES + 2 * W_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * N < 32 ? 32 : 2 * N;  // two accumulators
 };
 
 struct Smem {
@@ -66,13 +68,13 @@ struct Smem {
   int abort_flag;
 };
 
-template <int D>
+template <int D, int N>
 constexpr size_t smem_bytes() {
-  return 1024 + Cfg<D>::DATA_BYTES + sizeof(Smem);
+  return 1024 + Cfg<D, N>::DATA_BYTES + sizeof(Smem);
 }
-static_assert(smem_bytes<128>() <= MAX_SMEM, "score kernel shared memory");
-static_assert(smem_bytes<64>() <= MAX_SMEM, "score kernel shared memory");
-static_assert(Cfg<128>::K_STAGES >= 4, "key ring depth");
+static_assert(smem_bytes<128, 256>() <= MAX_SMEM, "score kernel shared memory");
+static_assert(smem_bytes<64, 256>() <= MAX_SMEM, "score kernel shared memory");
+static_assert(Cfg<128, 256>::K_STAGES >= 4, "key ring depth");
 
 // Untiled bulk copy of `bytes` contiguous bytes global -> shared, completing on
 // `bar` (both addresses 16-byte aligned, bytes a multiple of 16).
@@ -92,8 +94,10 @@ __host__ __device__ __forceinline__ int dsa_key_tiles(int qb, int qbs, int T, in
   return (S - T + t_last) / dsa::KT + 1;
 }
 
+int dsa_queries_per_tile(int T, int n_heads) { return T == 1 ? 1 : dsa::QN / n_heads; }
+
 int dsa_units_bound(int T, int S, int n_heads) {
-  const int qbs = dsa::QN / n_heads;
+  const int qbs = dsa_queries_per_tile(T, n_heads);
   const int nqb = (T + qbs - 1) / qbs;
   const int nkt = (S + dsa::KT - 1) / dsa::KT;
   return nqb * ((nkt + dsa::KCH - 1) / dsa::KCH);
@@ -140,18 +144,18 @@ __global__ void __launch_bounds__(1024)
 
 // ---------------------------------------------------------------- 2) scores
 
-template <int NH, int D>
+template <int NH, int D, int QB>
 __global__ void __launch_bounds__(dsa::THREADS, 1)
     dsa_score_kernel(const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k, const float *__restrict__ w,
                      float *__restrict__ scores, const int2 *__restrict__ units, int *ctl, int B,
                      int T, int S, float scale, int *err) {
   using namespace dsa;
-  using C = Cfg<D>;
-  constexpr int QB = QN / NH;          // queries per tile
-  constexpr int QW = QB / 2;           // queries per epilogue warp
-  constexpr int CPQ = NH / 32;         // 32-column TMEM loads per query
-  constexpr uint32_t IDESC = umma_idesc_f32acc(KT, QN, 1u);
+  constexpr int N = QB * NH;                // (query, head) rows per tile: the MMA's N
+  using C = Cfg<D, N>;
+  constexpr int QW = QB > 1 ? QB / 2 : 1;   // queries per epilogue warp
+  constexpr int CPQ = NH / 32;              // 32-column TMEM loads per query
+  constexpr uint32_t IDESC = umma_idesc_f32acc(KT, N, 1u);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   uint8_t *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
     tma_prefetch_desc(&tmap_k);
   }
   if (warp == 1) {
-    tmem_alloc(&s.tmem_base, 2 * QN);
+    tmem_alloc(&s.tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -238,8 +242,8 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
         const int row0 = (e.x * T + t0) * NH;
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_2d(dst + kb * (QN * 128), &tmap_q, &s.qfull[qbuf], kb * 64, row0);
-        bulk_load_1d(sW + qbuf * QN, w + static_cast<int64_t>(e.x * T + t0) * NH, w_bytes,
+          tma_load_2d(dst + kb * (N * 128), &tmap_q, &s.qfull[qbuf], kb * 64, row0);
+        bulk_load_1d(sW + qbuf * N, w + static_cast<int64_t>(e.x * T + t0) * NH, w_bytes,
                      &s.qfull[qbuf]);
       }
       q_last[qbuf] = ((n_unit - 1) >> 1) & 1;
@@ -292,7 +296,7 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + acc * QN;
+        const uint32_t d = tmem + acc * N;
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb) {
           if (!mbar_wait(&s.kfull[kstage], kphase, abort_flag, err)) {
@@ -305,7 +309,7 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)  // 16 elements (32 bytes) per MMA
               umma_bf16(d, umma_desc_sw128(k_addr + kk * 32),
-                        umma_desc_sw128(q_addr + kb * (QN * 128) + kk * 32), IDESC,
+                        umma_desc_sw128(q_addr + kb * (N * 128) + kk * 32), IDESC,
                         (kb > 0 || kk > 0) ? 1u : 0u);
             umma_commit(&s.kempty[kstage]);
           }
@@ -328,6 +332,7 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
     const int q = warp & 3;
     const int hf = (warp - 2) >> 2;
     constexpr int NL = QW * CPQ;  // 32-column TMEM loads per tile
+    const bool active = hf * QW < QB;  // with one query per tile the second half has none
     int n_unit = 0, n_tile = 0;
     for (;;) {
       const int slot = n_unit % RING;
@@ -340,7 +345,7 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
       ++n_unit;
       if (e.x < 0) break;
       if (!mbar_wait(&s.qfull[qbuf], qphase, abort_flag, err)) break;  // the weights landed
-      const float4 *wq = reinterpret_cast<const float4 *>(sW + qbuf * QN + hf * QW * NH);
+      const float4 *wq = reinterpret_cast<const float4 *>(sW + qbuf * N + hf * QW * NH);
       const int t0 = e.y * QB + hf * QW;  // first query of this warp
       bool ok = true;
       for (int kt = e.z; kt < e.w; ++kt, ++n_tile) {
@@ -352,12 +357,13 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
         tc_fence_after();
         const int key = kt * KT + q * 32 + lane;
         const uint32_t taddr =
-            tmem + acc * QN + hf * QW * NH + (static_cast<uint32_t>(q * 32) << 16);
+            tmem + acc * N + hf * QW * NH + (static_cast<uint32_t>(q * 32) << 16);
         float res[QW];
 #pragma unroll
         for (int j = 0; j < QW; ++j) res[j] = 0.f;
         // load n + 1 while n is being summed (two register buffers)
         uint32_t ra[32], rb[32];
+        if (active) {
         tmem_ld32(taddr, ra);
         tmem_ld_wait();
 #pragma unroll
@@ -378,13 +384,14 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
           res[j] = a;
           tmem_ld_wait();
         }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.tempty[acc]);
 #pragma unroll
         for (int j = 0; j < QW; ++j) {
           const int t = t0 + j;
-          if (t < T && key <= S - T + t)
+          if (active && t < T && key <= S - T + t)
             scores[(static_cast<int64_t>(e.x) * T + t) * S + key] = res[j] * scale;
         }
       }
@@ -427,7 +434,7 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * QN);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -464,52 +471,104 @@ __device__ __forceinline__ int warp_exclusive_scan(int *cnt, int n) {
   return __shfl_sync(0xffffffffu, incl, 31);
 }
 
-// One CTA per query row.  Thread i holds keys j*NT + i (j < VPT) of the
-// visible part of the row in registers (coalesced loads).  Keys are ordered by
-// index as (j, warp, lane), so ranks in index order come from per-(j, warp)
-// counts: ballots, one table, one warp scan.
-template <int NT, int VPT>
+// Cluster shared-memory access: add to / read a 32-bit word in another CTA.
+__device__ __forceinline__ void red_add_remote(uint32_t cluster_addr, int v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_remote(uint32_t cluster_addr) {
+  int v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
+// The top-k of one query row, by CL CTAs (a cluster when CL > 1; CL == 1 is one
+// CTA).  CTA r of the row holds keys r*NT*VPT + j*NT + i (thread i, j < VPT) of
+// the visible part in registers (coalesced loads), so the index order of keys is
+// (r, j, warp, lane).  Radix select of the n_sel-th largest key, 8 bits per pass:
+// every CTA counts its keys (shared-memory histogram, eight padded copies so
+// that at most four lanes of a warp hit one address) and, in a cluster, adds
+// its counts into the first CTA's histogram; every CTA reads the sum and takes
+// the same decision.  Ranks in index order for the output come from
+// per-(j, warp) ballot counts, a warp scan, and the earlier CTAs' totals.
+// Every CTA of a cluster runs the same sequence of cluster barriers.
+template <int NT, int VPT, int CL>
 __global__ void __launch_bounds__(NT)
     dsa_topk_kernel(const float *__restrict__ scores, int T, int S, int n_sel,
                     int32_t *__restrict__ sel) {
   constexpr int NW = NT / 32;
+  constexpr int HC = 8;     // histogram copies: lane l counts into copy l % 8
+  constexpr int HS = 257;   // copy stride (words): copies of one digit on different banks
+  constexpr int SLICE = NT * VPT;
+  __shared__ int hist8[HC * HS];
   __shared__ int hist[256];
   __shared__ int cnt[VPT * NW];
   __shared__ int pick[3];  // digit, keys above it, keys in it
-  const int64_t row = blockIdx.x;
+  __shared__ int merged[CL > 1 ? 4 * 256 : 1];  // the cluster's histograms (first CTA)
+  __shared__ int cta_cnt[2][CL];                // per-CTA totals: equal keys, taken keys
+  const int rank = CL > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int64_t row = blockIdx.x / CL;
   const int t = static_cast<int>(row % T);
   const int n_vis = S - T + t + 1;  // keys this query sees
   int32_t *out = sel + row * n_sel;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (n_vis <= n_sel) {  // every visible key, then the lowest-index hidden ones
-    for (int j = tid; j < n_sel; j += NT) out[j] = j;
+  if (n_vis <= n_sel) {  // every visible key, then the lowest-index hidden ones (same in all CTAs)
+    for (int j = rank * NT + tid; j < n_sel; j += CL * NT) out[j] = j;
     return;
   }
-  const float *src = scores + row * S;
+  const int k0 = rank * SLICE;                       // this CTA's first key
+  const int n_loc = max(0, min(SLICE, n_vis - k0));  // its visible keys
+  const float *src = scores + row * S + k0;
   uint32_t v[VPT];
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const int idx = j * NT + tid;
-    v[j] = idx < n_vis ? order_key(__ldg(src + idx)) : 0u;
+    v[j] = idx < n_loc ? order_key(__ldg(src + idx)) : 0u;
   }
-  // radix select of the n_sel-th largest key, 8 bits at a time
+  uint32_t leader_merged = 0, leader_cnt = 0;
+  if constexpr (CL > 1) {
+    leader_merged = cluster_map(merged, 0);
+    leader_cnt = cluster_map(&cta_cnt[0][0], 0);
+    if (rank == 0)
+      for (int i = tid; i < 4 * 256; i += NT) merged[i] = 0;
+    cluster_sync();
+  }
   uint32_t prefix = 0, pmask = 0;
   int k_rem = n_sel, n_eq = 0;
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += NT) hist[i] = 0;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < HC * HS; i += NT) hist8[i] = 0;
     __syncthreads();
+    int *my = hist8 + (lane & (HC - 1)) * HS;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int idx = j * NT + tid;
-      if (idx < n_vis && (v[j] & pmask) == prefix) atomicAdd(&hist[(v[j] >> shift) & 255u], 1);
+      if (idx < n_loc && (v[j] & pmask) == prefix) atomicAdd(&my[(v[j] >> shift) & 255u], 1);
     }
     __syncthreads();
+    for (int i = tid; i < 256; i += NT) {
+      int c = 0;
+#pragma unroll
+      for (int k = 0; k < HC; ++k) c += hist8[k * HS + i];
+      if constexpr (CL > 1) {
+        if (c) red_add_remote(leader_merged + (pass * 256 + i) * 4, c);
+      } else {
+        hist[i] = c;
+      }
+    }
+    if constexpr (CL > 1)
+      cluster_sync();
+    else
+      __syncthreads();
     if (tid < 32) {  // digits 255 .. 0, eight per lane: find the one holding the k_rem-th key
       int c[8], sum = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        c[i] = hist[255 - (tid * 8 + i)];
+        const int d = 255 - (tid * 8 + i);
+        if constexpr (CL > 1)
+          c[i] = ld_remote(leader_merged + (pass * 256 + d) * 4);
+        else
+          c[i] = hist[d];
         sum += c[i];
       }
       int incl = sum;
@@ -530,10 +589,9 @@ __global__ void __launch_bounds__(NT)
       }
     }
     __syncthreads();
-    const int digit = pick[0];
     k_rem -= pick[1];
     n_eq = pick[2];
-    prefix |= static_cast<uint32_t>(digit) << shift;
+    prefix |= static_cast<uint32_t>(pick[0]) << shift;
     pmask |= 255u << shift;
     __syncthreads();
   }
@@ -541,55 +599,76 @@ __global__ void __launch_bounds__(NT)
   // k_rem of the n_eq keys equal to it (lowest indices), listed by index
   const unsigned lt = (1u << lane) - 1u;
   uint64_t eq_take = ~uint64_t(0);  // bit j: this thread's key j, if equal, is taken
-  if (n_eq > k_rem) {  // ties across the threshold: rank the equal keys by index
+  if (n_eq > k_rem) {  // ties across the threshold (the same branch in every CTA)
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && v[j] == prefix);
+      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_loc && v[j] == prefix);
       if (lane == 0) cnt[j * NW + warp] = __popc(m);
     }
     __syncthreads();
-    if (warp == 0) warp_exclusive_scan(cnt, VPT * NW);
-    __syncthreads();
+    if (warp == 0) {
+      const int tot = warp_exclusive_scan(cnt, VPT * NW);
+      if constexpr (CL > 1) {
+        if (lane == 0) st_shared_remote(leader_cnt + (0 * CL + rank) * 4, tot);
+      }
+    }
+    int base = 0;
+    if constexpr (CL > 1) {
+      cluster_sync();
+      for (int r = 0; r < rank; ++r) base += ld_remote(leader_cnt + (0 * CL + r) * 4);
+    } else {
+      __syncthreads();
+    }
     eq_take = 0;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && v[j] == prefix);
-      if (cnt[j * NW + warp] + __popc(m & lt) < k_rem) eq_take |= uint64_t(1) << j;
+      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_loc && v[j] == prefix);
+      if (base + cnt[j * NW + warp] + __popc(m & lt) < k_rem) eq_take |= uint64_t(1) << j;
     }
     __syncthreads();
   }
   uint64_t take_bits = 0;
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
-    const bool take = j * NT + tid < n_vis && (v[j] > prefix || (v[j] == prefix && ((eq_take >> j) & 1u)));
+    const bool take =
+        j * NT + tid < n_loc && (v[j] > prefix || (v[j] == prefix && ((eq_take >> j) & 1u)));
     const unsigned m = __ballot_sync(0xffffffffu, take);
     if (take) take_bits |= uint64_t(1) << j;
     if (lane == 0) cnt[j * NW + warp] = __popc(m);
   }
   __syncthreads();
-  if (warp == 0) warp_exclusive_scan(cnt, VPT * NW);
-  __syncthreads();
+  if (warp == 0) {
+    const int tot = warp_exclusive_scan(cnt, VPT * NW);
+    if constexpr (CL > 1) {
+      if (lane == 0) st_shared_remote(leader_cnt + (1 * CL + rank) * 4, tot);
+    }
+  }
+  int base = 0;
+  if constexpr (CL > 1) {
+    cluster_sync();
+    for (int r = 0; r < rank; ++r) base += ld_remote(leader_cnt + (1 * CL + r) * 4);
+  } else {
+    __syncthreads();
+  }
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const bool take = (take_bits >> j) & 1u;
     const unsigned m = __ballot_sync(0xffffffffu, take);
-    const int pos = cnt[j * NW + warp] + __popc(m & lt);
-    if (take && pos < n_sel) out[pos] = j * NT + tid;
+    const int pos = base + cnt[j * NW + warp] + __popc(m & lt);
+    if (take && pos < n_sel) out[pos] = k0 + j * NT + tid;
   }
+  if constexpr (CL > 1) cluster_sync();  // the first CTA's counters stay until all have read them
 }
 
 // ---------------------------------------------------------------- launches
 
-int dsa_score_smem(int head_dim) {
-  return static_cast<int>(head_dim == 128 ? dsa::smem_bytes<128>() : dsa::smem_bytes<64>());
-}
-
-template <int NH, int D>
+template <int NH, int D, int QB>
 static cudaError_t launch_score(const CUtensorMap &tq, const CUtensorMap &tk, const float *w,
                                 float *scores, const int2 *units, int *ctl, int64_t B, int T,
                                 int S, float scale, int *err, int num_sms, cudaStream_t stream) {
-  auto kern = dsa_score_kernel<NH, D>;
-  constexpr size_t smem = dsa::smem_bytes<D>();
+  auto kern = dsa_score_kernel<NH, D, QB>;
+  constexpr size_t smem = dsa::smem_bytes<D, QB * NH>();
+  static_assert(smem <= dsa::MAX_SMEM, "score kernel shared memory");
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -598,18 +677,23 @@ static cudaError_t launch_score(const CUtensorMap &tq, const CUtensorMap &tk, co
   return cudaGetLastError();
 }
 
+// Rows of the query operand per tile (the box height of the query tensor map).
+int dsa_query_rows_per_tile(int T, int n_heads) { return dsa_queries_per_tile(T, n_heads) * n_heads; }
+
 cudaError_t launch_dsa_scores(const CUtensorMap &tq, const CUtensorMap &tk, const float *w,
                               float *scores, int2 *units, int *ctl, int64_t B, int T, int S,
                               int n_heads, int head_dim, float scale, int *err, int num_sms,
                               cudaStream_t stream) {
-  const int qbs = dsa::QN / n_heads;
+  const int qbs = dsa_queries_per_tile(T, n_heads);
   dsa_plan_kernel<<<1, 1024, 0, stream>>>(T, S, qbs, units, ctl);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-#define SRM_DSA_CASE(NH_, D_)                                                                    \
+#define SRM_DSA_CASE(NH_, D_)                                                                  \
   if (n_heads == NH_ && head_dim == D_)                                                        \
-    return launch_score<NH_, D_>(tq, tk, w, scores, units, ctl, B, T, S, scale, err, num_sms, \
-                                 stream);
+    return qbs == 1 ? launch_score<NH_, D_, 1>(tq, tk, w, scores, units, ctl, B, T, S, scale,  \
+                                               err, num_sms, stream)                           \
+                    : launch_score<NH_, D_, dsa::QN / NH_>(tq, tk, w, scores, units, ctl, B, T, \
+                                                            S, scale, err, num_sms, stream);
   SRM_DSA_CASE(32, 128)
   SRM_DSA_CASE(64, 128)
   SRM_DSA_CASE(128, 128)
@@ -620,21 +704,45 @@ cudaError_t launch_dsa_scores(const CUtensorMap &tq, const CUtensorMap &tk, cons
   return cudaErrorInvalidValue;
 }
 
+template <int CL>
+static cudaError_t launch_topk_cluster(const float *scores, int64_t rows, int T, int S, int n_sel,
+                                       int32_t *sel, cudaStream_t stream) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(rows * CL));
+  lc.blockDim = dim3(256);
+  lc.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, dsa_topk_kernel<256, 16, CL>, scores, T, S, n_sel, sel);
+}
+
 cudaError_t launch_dsa_topk(const float *scores, int64_t B, int T, int S, int topk, int32_t *sel,
-                            cudaStream_t stream) {
+                            int num_sms, cudaStream_t stream) {
   const int n_sel = min(topk, S);
   const int64_t rows = B * T;
   if (rows == 0) return cudaSuccess;
-  if (rows > 0x7fffffff) return cudaErrorInvalidValue;
+  if (rows * 8 > 0x7fffffff) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(rows));
-  if (S <= 256 * 16)
-    dsa_topk_kernel<256, 16><<<grid, 256, 0, stream>>>(scores, T, S, n_sel, sel);
-  else if (S <= 1024 * 16)
-    dsa_topk_kernel<1024, 16><<<grid, 1024, 0, stream>>>(scores, T, S, n_sel, sel);
-  else if (S <= 512 * 64)
-    dsa_topk_kernel<512, 64><<<grid, 512, 0, stream>>>(scores, T, S, n_sel, sel);
-  else
+  if (S <= 256 * 16) {
+    dsa_topk_kernel<256, 16, 1><<<grid, 256, 0, stream>>>(scores, T, S, n_sel, sel);
+  } else if (rows < 2 * num_sms) {
+    // few rows: each row split over a cluster of 2, 4 or 8 CTAs of 4096 keys
+    if (S <= 2 * 4096) return launch_topk_cluster<2>(scores, rows, T, S, n_sel, sel, stream);
+    if (S <= 4 * 4096) return launch_topk_cluster<4>(scores, rows, T, S, n_sel, sel, stream);
+    if (S <= 8 * 4096) return launch_topk_cluster<8>(scores, rows, T, S, n_sel, sel, stream);
     return cudaErrorInvalidValue;
+  } else if (S <= 1024 * 16) {
+    dsa_topk_kernel<1024, 16, 1><<<grid, 1024, 0, stream>>>(scores, T, S, n_sel, sel);
+  } else if (S <= 512 * 64) {
+    dsa_topk_kernel<512, 64, 1><<<grid, 512, 0, stream>>>(scores, T, S, n_sel, sel);
+  } else {
+    return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

@@ -67,7 +67,8 @@ moe_status_t run_scores(const dsa_cfg_t *cfg, const void *q, const void *k, cons
   const int64_t B = cfg->B;
   const int T = cfg->T, S = cfg->S, NH = cfg->n_heads, D = cfg->head_dim;
   CUtensorMap tq, tk;
-  if (!make_tmap(&tq, q, static_cast<uint64_t>(D), static_cast<uint64_t>(B) * T * NH, 64, 256) ||
+  if (!make_tmap(&tq, q, static_cast<uint64_t>(D), static_cast<uint64_t>(B) * T * NH, 64,
+                 static_cast<uint32_t>(srm::dsa_query_rows_per_tile(T, NH))) ||
       !make_tmap(&tk, k, static_cast<uint64_t>(D), static_cast<uint64_t>(B) * S, 64, 128))
     return MOE_ERR_CUDA;
   const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(NH) * D));
@@ -110,7 +111,7 @@ moe_status_t dsa_topk(const dsa_cfg_t *cfg, const float *scores, int32_t *sel, v
   if (!scores || !sel) return MOE_ERR_ARG;
   if (!aligned(scores, 4) || !aligned(sel, 4)) return MOE_ERR_ALIGN;
   return cuda_status(srm::launch_dsa_topk(scores, cfg->B, cfg->T, cfg->S, cfg->topk, sel,
-                                          static_cast<cudaStream_t>(stream)));
+                                          num_sms(), static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t dsa_select(const dsa_cfg_t *cfg, const void *q, const void *k, const float *w,
@@ -129,7 +130,7 @@ moe_status_t dsa_select(const dsa_cfg_t *cfg, const void *q, const void *k, cons
   if (cudaMemsetAsync(wsb + L.ctl, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   st = run_scores(cfg, q, k, w, sc, wsb, L, s);
   if (st != MOE_OK) return st;
-  return cuda_status(srm::launch_dsa_topk(sc, cfg->B, cfg->T, cfg->S, cfg->topk, sel, s));
+  return cuda_status(srm::launch_dsa_topk(sc, cfg->B, cfg->T, cfg->S, cfg->topk, sel, num_sms(), s));
 }
 
 }  // extern "C"

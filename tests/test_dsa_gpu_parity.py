@@ -132,6 +132,16 @@ def test_head_shapes(NH, D):
     r.check_rows(all_rows(wl))
 
 
+@pytest.mark.parametrize("NH,D", [(32, 128), (64, 64), (128, 128)])
+def test_single_query_sequences(NH, D):
+    """One query per sequence (decode): tiles of one query's heads (N = NH)."""
+    wl = W.DsaWorkload("decode", B=5, T=1, S=3000, n_heads=NH, head_dim=D, topk=300,
+                       seed=2250 + NH + D)
+    r = Run(wl)
+    assert r.device_error() == 0
+    r.check_rows(all_rows(wl))
+
+
 def test_short_prompt_lists_every_key():
     """S <= topk: every query selects keys 0 .. S-1 (the page's short-prompt rule)."""
     wl = W.DsaWorkload("short", B=2, T=200, S=200, topk=2048, seed=2300)

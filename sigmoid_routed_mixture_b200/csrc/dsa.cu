@@ -471,104 +471,52 @@ __device__ __forceinline__ int warp_exclusive_scan(int *cnt, int n) {
   return __shfl_sync(0xffffffffu, incl, 31);
 }
 
-// Cluster shared-memory access: add to / read a 32-bit word in another CTA.
-__device__ __forceinline__ void red_add_remote(uint32_t cluster_addr, int v) {
-  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_remote(uint32_t cluster_addr) {
-  int v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
-  return v;
-}
-
-// The top-k of one query row, by CL CTAs (a cluster when CL > 1; CL == 1 is one
-// CTA).  CTA r of the row holds keys r*NT*VPT + j*NT + i (thread i, j < VPT) of
-// the visible part in registers (coalesced loads), so the index order of keys is
-// (r, j, warp, lane).  Radix select of the n_sel-th largest key, 8 bits per pass:
-// every CTA counts its keys (shared-memory histogram, eight padded copies so
-// that at most four lanes of a warp hit one address) and, in a cluster, adds
-// its counts into the first CTA's histogram; every CTA reads the sum and takes
-// the same decision.  Ranks in index order for the output come from
-// per-(j, warp) ballot counts, a warp scan, and the earlier CTAs' totals.
-// Every CTA of a cluster runs the same sequence of cluster barriers.
-template <int NT, int VPT, int CL>
+// One CTA per query row.  Thread i holds keys j*NT + i (j < VPT) of the
+// visible part of the row in registers (coalesced loads).  Keys are ordered by
+// index as (j, warp, lane), so ranks in index order come from per-(j, warp)
+// counts: ballots, one table, one warp scan.
+template <int NT, int VPT>
 __global__ void __launch_bounds__(NT)
     dsa_topk_kernel(const float *__restrict__ scores, int T, int S, int n_sel,
                     int32_t *__restrict__ sel) {
   constexpr int NW = NT / 32;
-  constexpr int HC = 8;     // histogram copies: lane l counts into copy l % 8
-  constexpr int HS = 257;   // copy stride (words): copies of one digit on different banks
-  constexpr int SLICE = NT * VPT;
-  __shared__ int hist8[HC * HS];
   __shared__ int hist[256];
   __shared__ int cnt[VPT * NW];
   __shared__ int pick[3];  // digit, keys above it, keys in it
-  __shared__ int merged[CL > 1 ? 4 * 256 : 1];  // the cluster's histograms (first CTA)
-  __shared__ int cta_cnt[2][CL];                // per-CTA totals: equal keys, taken keys
-  const int rank = CL > 1 ? static_cast<int>(cluster_ctarank()) : 0;
-  const int64_t row = blockIdx.x / CL;
+  const int64_t row = blockIdx.x;
   const int t = static_cast<int>(row % T);
   const int n_vis = S - T + t + 1;  // keys this query sees
   int32_t *out = sel + row * n_sel;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (n_vis <= n_sel) {  // every visible key, then the lowest-index hidden ones (same in all CTAs)
-    for (int j = rank * NT + tid; j < n_sel; j += CL * NT) out[j] = j;
+  if (n_vis <= n_sel) {  // every visible key, then the lowest-index hidden ones
+    for (int j = tid; j < n_sel; j += NT) out[j] = j;
     return;
   }
-  const int k0 = rank * SLICE;                       // this CTA's first key
-  const int n_loc = max(0, min(SLICE, n_vis - k0));  // its visible keys
-  const float *src = scores + row * S + k0;
+  const float *src = scores + row * S;
   uint32_t v[VPT];
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const int idx = j * NT + tid;
-    v[j] = idx < n_loc ? order_key(__ldg(src + idx)) : 0u;
+    v[j] = idx < n_vis ? order_key(__ldg(src + idx)) : 0u;
   }
-  uint32_t leader_merged = 0, leader_cnt = 0;
-  if constexpr (CL > 1) {
-    leader_merged = cluster_map(merged, 0);
-    leader_cnt = cluster_map(&cta_cnt[0][0], 0);
-    if (rank == 0)
-      for (int i = tid; i < 4 * 256; i += NT) merged[i] = 0;
-    cluster_sync();
-  }
+  // radix select of the n_sel-th largest key, 8 bits at a time
   uint32_t prefix = 0, pmask = 0;
   int k_rem = n_sel, n_eq = 0;
 #pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = tid; i < HC * HS; i += NT) hist8[i] = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += NT) hist[i] = 0;
     __syncthreads();
-    int *my = hist8 + (lane & (HC - 1)) * HS;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int idx = j * NT + tid;
-      if (idx < n_loc && (v[j] & pmask) == prefix) atomicAdd(&my[(v[j] >> shift) & 255u], 1);
+      if (idx < n_vis && (v[j] & pmask) == prefix) atomicAdd(&hist[(v[j] >> shift) & 255u], 1);
     }
     __syncthreads();
-    for (int i = tid; i < 256; i += NT) {
-      int c = 0;
-#pragma unroll
-      for (int k = 0; k < HC; ++k) c += hist8[k * HS + i];
-      if constexpr (CL > 1) {
-        if (c) red_add_remote(leader_merged + (pass * 256 + i) * 4, c);
-      } else {
-        hist[i] = c;
-      }
-    }
-    if constexpr (CL > 1)
-      cluster_sync();
-    else
-      __syncthreads();
     if (tid < 32) {  // digits 255 .. 0, eight per lane: find the one holding the k_rem-th key
       int c[8], sum = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int d = 255 - (tid * 8 + i);
-        if constexpr (CL > 1)
-          c[i] = ld_remote(leader_merged + (pass * 256 + d) * 4);
-        else
-          c[i] = hist[d];
+        c[i] = hist[255 - (tid * 8 + i)];
         sum += c[i];
       }
       int incl = sum;
@@ -589,9 +537,10 @@ __global__ void __launch_bounds__(NT)
       }
     }
     __syncthreads();
+    const int digit = pick[0];
     k_rem -= pick[1];
     n_eq = pick[2];
-    prefix |= static_cast<uint32_t>(pick[0]) << shift;
+    prefix |= static_cast<uint32_t>(digit) << shift;
     pmask |= 255u << shift;
     __syncthreads();
   }
@@ -599,65 +548,41 @@ __global__ void __launch_bounds__(NT)
   // k_rem of the n_eq keys equal to it (lowest indices), listed by index
   const unsigned lt = (1u << lane) - 1u;
   uint64_t eq_take = ~uint64_t(0);  // bit j: this thread's key j, if equal, is taken
-  if (n_eq > k_rem) {  // ties across the threshold (the same branch in every CTA)
+  if (n_eq > k_rem) {  // ties across the threshold: rank the equal keys by index
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_loc && v[j] == prefix);
+      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && v[j] == prefix);
       if (lane == 0) cnt[j * NW + warp] = __popc(m);
     }
     __syncthreads();
-    if (warp == 0) {
-      const int tot = warp_exclusive_scan(cnt, VPT * NW);
-      if constexpr (CL > 1) {
-        if (lane == 0) st_shared_remote(leader_cnt + (0 * CL + rank) * 4, tot);
-      }
-    }
-    int base = 0;
-    if constexpr (CL > 1) {
-      cluster_sync();
-      for (int r = 0; r < rank; ++r) base += ld_remote(leader_cnt + (0 * CL + r) * 4);
-    } else {
-      __syncthreads();
-    }
+    if (warp == 0) warp_exclusive_scan(cnt, VPT * NW);
+    __syncthreads();
     eq_take = 0;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_loc && v[j] == prefix);
-      if (base + cnt[j * NW + warp] + __popc(m & lt) < k_rem) eq_take |= uint64_t(1) << j;
+      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && v[j] == prefix);
+      if (cnt[j * NW + warp] + __popc(m & lt) < k_rem) eq_take |= uint64_t(1) << j;
     }
     __syncthreads();
   }
   uint64_t take_bits = 0;
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
-    const bool take =
-        j * NT + tid < n_loc && (v[j] > prefix || (v[j] == prefix && ((eq_take >> j) & 1u)));
+    const bool take = j * NT + tid < n_vis && (v[j] > prefix || (v[j] == prefix && ((eq_take >> j) & 1u)));
     const unsigned m = __ballot_sync(0xffffffffu, take);
     if (take) take_bits |= uint64_t(1) << j;
     if (lane == 0) cnt[j * NW + warp] = __popc(m);
   }
   __syncthreads();
-  if (warp == 0) {
-    const int tot = warp_exclusive_scan(cnt, VPT * NW);
-    if constexpr (CL > 1) {
-      if (lane == 0) st_shared_remote(leader_cnt + (1 * CL + rank) * 4, tot);
-    }
-  }
-  int base = 0;
-  if constexpr (CL > 1) {
-    cluster_sync();
-    for (int r = 0; r < rank; ++r) base += ld_remote(leader_cnt + (1 * CL + r) * 4);
-  } else {
-    __syncthreads();
-  }
+  if (warp == 0) warp_exclusive_scan(cnt, VPT * NW);
+  __syncthreads();
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const bool take = (take_bits >> j) & 1u;
     const unsigned m = __ballot_sync(0xffffffffu, take);
-    const int pos = base + cnt[j * NW + warp] + __popc(m & lt);
-    if (take && pos < n_sel) out[pos] = k0 + j * NT + tid;
+    const int pos = cnt[j * NW + warp] + __popc(m & lt);
+    if (take && pos < n_sel) out[pos] = j * NT + tid;
   }
-  if constexpr (CL > 1) cluster_sync();  // the first CTA's counters stay until all have read them
 }
 
 // ---------------------------------------------------------------- launches
@@ -704,45 +629,21 @@ cudaError_t launch_dsa_scores(const CUtensorMap &tq, const CUtensorMap &tk, cons
   return cudaErrorInvalidValue;
 }
 
-template <int CL>
-static cudaError_t launch_topk_cluster(const float *scores, int64_t rows, int T, int S, int n_sel,
-                                       int32_t *sel, cudaStream_t stream) {
-  cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(static_cast<unsigned>(rows * CL));
-  lc.blockDim = dim3(256);
-  lc.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  lc.attrs = attr;
-  lc.numAttrs = 1;
-  return cudaLaunchKernelEx(&lc, dsa_topk_kernel<256, 16, CL>, scores, T, S, n_sel, sel);
-}
-
 cudaError_t launch_dsa_topk(const float *scores, int64_t B, int T, int S, int topk, int32_t *sel,
-                            int num_sms, cudaStream_t stream) {
+                            cudaStream_t stream) {
   const int n_sel = min(topk, S);
   const int64_t rows = B * T;
   if (rows == 0) return cudaSuccess;
-  if (rows * 8 > 0x7fffffff) return cudaErrorInvalidValue;
+  if (rows > 0x7fffffff) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(rows));
-  if (S <= 256 * 16) {
-    dsa_topk_kernel<256, 16, 1><<<grid, 256, 0, stream>>>(scores, T, S, n_sel, sel);
-  } else if (rows < 2 * num_sms) {
-    // few rows: each row split over a cluster of 2, 4 or 8 CTAs of 4096 keys
-    if (S <= 2 * 4096) return launch_topk_cluster<2>(scores, rows, T, S, n_sel, sel, stream);
-    if (S <= 4 * 4096) return launch_topk_cluster<4>(scores, rows, T, S, n_sel, sel, stream);
-    if (S <= 8 * 4096) return launch_topk_cluster<8>(scores, rows, T, S, n_sel, sel, stream);
+  if (S <= 256 * 16)
+    dsa_topk_kernel<256, 16><<<grid, 256, 0, stream>>>(scores, T, S, n_sel, sel);
+  else if (S <= 1024 * 16)
+    dsa_topk_kernel<1024, 16><<<grid, 1024, 0, stream>>>(scores, T, S, n_sel, sel);
+  else if (S <= 512 * 64)
+    dsa_topk_kernel<512, 64><<<grid, 512, 0, stream>>>(scores, T, S, n_sel, sel);
+  else
     return cudaErrorInvalidValue;
-  } else if (S <= 1024 * 16) {
-    dsa_topk_kernel<1024, 16, 1><<<grid, 1024, 0, stream>>>(scores, T, S, n_sel, sel);
-  } else if (S <= 512 * 64) {
-    dsa_topk_kernel<512, 64, 1><<<grid, 512, 0, stream>>>(scores, T, S, n_sel, sel);
-  } else {
-    return cudaErrorInvalidValue;
-  }
   return cudaGetLastError();
 }
 

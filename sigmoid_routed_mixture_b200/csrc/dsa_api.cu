@@ -111,7 +111,7 @@ moe_status_t dsa_topk(const dsa_cfg_t *cfg, const float *scores, int32_t *sel, v
   if (!scores || !sel) return MOE_ERR_ARG;
   if (!aligned(scores, 4) || !aligned(sel, 4)) return MOE_ERR_ALIGN;
   return cuda_status(srm::launch_dsa_topk(scores, cfg->B, cfg->T, cfg->S, cfg->topk, sel,
-                                          num_sms(), static_cast<cudaStream_t>(stream)));
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t dsa_select(const dsa_cfg_t *cfg, const void *q, const void *k, const float *w,
@@ -130,7 +130,7 @@ moe_status_t dsa_select(const dsa_cfg_t *cfg, const void *q, const void *k, cons
   if (cudaMemsetAsync(wsb + L.ctl, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   st = run_scores(cfg, q, k, w, sc, wsb, L, s);
   if (st != MOE_OK) return st;
-  return cuda_status(srm::launch_dsa_topk(sc, cfg->B, cfg->T, cfg->S, cfg->topk, sel, num_sms(), s));
+  return cuda_status(srm::launch_dsa_topk(sc, cfg->B, cfg->T, cfg->S, cfg->topk, sel, s));
 }
 
 }  // extern "C"

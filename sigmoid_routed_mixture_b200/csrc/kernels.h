@@ -88,6 +88,6 @@ cudaError_t launch_dsa_scores(const CUtensorMap &tq, const CUtensorMap &tk, cons
                               int n_heads, int head_dim, float scale, int *err, int num_sms,
                               cudaStream_t stream);
 cudaError_t launch_dsa_topk(const float *scores, int64_t B, int T, int S, int topk, int32_t *sel,
-                            int num_sms, cudaStream_t stream);
+                            cudaStream_t stream);
 
 }  // namespace srm

@@ -113,10 +113,12 @@ def test_tiny_full_parity():
 
 
 @pytest.mark.parametrize("B,T,S,topk", [(3, 37, 300, 50), (1, 5, 1000, 128), (2, 129, 129, 40),
-                                        (1, 1, 777, 700)])
+                                        (1, 1, 777, 700), (2, 333, 333, 100), (3, 250, 700, 300)])
 def test_ragged_queries_keys_and_cache(B, T, S, topk):
     """Query counts not a multiple of the 8-query block, key counts not a multiple
-    of the 128-key tile, and a cache (T < S: queries sit at the last T positions)."""
+    of the 128-key tile, and a cache (T < S: queries sit at the last T positions);
+    enough rows for the persistent top-k, with rows that do (S % 4 == 0) and do
+    not start on 16-byte boundaries."""
     wl = W.DsaWorkload("ragged", B=B, T=T, S=S, topk=topk, seed=2100 + T + S)
     r = Run(wl)
     assert r.device_error() == 0

@@ -158,27 +158,44 @@ def cores():
     return len(os.sched_getaffinity(0))
 
 
-def measured_traffic(workload, kernel):
-    """DRAM bytes per launch from a committed ncu capture (profiles/dram_traffic_glm5.md),
-    or None when the GEMM sources (grouped_gemm.cu, common.cuh, the GemmArgs block
-    of kernels.h) changed since it was taken."""
+def kernel_source_hash(kernel):
+    """md5 of the sources a kernel's DRAM traffic depends on: the grouped GEMM
+    (grouped_gemm.cu, common.cuh, the GemmArgs block of kernels.h) or the key
+    selection's score kernel (its section of dsa.cu, common.cuh)."""
     import hashlib
 
-    path = os.path.join(ROOT, "profiles", "dram_traffic_glm5.md")
-    if not os.path.exists(path):
-        return None
     h = hashlib.md5()
     csrc = os.path.join(ROOT, "sigmoid_routed_mixture_b200", "csrc")
-    for f in ("grouped_gemm.cu", "common.cuh"):
-        h.update(open(os.path.join(csrc, f), "rb").read())
+    if kernel.startswith("dsa_score"):
+        h.update(open(os.path.join(csrc, "common.cuh"), "rb").read())
+        src = open(os.path.join(csrc, "dsa.cu"), "rb").read()
+        a = src.index(b"// ---------------------------------------------------------------- 2) scores")
+        b = src.index(b"// ---------------------------------------------------------------- 3) top-k")
+        h.update(src[a:b])
+        return h.hexdigest()
+    h.update(open(os.path.join(csrc, "grouped_gemm.cu"), "rb").read())
+    h.update(open(os.path.join(csrc, "common.cuh"), "rb").read())
     hdr = open(os.path.join(csrc, "kernels.h"), "rb").read()
     a = hdr.index(b"struct GemmArgs {")
     h.update(hdr[a:hdr.index(b"};", a) + 2])  # the GEMM's argument block, not the other declarations
-    for line in open(path):
-        parts = line.split()
-        if len(parts) == 5 and parts[0] == "traffic" and parts[1] == workload and parts[2] == kernel:
-            if parts[4] == "src=" + h.hexdigest():
-                return float(parts[3])
+    return h.hexdigest()
+
+
+def measured_traffic(workload, kernel):
+    """DRAM bytes per launch from a committed ncu capture (the `traffic` lines of
+    profiles/*.md), or None when the kernel's sources changed since it was taken."""
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    want = "src=" + kernel_source_hash(kernel)
+    for fn in sorted(os.listdir(pdir)):
+        if not fn.endswith(".md"):
+            continue
+        for line in open(os.path.join(pdir, fn)):
+            parts = line.split()
+            if len(parts) == 5 and parts[0] == "traffic" and parts[1] == workload and parts[2] == kernel:
+                if parts[4] == want:
+                    return float(parts[3])
     return None
 
 

@@ -86,6 +86,23 @@ __device__ __forceinline__ void bulk_load_1d(void *dst, const void *src, uint32_
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
+// Two fp32 values in one 64-bit register pair, and the packed fused multiply-add
+// of sm_100 (each half rounds like fmaf).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float sum_f32x2(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo + hi;
+}
 }  // namespace dsa
 
 // key tiles query block qb needs (its last query sees keys 0 .. S - T + t_last)
@@ -358,9 +375,11 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
         const int key = kt * KT + q * 32 + lane;
         const uint32_t taddr =
             tmem + acc * N + hf * QW * NH + (static_cast<uint32_t>(q * 32) << 16);
-        float res[QW];
+        // two running sums per query (even and odd heads) in one f32x2 register
+        // pair: one packed FMA per two heads
+        uint64_t acc2[QW];
 #pragma unroll
-        for (int j = 0; j < QW; ++j) res[j] = 0.f;
+        for (int j = 0; j < QW; ++j) acc2[j] = pack_f32x2(0.f, 0.f);
         // load n + 1 while n is being summed (two register buffers)
         uint32_t ra[32], rb[32];
         if (active) {
@@ -372,16 +391,18 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
           uint32_t(&nxt)[32] = (n & 1) ? ra : rb;
           if (n + 1 < NL) tmem_ld32(taddr + (n + 1) * 32, nxt);
           const int j = n / CPQ;
-          float a = res[j];
+          uint64_t a = acc2[j];
 #pragma unroll
           for (int i4 = 0; i4 < 8; ++i4) {
             const float4 wv = wq[n * 8 + i4];  // same address in every lane: broadcast
-            a = fmaf(wv.x, fmaxf(__uint_as_float(cur[4 * i4 + 0]), 0.f), a);
-            a = fmaf(wv.y, fmaxf(__uint_as_float(cur[4 * i4 + 1]), 0.f), a);
-            a = fmaf(wv.z, fmaxf(__uint_as_float(cur[4 * i4 + 2]), 0.f), a);
-            a = fmaf(wv.w, fmaxf(__uint_as_float(cur[4 * i4 + 3]), 0.f), a);
+            const float r0 = fmaxf(__uint_as_float(cur[4 * i4 + 0]), 0.f);
+            const float r1 = fmaxf(__uint_as_float(cur[4 * i4 + 1]), 0.f);
+            const float r2 = fmaxf(__uint_as_float(cur[4 * i4 + 2]), 0.f);
+            const float r3 = fmaxf(__uint_as_float(cur[4 * i4 + 3]), 0.f);
+            a = fma_f32x2(pack_f32x2(wv.x, wv.y), pack_f32x2(r0, r1), a);
+            a = fma_f32x2(pack_f32x2(wv.z, wv.w), pack_f32x2(r2, r3), a);
           }
-          res[j] = a;
+          acc2[j] = a;
           tmem_ld_wait();
         }
         }
@@ -392,7 +413,7 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
         for (int j = 0; j < QW; ++j) {
           const int t = t0 + j;
           if (active && t < T && key <= S - T + t)
-            scores[(static_cast<int64_t>(e.x) * T + t) * S + key] = res[j] * scale;
+            scores[(static_cast<int64_t>(e.x) * T + t) * S + key] = sum_f32x2(acc2[j]) * scale;
         }
       }
       // this warp is done with the unit's weights

@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
     dsa_score_kernel(const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k, const float *__restrict__ w,
                      float *__restrict__ scores, const int2 *__restrict__ units, int *ctl, int B,
-                     int T, int S, float scale, int *err) {
+                     int T, int S, float scale, int *err, int stall) {
   using namespace dsa;
   constexpr int N = QB * NH;                // (query, head) rows per tile: the MMA's N
   using C = Cfg<D, N>;
@@ -271,6 +271,10 @@ __global__ void __launch_bounds__(dsa::THREADS, 1)
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb) {
           if (!mbar_wait(&s.kempty[kstage], kphase ^ 1u, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          if (stall) {  // failure-detection tests: arm nothing, so the MMA warp's wait runs out
             ok = false;
             break;
           }
@@ -611,7 +615,8 @@ __global__ void __launch_bounds__(NT)
 template <int NH, int D, int QB>
 static cudaError_t launch_score(const CUtensorMap &tq, const CUtensorMap &tk, const float *w,
                                 float *scores, const int2 *units, int *ctl, int64_t B, int T,
-                                int S, float scale, int *err, int num_sms, cudaStream_t stream) {
+                                int S, float scale, int *err, int stall, int num_sms,
+                                cudaStream_t stream) {
   auto kern = dsa_score_kernel<NH, D, QB>;
   constexpr size_t smem = dsa::smem_bytes<D, QB * NH>();
   static_assert(smem <= dsa::MAX_SMEM, "score kernel shared memory");
@@ -619,7 +624,7 @@ static cudaError_t launch_score(const CUtensorMap &tq, const CUtensorMap &tk, co
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   kern<<<num_sms, dsa::THREADS, smem, stream>>>(tq, tk, w, scores, units, ctl, static_cast<int>(B),
-                                                T, S, scale, err);
+                                                T, S, scale, err, stall);
   return cudaGetLastError();
 }
 
@@ -628,8 +633,8 @@ int dsa_query_rows_per_tile(int T, int n_heads) { return dsa_queries_per_tile(T,
 
 cudaError_t launch_dsa_scores(const CUtensorMap &tq, const CUtensorMap &tk, const float *w,
                               float *scores, int2 *units, int *ctl, int64_t B, int T, int S,
-                              int n_heads, int head_dim, float scale, int *err, int num_sms,
-                              cudaStream_t stream) {
+                              int n_heads, int head_dim, float scale, int *err, int stall,
+                              int num_sms, cudaStream_t stream) {
   const int qbs = dsa_queries_per_tile(T, n_heads);
   dsa_plan_kernel<<<1, 1024, 0, stream>>>(T, S, qbs, units, ctl);
   cudaError_t e = cudaGetLastError();
@@ -637,9 +642,9 @@ cudaError_t launch_dsa_scores(const CUtensorMap &tq, const CUtensorMap &tk, cons
 #define SRM_DSA_CASE(NH_, D_)                                                                  \
   if (n_heads == NH_ && head_dim == D_)                                                        \
     return qbs == 1 ? launch_score<NH_, D_, 1>(tq, tk, w, scores, units, ctl, B, T, S, scale,  \
-                                               err, num_sms, stream)                           \
+                                               err, stall, num_sms, stream)                    \
                     : launch_score<NH_, D_, dsa::QN / NH_>(tq, tk, w, scores, units, ctl, B, T, \
-                                                            S, scale, err, num_sms, stream);
+                                                            S, scale, err, stall, num_sms, stream);
   SRM_DSA_CASE(32, 128)
   SRM_DSA_CASE(64, 128)
   SRM_DSA_CASE(128, 128)

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "../../include/srm_dsa.h"
 #include "host_util.h"
@@ -72,10 +73,14 @@ moe_status_t run_scores(const dsa_cfg_t *cfg, const void *q, const void *k, cons
       !make_tmap(&tk, k, static_cast<uint64_t>(D), static_cast<uint64_t>(B) * S, 64, 128))
     return MOE_ERR_CUDA;
   const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(NH) * D));
+  // failure-detection tests only: SRM_MOE_INJECT_STALL=1 makes the producer
+  // arm no key copy, so the call ends with MOE_ERR_TIMEOUT after the wait limit
+  const char *inject = getenv("SRM_MOE_INJECT_STALL");
+  const int stall = (inject && inject[0] == '1') ? 1 : 0;
   return cuda_status(srm::launch_dsa_scores(
       tq, tk, w, scores, reinterpret_cast<int2 *>(wsb + L.units),
       reinterpret_cast<int *>(wsb + L.ctl + 128), B, T, S, NH, D, scale,
-      reinterpret_cast<int *>(wsb + L.ctl), num_sms(), s));
+      reinterpret_cast<int *>(wsb + L.ctl), stall, num_sms(), s));
 }
 
 }  // namespace

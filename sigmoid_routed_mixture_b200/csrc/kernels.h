@@ -85,8 +85,8 @@ int dsa_units_bound(int T, int S, int n_heads);
 int dsa_query_rows_per_tile(int T, int n_heads);
 cudaError_t launch_dsa_scores(const CUtensorMap &tq, const CUtensorMap &tk, const float *w,
                               float *scores, int2 *units, int *ctl, int64_t B, int T, int S,
-                              int n_heads, int head_dim, float scale, int *err, int num_sms,
-                              cudaStream_t stream);
+                              int n_heads, int head_dim, float scale, int *err, int stall,
+                              int num_sms, cudaStream_t stream);
 cudaError_t launch_dsa_topk(const float *scores, int64_t B, int T, int S, int topk, int32_t *sel,
                             cudaStream_t stream);
 

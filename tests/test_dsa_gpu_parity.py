@@ -273,3 +273,25 @@ def test_glm5_decode_sampled():
     """64 sequences, one query each over a 32768-key cache."""
     check_sampled(W.DSA_WORKLOADS["dsa_decode"], 12, 8)
     torch.cuda.empty_cache()
+
+
+def test_timeout_is_reported_and_context_survives(monkeypatch):
+    """Failure detection without a GPU fault: with SRM_MOE_INJECT_STALL=1 the score
+    kernel's producer arms no key copy, so the MMA warp's bounded wait on the key
+    ring runs out (2 s), the kernel drains and returns, and the host reads
+    MOE_ERR_TIMEOUT.  The next call on the same context is correct."""
+    from sigmoid_routed_mixture_b200 import moe
+
+    wl = W.DsaWorkload("stall", B=1, T=64, S=300, topk=32, seed=2700)
+    q, k, w = W.dsa_inputs(wl)
+    cfg = dsa.Config(wl.B, wl.T, wl.S, topk=wl.topk)
+    ws = dsa.workspace(cfg)
+    qd, kd, wd = dev_bf16(q), dev_bf16(k), torch.from_numpy(w).cuda()
+    monkeypatch.setenv("SRM_MOE_INJECT_STALL", "1")
+    dsa.scores(cfg, qd, kd, wd, ws)
+    torch.cuda.synchronize()
+    assert moe.device_error(ws) == 6  # MOE_ERR_TIMEOUT
+    monkeypatch.delenv("SRM_MOE_INJECT_STALL")
+    r = Run(wl)
+    assert r.device_error() == 0
+    r.check_rows(all_rows(wl))

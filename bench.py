@@ -318,6 +318,12 @@ def dsa_visible_pairs(w):
     return w.B * (w.T * (w.S - w.T) + w.T * (w.T + 1) // 2)
 
 
+def dsa_replica_inputs(w, rank):
+    """(q, k, w) of replica `rank`: the workload's own inputs on rank 0, an
+    independently seeded draw of the same shapes on the others."""
+    return W.dsa_inputs(w if rank == 0 else w.replace(seed=w.seed + 7919 * rank))
+
+
 def dsa_oracle_sample(w, n, inputs):
     """A bounded oracle sample: n consecutive queries of sequence 0 around the
     middle of the prompt (prefill), or the single query of n sequences (decode).
@@ -383,7 +389,7 @@ def run_dsa(args, world, rank, dist, dev):
     from sigmoid_routed_mixture_b200 import dsa, moe
 
     w = W.DSA_WORKLOADS[args.workload]
-    q, k, wt = W.dsa_inputs(w if rank == 0 else w.replace(seed=w.seed + 7919 * rank))
+    q, k, wt = dsa_replica_inputs(w, rank)
     cfg = dsa.Config(w.B, w.T, w.S, w.n_heads, w.head_dim, w.topk)
     ws = dsa.workspace(cfg, device=dev)
     q_dev = torch.from_numpy(q.view(np.int16)).to(dev).view(torch.bfloat16)

@@ -32,13 +32,18 @@ def _rank_main(rank, world, port, out):
 
     w = W.WORKLOADS["tiny"]
     x, w_r, b = bench.replica_tokens(w, rank)
+    q, k, _ = bench.dsa_replica_inputs(W.DSA_WORKLOADS["dsa_tiny"], rank)
+    dsa_digest = torch.tensor([float(q.astype(np.float64).sum() + k.astype(np.float64).sum())])
+    dsa_gathered = [torch.zeros(1) for _ in range(world)]
+    dist.all_gather(dsa_gathered, dsa_digest)
     ms = 10.0 + 5.0 * rank  # rank 1 is the slower replica
     t_max = bench.max_over_ranks(ms, dist, "cpu")
     value = bench.aggregate_tokens_per_s(w.T, world, 7, t_max)
     digest = torch.tensor([float(x.astype(np.float64).sum())])
     gathered = [torch.zeros(1) for _ in range(world)]
     dist.all_gather(gathered, digest)
-    out[rank] = (t_max, value, [float(g) for g in gathered], float(w_r.sum()))
+    out[rank] = (t_max, value, [float(g) for g in gathered], float(w_r.sum()),
+                 [float(g) for g in dsa_gathered])
     dist.destroy_process_group()
 
 
@@ -46,11 +51,12 @@ def test_two_replicas_with_gloo():
     world = 2
     out = mp.Manager().dict()
     mp.spawn(_rank_main, args=(world, free_port(), out), nprocs=world, join=True)
-    (t0, v0, d0, r0), (t1, v1, d1, r1) = out[0], out[1]
+    (t0, v0, d0, r0, q0), (t1, v1, d1, r1, q1) = out[0], out[1]
     assert t0 == t1 == 15.0                      # every rank sees the slowest replica
     assert v0 == v1 == pytest.approx(64 * 2 * 7 / 0.015)
     assert d0[0] != d0[1]                        # replicas draw different token batches
     assert r0 == r1                              # ... with the same router weights
+    assert q0[0] != q0[1]                        # key-selection replicas: different q, k too
 
 
 def test_reference_arm_under_torchrun_prints_one_line():
@@ -63,3 +69,29 @@ def test_reference_arm_under_torchrun_prints_one_line():
     lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1
     assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2 and lines[0]["value"] > 0
+
+
+def test_key_selection_reference_arm_under_torchrun_prints_one_line():
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--workload", "dsa_tiny", "--gpus", "2", "--steps", "1", "--warmup", "3",
+           "--ref-tokens", "4"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference" and line["unit"] == "queries/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_visible_pairs_count():
+    """The causal (query, key) pairs the bench counts as algorithmic work, by brute force."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from sigmoid_routed_mixture_b200 import workloads as W
+
+    for B, T, S in ((1, 1, 1), (2, 5, 5), (3, 4, 9), (1, 7, 300)):
+        w = W.DsaWorkload("x", B=B, T=T, S=S)
+        brute = sum(1 for b in range(B) for t in range(T) for s in range(S) if s <= S - T + t)
+        assert bench.dsa_visible_pairs(w) == brute

@@ -261,6 +261,50 @@ def replica_tokens(w, rank):
     return x, w_r, b
 
 
+def pipelined_e2e(torch, stream, dev, n_steps, dist, copy_in, replays, copy_out):
+    """Device time (max over ranks) of n_steps end-to-end steps, each made of its
+    input copy (host -> device, copy_in(j)), its compute (replays[j]() on `stream`)
+    and its output copy (device -> host, copy_out(j)), for the buffer set
+    j = step % 2.  The copies run on their own streams, so step i + 1's input
+    and step i - 1's output move while step i computes; the events keep a
+    buffer set from being refilled before its compute and output copy are done."""
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def run(n):
+        for i in range(n):
+            j = i % 2
+            if i >= 2:
+                h2d.wait_event(ev_comp[j])
+            with torch.cuda.stream(h2d):
+                copy_in(j)
+                ev_in[j].record(h2d)
+            stream.wait_event(ev_in[j])
+            if i >= 2:
+                stream.wait_event(ev_out[j])
+            replays[j]()
+            ev_comp[j].record(stream)
+            d2h.wait_event(ev_comp[j])
+            with torch.cuda.stream(d2h):
+                copy_out(j)
+                ev_out[j].record(d2h)
+
+    run(2)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    z = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a.record(h2d)
+    run(n_steps)
+    z.record(d2h)
+    torch.cuda.synchronize()
+    return max_over_ranks(a.elapsed_time(z), dist, dev)
+
+
 def max_over_ranks(ms, dist, device):
     """The slowest replica's device time (every rank takes the same collective)."""
     if dist is None:
@@ -399,13 +443,14 @@ def run_dsa(args, world, rank, dist, dev):
     sel = torch.empty((w.B, w.T, cfg.n_sel), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
+    def step(ev=None, bufs=None):
+        qd, kd, wd, sd = bufs if bufs is not None else (q_dev, k_dev, w_dev, sel)
         if ev is not None:
             ev[0].record(stream)
-        dsa.scores(cfg, q_dev, k_dev, w_dev, ws, out=scores)
+        dsa.scores(cfg, qd, kd, wd, ws, out=scores)
         if ev is not None:
             ev[1].record(stream)
-        dsa.topk(cfg, scores, ws, out=sel)
+        dsa.topk(cfg, scores, ws, out=sd)
         if ev is not None:
             ev[2].record(stream)
 
@@ -447,32 +492,35 @@ def run_dsa(args, world, rank, dist, dev):
     t_max = max_over_ranks(total_ms, dist, dev)
     value = w.B * w.T * world * args.steps / (t_max / 1e3)
 
-    # end to end: q, k, w from pinned host memory in, the selection out, every step
+    # end to end: q, k, w from pinned host memory in, the selection out, every
+    # step; two buffer sets and copy streams overlap the copies with the compute
     hq = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).pin_memory()
     hk = torch.from_numpy(k.view(np.int16)).view(torch.bfloat16).pin_memory()
     hw = torch.from_numpy(wt).pin_memory()
-    hsel = torch.empty(tuple(sel.shape), dtype=torch.int32).pin_memory()
-
-    def e2e_step():
-        q_dev.copy_(hq, non_blocking=True)
-        k_dev.copy_(hk, non_blocking=True)
-        w_dev.copy_(hw, non_blocking=True)
-        if graph is not None:
-            graph.replay()
+    hsel = [torch.empty(tuple(sel.shape), dtype=torch.int32).pin_memory() for _ in range(2)]
+    bufs = [(q_dev, k_dev, w_dev, sel),
+            (torch.empty_like(q_dev), torch.empty_like(k_dev), torch.empty_like(w_dev), torch.empty_like(sel))]
+    replays = []
+    for j in range(2):
+        if graph is not None and j == 0:
+            replays.append(graph.replay)
+        elif graph is not None:
+            step(bufs=bufs[1])
+            torch.cuda.synchronize()
+            g1 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g1):
+                step(bufs=bufs[1])
+            replays.append(g1.replay)
         else:
-            step()
-        hsel.copy_(sel, non_blocking=True)
+            replays.append(lambda j=j: step(bufs=bufs[j]))
 
-    e2e_step()
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    def copy_in(j):
+        bufs[j][0].copy_(hq, non_blocking=True)
+        bufs[j][1].copy_(hk, non_blocking=True)
+        bufs[j][2].copy_(hw, non_blocking=True)
+
+    e2e_ms = pipelined_e2e(torch, stream, dev, args.e2e_steps, dist, copy_in, replays,
+                           lambda j: hsel[j].copy_(bufs[j][3], non_blocking=True))
     if moe.device_error(ws) != 0:
         raise RuntimeError("device error during the timed steps")
 
@@ -513,7 +561,9 @@ def run_dsa(args, world, rank, dist, dev):
             "topk": {"bound": "hbm", "frac": b_topk / (mean[1] / 1e3) / 1e9 / pk["hbm"]}},
         "launch": "cuda graph replay" if graph is not None else "eager",
         "e2e": {"value": w.B * w.T * world * args.e2e_steps / (e2e_ms / 1e3), "unit": DSA_UNIT,
-                "h2d_bytes_per_step": int(b_in), "d2h_bytes_per_step": int(b_sel), "steps": args.e2e_steps},
+                "h2d_bytes_per_step": int(b_in), "d2h_bytes_per_step": int(b_sel), "steps": args.e2e_steps,
+                "copies": "pinned host buffers, H2D and D2H on their own streams overlapping the compute of the "
+                          "neighbouring steps (two device buffer sets)"},
         "gpu_launches": DSA_KERNELS_PER_STEP * args.steps,
         "clocks": clocks,
     }
@@ -544,7 +594,7 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=0)
     ap.add_argument("--cpu-tokens", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--tokens", type=int, default=0, help="run the workload at this many tokens")
     ap.add_argument("--eager", action="store_true",
                     help="launch every step from the host instead of replaying a CUDA graph of it")
@@ -604,26 +654,28 @@ def main():
     x_dev = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
+    def step(ev=None, xin=None, yout=None):
+        xin = x_dev if xin is None else xin
+        yout = blk.y if yout is None else yout
         if dense:
             # one stage: the dense MLP (identity rows, up, down, combine)
             if ev is not None:
                 for j in range(4):
                     ev[j].record(stream)
-            moe.dense_mlp(cfg, blk.weights, x_dev, blk.ws, y=blk.y)
+            moe.dense_mlp(cfg, blk.weights, xin, blk.ws, y=yout)
             if ev is not None:
                 for j in range(4, 7):
                     ev[j].record(stream)
             return
         if ev is not None:
             ev[0].record(stream)
-        moe.route(cfg, x_dev, blk.w_router, blk.bias, blk.ws, out=(blk.idx, blk.gate, blk.margin))
+        moe.route(cfg, xin, blk.w_router, blk.bias, blk.ws, out=(blk.idx, blk.gate, blk.margin))
         if ev is not None:
             ev[1].record(stream)
         moe.permute(cfg, blk.idx, blk.ws, out=(blk.counts, blk.offsets, blk.sorted))
         if ev is not None:
             ev[2].record(stream)
-        moe.gather_tokens(cfg, x_dev, blk.sorted, blk.ws)
+        moe.gather_tokens(cfg, xin, blk.sorted, blk.ws)
         if ev is not None:
             ev[3].record(stream)
         moe.expert_up(cfg, blk.weights, blk.offsets, blk.sorted, blk.ws)
@@ -632,7 +684,7 @@ def main():
         moe.expert_down(cfg, blk.weights, blk.gate, blk.offsets, blk.sorted, blk.ws)
         if ev is not None:
             ev[5].record(stream)
-        moe.combine(cfg, blk.ws, blk.y)
+        moe.combine(cfg, blk.ws, yout)
         if ev is not None:
             ev[6].record(stream)
 
@@ -688,32 +740,28 @@ def main():
     t_max = max_over_ranks(total_ms, dist, dev)
     value = aggregate_tokens_per_s(w.T, world, args.steps, t_max)
 
-    # ---- end to end: pinned host x in, result out, every step
+    # ---- end to end: every step copies its token batch in from pinned host
+    # memory and its output back to the host.  Two device buffer sets and
+    # separate copy streams let step i + 1's input copy and step i - 1's output
+    # copy run under step i's compute (the copies of every timed step are inside
+    # the timed region).
     x_host = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
-    y_host = torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory()
-    x_in = torch.empty_like(x_dev)
-
-    def e2e_step():
-        if graph is not None:
-            x_dev.copy_(x_host, non_blocking=True)  # into the buffer the graph reads
-            graph.replay()
-        else:
-            x_in.copy_(x_host, non_blocking=True)
-            blk(x_in)
-        y_host.copy_(blk.y, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize()
-    a = torch.cuda.Event(enable_timing=True)
-    z = torch.cuda.Event(enable_timing=True)
-    if dist is not None:
-        dist.barrier()
-    a.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    z.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(a.elapsed_time(z), dist, dev)
+    xs = [x_dev, torch.empty_like(x_dev)]
+    ys = [blk.y, torch.empty_like(blk.y)]
+    y_host = [torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    replays = [graph.replay if graph is not None else (lambda: step(xin=xs[0], yout=ys[0]))]
+    if graph is not None:
+        step(xin=xs[1], yout=ys[1])
+        torch.cuda.synchronize()
+        graph1 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph1):
+            step(xin=xs[1], yout=ys[1])
+        replays.append(graph1.replay)
+    else:
+        replays.append(lambda: step(xin=xs[1], yout=ys[1]))
+    e2e_ms = pipelined_e2e(torch, stream, dev, args.e2e_steps, dist,
+                           lambda j: xs[j].copy_(x_host, non_blocking=True), replays,
+                           lambda j: y_host[j].copy_(ys[j], non_blocking=True))
     e2e_value = aggregate_tokens_per_s(w.T, world, args.e2e_steps, e2e_ms)
     if moe.device_error(blk.ws) != 0:
         raise RuntimeError("device error during the timed steps")
@@ -796,7 +844,9 @@ def main():
             "max_count": int(counts[: w.E].max()), "min_count": int(counts[: w.E].min()),
             "near_ties": int((blk.margin <= 1e-4).sum().item())},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(w.T * H * 2),
-                "d2h_bytes_per_step": int(w.T * H * 2), "steps": args.e2e_steps},
+                "d2h_bytes_per_step": int(w.T * H * 2), "steps": args.e2e_steps,
+                "copies": "pinned host buffers, H2D and D2H on their own streams overlapping the compute of the "
+                          "neighbouring steps (two device buffer sets)"},
         "gpu_launches": (KERNELS_PER_DENSE_STEP if dense else kernels_per_step(w)) * args.steps,
         "cublas_same_gemms_ms": cublas_ms,
         "clocks": clocks,

@@ -62,6 +62,17 @@ def peaks():
     return dict(hbm=6650.0, tflops=1590.0, tflops_sustained=1400.0, source="fallback")
 
 
+def tensor_peak(pk, timed_loop_ms):
+    """The bf16 peak a tensor-bound kernel is judged against: the sustained
+    figure (cuBLAS back to back for seconds, under the board power cap) when the
+    kernel was timed inside a timed loop of at least half a second, else the
+    burst figure (a kernel timed alone).  Returns (TFLOP/s, description)."""
+    if timed_loop_ms >= 500.0:
+        return pk["tflops_sustained"], "sustained bf16 (cuBLAS back to back), %s; timed loop %.2f s" % (
+            pk["source"], timed_loop_ms / 1e3)
+    return pk["tflops"], "burst bf16 (cuBLAS), %s; timed loop %.2f s" % (pk["source"], timed_loop_ms / 1e3)
+
+
 # ------------------------------------------------------------------ clocks
 
 CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -532,20 +543,20 @@ def run_dsa(args, world, rank, dist, dev):
     b_score = b_in + pairs * 4       # inputs + the scores it writes
     b_topk = pairs * 4 + b_sel       # the visible scores read + the selection written
     mean = stage.mean(axis=0)
-    ridge = pk["tflops"] * 1e12 / (pk["hbm"] * 1e9)
+    tpk, tpk_kind = tensor_peak(pk, total_ms)
+    ridge = tpk * 1e12 / (pk["hbm"] * 1e9)
     kernels = [("dsa_score_kernel", f_score, b_score, mean[0]), ("dsa_topk_kernel", 0.0, b_topk, mean[1])]
     name, f, by, ms = max(kernels, key=lambda x: x[3])
     if f > 0 and f / by > ridge:
-        roof = {"kernel": name, "bound": "tensor", "achieved": f / (ms / 1e3) / 1e12, "peak": pk["tflops"],
-                "unit": "TFLOP/s", "peak_kind": "burst bf16 (cuBLAS), " + pk["source"],
-                "algorithmic_per_launch": f}
+        roof = {"kernel": name, "bound": "tensor", "achieved": f / (ms / 1e3) / 1e12, "peak": tpk,
+                "unit": "TFLOP/s", "peak_kind": tpk_kind, "algorithmic_per_launch": f}
     else:
         roof = {"kernel": name, "bound": "hbm", "achieved": by / (ms / 1e3) / 1e9, "peak": pk["hbm"],
                 "unit": "GB/s", "peak_kind": "copy bandwidth, " + pk["source"], "algorithmic_per_launch": by}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = measured_traffic(w.name, name)
     step_s = t_max / 1e3 / args.steps
-    t_roof = max(f_score / (pk["tflops"] * 1e12), (b_in + b_sel) / (pk["hbm"] * 1e9))
+    t_roof = max(f_score / (tpk * 1e12), (b_in + b_sel) / (pk["hbm"] * 1e9))
     line = {
         "metric": DSA_METRIC, "value": value, "unit": DSA_UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -556,7 +567,7 @@ def run_dsa(args, world, rank, dist, dev):
         "stage_ms": {"scores": float(mean[0]), "topk": float(mean[1])},
         "stage_roofline": {
             "scores": {"bound": "tensor" if f_score / b_score > ridge else "hbm",
-                       "frac": (f_score / (mean[0] / 1e3) / 1e12 / pk["tflops"]) if f_score / b_score > ridge
+                       "frac": (f_score / (mean[0] / 1e3) / 1e12 / tpk) if f_score / b_score > ridge
                        else (b_score / (mean[0] / 1e3) / 1e9 / pk["hbm"])},
             "topk": {"bound": "hbm", "frac": b_topk / (mean[1] / 1e3) / 1e9 / pk["hbm"]}},
         "launch": "cuda graph replay" if graph is not None else "eager",
@@ -804,7 +815,8 @@ def main():
     if dense:
         names[3] = "dense_mlp"
     dom = int(np.argmax(mean_stage))
-    ridge = pk["tflops"] * 1e12 / (pk["hbm"] * 1e9)
+    tpk, tpk_kind = tensor_peak(pk, total_ms)
+    ridge = tpk * 1e12 / (pk["hbm"] * 1e9)
     work = {"expert_up": (f_up, b_up), "expert_down": (f_down, b_down),
             "route": (f_router, w.T * H * 2 + w.E * H * 4 + w.T * w.K * 8),
             "permute": (0.0, w.T * w.K * 4 * 3 + rows * 4),
@@ -815,7 +827,8 @@ def main():
     dur_s = mean_stage[dom] / 1e3
     if f > 0 and f / by > ridge:
         roof = {"kernel": names[dom], "bound": "tensor", "achieved": f / dur_s / 1e12,
-                "peak": pk["tflops"], "unit": "TFLOP/s", "peak_kind": "burst bf16 (cuBLAS), " + pk["source"]}
+                "peak": tpk, "unit": "TFLOP/s", "peak_kind": tpk_kind,
+                "frac_of_burst": f / dur_s / 1e12 / pk["tflops"]}
     else:
         roof = {"kernel": names[dom], "bound": "hbm", "achieved": by / dur_s / 1e9, "peak": pk["hbm"],
                 "unit": "GB/s", "peak_kind": "copy bandwidth, " + pk["source"]}
@@ -825,7 +838,7 @@ def main():
     f_alg = f_router + f_up + f_down
     b_alg = touched * 3 * H * I * 2 + w.E * H * 4 + w.E * 4 + 2 * w.T * H * 2
     step_s = t_max / 1e3 / args.steps
-    t_roof = max(f_alg / (pk["tflops"] * 1e12), b_alg / (pk["hbm"] * 1e9))
+    t_roof = max(f_alg / (tpk * 1e12), b_alg / (pk["hbm"] * 1e9))
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

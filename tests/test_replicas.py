@@ -95,3 +95,16 @@ def test_visible_pairs_count():
         w = W.DsaWorkload("x", B=B, T=T, S=S)
         brute = sum(1 for b in range(B) for t in range(T) for s in range(S) if s <= S - T + t)
         assert bench.dsa_visible_pairs(w) == brute
+
+
+def test_tensor_peak_follows_the_timed_loop_length():
+    """A tensor-bound kernel timed inside a loop of at least 0.5 s is judged
+    against the sustained (power-capped) bf16 figure, a short loop against the
+    burst figure."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    pk = dict(tflops=1629.0, tflops_sustained=1389.6, hbm=6548.2, source="measured")
+    assert bench.tensor_peak(pk, 650.0)[0] == 1389.6
+    assert "sustained" in bench.tensor_peak(pk, 650.0)[1]
+    assert bench.tensor_peak(pk, 22.0)[0] == 1629.0

@@ -584,10 +584,16 @@ def run_dsa(args, world, rank, dist, dev):
 
         O.build()
         secs, nq = dsa_oracle_sample(w, args.cpu_tokens or 2 * cores(), (q, k, wt))
+        reps = 1
+        while secs < 10.0 and secs * (reps + 1) / reps < 30.0:  # about 10 s of oracle work
+            s_, q_ = dsa_oracle_sample(w, args.cpu_tokens or 2 * cores(), (q, k, wt))
+            secs += s_
+            nq += q_
+            reps += 1
         line["cpu_baseline"] = {"value": nq / secs, "unit": DSA_UNIT, "cores": int(os.environ["OMP_NUM_THREADS"]),
                                 "kind": "oracle",
-                                "sample": "scores + top-%d of %d queries (double-precision C oracle, OpenMP), "
-                                          "%.1f s" % (w.topk, nq, secs)}
+                                "sample": "scores + top-%d of %d queries, %d times (double-precision C oracle, "
+                                          "OpenMP), %.1f s" % (w.topk, nq // reps, reps, secs)}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -888,12 +894,16 @@ def main():
 
         tables = host_expert_tables(w, experts, getter)
         shared = [getter("w1", w.E), getter("w3", w.E), getter("w2", w.E)]
+        # the same bounded sample repeated until the oracle has worked about 10 s
+        # (at most ~30 s): more tokens would make the host hold more experts' weights
         times = run_oracle_steps(w, x, w_r, b, tokens, tables, shared, 1)
+        while sum(times) < 10.0 and sum(times) + times[0] < 30.0:
+            times += run_oracle_steps(w, x, w_r, b, tokens, tables, shared, 1)
         line["cpu_baseline"] = {
-            "value": len(tokens) / times[0], "unit": UNIT, "cores": int(os.environ["OMP_NUM_THREADS"]),
-            "kind": "oracle",
-            "sample": "route+permute+forward of %d of the %d tokens (double-precision C oracle, OpenMP), "
-                      "%.1f s" % (len(tokens), w.T, times[0])}
+            "value": len(tokens) * len(times) / sum(times), "unit": UNIT,
+            "cores": int(os.environ["OMP_NUM_THREADS"]), "kind": "oracle",
+            "sample": "route+permute+forward of %d of the %d tokens, %d times (double-precision C oracle, "
+                      "OpenMP), %.1f s" % (len(tokens), w.T, len(times), sum(times))}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -33,9 +33,12 @@
  * moe_get_device_error(ws, ...).
  *
  * Supported shapes: NH in {32, 64, 128}, D in {64, 128}, 1 <= topk <= 65536,
- * 1 <= T <= S, B >= 1 (B == 0 is a no-op), B*T*NH < 2^31, B*S < 2^31,
- * B*T*S < 2^40.  q, k and the workspace must be 16-byte aligned; w, scores
- * and sel 4-byte aligned.
+ * 1 <= T <= S <= 32768 (the top-k holds a row's keys in registers),
+ * B >= 0 (B == 0 is a no-op), B*T*NH < 2^31, B*S < 2^31, B*T*S < 2^40.
+ * q, k, w and the workspace must be 16-byte aligned (w is read by a bulk
+ * copy); scores and sel 4-byte aligned.  Anything else returns
+ * MOE_ERR_UNSUPPORTED (shape), MOE_ERR_ARG (T < 1, S < T, topk < 1, B < 0)
+ * or MOE_ERR_ALIGN before any launch.
  */
 #ifndef SRM_DSA_H
 #define SRM_DSA_H
@@ -64,7 +67,7 @@ size_t dsa_workspace_size(const dsa_cfg_t *cfg);
 /* Indexer scores.
  *   q       bf16 [B][T][NH][D]   index queries (after their rotary step)
  *   k       bf16 [B][S][D]       index keys (after their norm and rotary step)
- *   w       fp32 [B][T][NH]      per-head weights (x W_w)
+ *   w       fp32 [B][T][NH]      per-head weights (x W_w), 16-byte aligned
  *   scores  fp32 [B][T][S]       out: S[t,s] for every key query t sees; the
  *                                entries s > S - T + t are not written
  * Errors: MOE_ERR_ARG (NULL pointer), MOE_ERR_UNSUPPORTED, MOE_ERR_ALIGN,

@@ -60,13 +60,13 @@ def test_cta_pair_tiles(T):
         assert np.any((rem > 0) & (rem <= 128)) and np.any(rem > 128)
 
 
-@pytest.mark.parametrize("T", [300, 2100])
+@pytest.mark.parametrize("T", [300, 8192])
 def test_widest_selection_256_experts_top16(T):
     """The largest supported routing: 256 experts, top-16 (the router's widest
-    expert tile, 16 selection rounds, 256 groups in the permutation); 2100
-    tokens give T*K >= 512*E, so the CTA-pair tiles run with 257 groups."""
+    expert tile, 16 selection rounds, 256 groups in the permutation); 8192
+    tokens give T*K = 512*E, so the CTA-pair tiles run with 257 groups."""
     w = W.WORKLOADS["tiny"].replace(E=256, K=16, T=T, seed=3300 + T)
-    assert (T * w.K >= 512 * w.E) == (T == 2100)
+    assert (T * w.K >= 512 * w.E) == (T == 8192)
     full_check(w, lambda res: MH.sample_tokens(res, w.T, 200))
 
 

@@ -170,3 +170,29 @@ def test_key_permutation_moves_the_selection_with_it():
     sel, _, _ = O.dsa_select(s, 11)
     selp, _, _ = O.dsa_select(sp, 11)
     assert sorted(perm[selp].tolist()) == sel.tolist()
+
+
+def test_the_2048_key_boundary():
+    """At the pages' index_topk = 2048: a query that sees exactly 2048 keys takes
+    them all; one that sees 2049 drops exactly its lowest-scored key (the page's
+    short-prompt rule and its first exception)."""
+    S = 2049
+    rng = np.random.default_rng(12)
+    scores = np.full((2, S), -np.inf)
+    scores[0, :2048] = rng.standard_normal(2048)      # sees keys 0 .. 2047
+    scores[1, :] = rng.standard_normal(S)             # sees all 2049
+    sel, kth, nxt = O.dsa_select(scores, GOLDEN["glm5_indexer"]["index_topk"])
+    assert sel[0].tolist() == list(range(2048)) and nxt[0] == -math.inf
+    dropped = int(np.argmin(scores[1]))
+    assert sel[1].tolist() == [s for s in range(S) if s != dropped]
+    assert nxt[1] == scores[1, dropped]
+
+
+def test_scores_of_a_cache_query_equal_those_of_a_prefill_row():
+    """Query t of a prefill (T = S) and the single query of a cached decode step at
+    the same position see the same keys and score them identically."""
+    q, k, w = rand_case(B=1, T=10, S=10, seed=13)
+    pre = O.dsa_scores(q, k, w)[0]
+    for t in (0, 4, 9):
+        dec = O.dsa_scores(q[:, t:t + 1], k[:, :t + 1], w[:, t:t + 1])[0, 0]
+        assert np.array_equal(dec, pre[t, :t + 1])

@@ -108,3 +108,17 @@ def test_tensor_peak_follows_the_timed_loop_length():
     assert bench.tensor_peak(pk, 650.0)[0] == 1389.6
     assert "sustained" in bench.tensor_peak(pk, 650.0)[1]
     assert bench.tensor_peak(pk, 22.0)[0] == 1629.0
+
+
+def test_launches_per_step_match_the_kernel_structure():
+    """The bench's gpu_launches claim: decode runs W_r split, split-K logits,
+    their reduction, selection, the one-CTA permutation, invert, gather, up,
+    down, combine (10 kernels, as the ncu launch list shows); prefill runs the
+    router without split-K and the three-kernel permutation (11)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from sigmoid_routed_mixture_b200 import workloads as W
+
+    assert bench.kernels_per_step(W.WORKLOADS["glm5_decode"]) == 10
+    assert bench.kernels_per_step(W.WORKLOADS["glm5_prefill"]) == 11
+    assert bench.DSA_KERNELS_PER_STEP == 3  # plan, scores, top-k

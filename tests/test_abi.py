@@ -153,3 +153,42 @@ def test_dsa_no_sequences_is_a_no_op(L):
     dsa.lib()
     c = dsa_cfg(B=0).c()
     assert L.dsa_select(ctypes.byref(c), None, None, None, None, None, None, 0, None) == 0
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include "srm_moe.h"
+#include "srm_dsa.h"
+
+int main(void) {
+    moe_cfg_t cfg = {16384, 6144, 2048, 256, 8, 2.5f, 1};
+    dsa_cfg_t kcfg = {4, 4096, 4096, 32, 128, 2048};
+    size_t a = moe_workspace_size(&cfg), b = dsa_workspace_size(&kcfg);
+    moe_cfg_t bad = cfg;
+    bad.K = 0;
+    /* host validation only: no pointer is dereferenced, nothing is launched */
+    moe_status_t st = moe_route(&bad, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0);
+    printf("%zu %zu %d %s\n", a, b, (int)st, moe_status_string(MOE_ERR_ARG));
+    return (a > 0 && b > 0 && st == MOE_ERR_ARG) ? 0 : 1;
+}
+"""
+
+
+def test_headers_are_plain_c_and_link(L, tmp_path):
+    """include/*.h compile as C99 and a C program links against the library and
+    calls its host-side entry points (no GPU needed)."""
+    import subprocess
+
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    lib_dir = os.path.dirname(moe.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                        "-L", lib_dir, "-lsrm_moe", "-Wl,-rpath," + lib_dir, "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    a, b, st, msg = r.stdout.split(maxsplit=3)
+    assert int(a) == moe.workspace_bytes(moe.Config(16384, 6144, 2048, 256, 8))
+    assert int(st) == 1 and msg.strip() == "invalid argument"

@@ -180,6 +180,65 @@ def test_selection_equals_best_subset_brute_force():
         assert margin[0] == pytest.approx(min(key[list(best[1])]) - max(key[rest]), abs=1e-15)
 
 
+def test_gates_for_given_selection_closed_forms():
+    """Gates of a GIVEN selection (the GPU's own choice in every output check):
+    G_slot = scale * s_idx[slot] / sum over the selection of s, s = sigmoid(z),
+    the un-biased sigmoids ("All 43 steps", G_i; nnterp section 03 note: the
+    weights are the un-biased scores renormalised, times the routed scale).
+
+    The 1-token example of test_worked_example_by_hand: z = (2, -1, 0.5, 1).  A
+    forced selection (0, 3) -- not the biased choice (0, 1) -- must give
+    2.5 s0/(s0+s3), 2.5 s3/(s0+s3) in slot order; the reversed order (3, 0)
+    swaps them.  A dropped scale, a sum over all four experts, a sum over the
+    biased keys or a gate read at the slot number instead of the expert id each
+    fails one of these."""
+    sig = lambda v: 1.0 / (1.0 + math.exp(-v))  # noqa: E731
+    z = np.array([[2.0, -1.0, 0.5, 1.0]])
+    s0, s3 = sig(2.0), sig(1.0)
+    g = O.gates_for(z, np.array([[0, 3]], dtype=np.int32), 2.5)
+    assert g[0, 0] == pytest.approx(2.5 * s0 / (s0 + s3), rel=1e-15, abs=0)
+    assert g[0, 1] == pytest.approx(2.5 * s3 / (s0 + s3), rel=1e-15, abs=0)
+    g = O.gates_for(z, np.array([[3, 0]], dtype=np.int32), 1.8)
+    assert g[0, 0] == pytest.approx(1.8 * s3 / (s0 + s3), rel=1e-15, abs=0)
+    assert g[0, 1] == pytest.approx(1.8 * s0 / (s0 + s3), rel=1e-15, abs=0)
+    # one selected expert takes the whole scale, whatever its score
+    g = O.gates_for(z, np.array([[1]], dtype=np.int32), 2.5)
+    assert g[0, 0] == 2.5
+    # equal logits (s = 1/2 everywhere): every gate is scale / K for any selection
+    zt = np.zeros((3, 10))
+    sel = np.array([[9, 0, 4], [2, 3, 1], [7, 8, 5]], dtype=np.int32)
+    assert np.all(O.gates_for(zt, sel, 2.5) == 2.5 / 3)
+
+
+def test_gates_for_sum_ratio_and_out_of_range():
+    """For any selection the gates sum to the scale (to 1e-12) and the ratio of
+    two slots' gates is the ratio of their sigmoids, s_a / s_b, exactly the
+    ratio of 1/(1+exp(-z)) values (a closed form independent of the sum)."""
+    rng = np.random.default_rng(5)
+    T, E, K = 40, 16, 5
+    z = rng.standard_normal((T, E)) * 3.0
+    idx = np.array([rng.permutation(E)[:K] for _ in range(T)], dtype=np.int32)
+    g = O.gates_for(z, idx, 2.5)
+    assert np.max(np.abs(g.sum(axis=1) - 2.5)) <= 1e-12
+    s = 1.0 / (1.0 + np.exp(-z))
+    for t in range(T):
+        for a in range(1, K):
+            assert g[t, a] / g[t, 0] == pytest.approx(s[t, idx[t, a]] / s[t, idx[t, 0]], rel=1e-13)
+    # scale enters linearly
+    np.testing.assert_allclose(O.gates_for(z, idx, 1.8), g * (1.8 / 2.5), rtol=1e-15, atol=0)
+    # the given selection is used as is: select's own choice under a bias that
+    # forces experts {1, 4, 6} gives the same gates as the forced selection
+    b = np.zeros(E, np.float32)
+    b[[1, 4, 6]] = 10.0
+    i_b, g_b, _ = O.select(z, b, 3, 2.5)
+    np.testing.assert_allclose(O.gates_for(z, i_b, 2.5), g_b, rtol=1e-15, atol=0)
+    for bad in (E, -1):
+        wrong = idx.copy()
+        wrong[3, 2] = bad
+        with pytest.raises(ValueError):
+            O.gates_for(z, wrong, 2.5)
+
+
 def test_permute_brute_force_and_invariants():
     rng = np.random.default_rng(11)
     for T, E, K, has_shared in [(37, 8, 3, True), (1, 4, 4, True), (50, 16, 2, False), (0, 8, 2, True)]:

@@ -39,15 +39,11 @@ KERNELS_PER_DENSE_STEP = 4  # identity rows 1 + up 1 + down 1 + combine 1
 
 
 def kernels_per_step(w, num_sms=148):
-    """Kernel launches of one routed step: router split + logits (+ split-K
-    reduction when the H range is split) + select; permutation (one CTA for
-    small batches, else histogram + scan + scatter); token gather (invert +
-    scatter); up GEMM; down GEMM; combine."""
-    m_tiles = -(-w.T // 128)
-    kblocks = w.H // 64
-    splits = max(1, min(num_sms // max(1, m_tiles), max(1, kblocks // 2)))
-    kb_per = -(-kblocks // splits)
-    route = 3 + (1 if -(-kblocks // kb_per) > 1 else 0)
+    """Kernel launches of one routed step: the router (one kernel: logits,
+    selection and gates, with the router weights split once at pack time);
+    permutation (one CTA for small batches, else histogram + scan + scatter);
+    token gather (invert + scatter); up GEMM; down GEMM; combine."""
+    route = 1
     permute = 1 if w.T * w.K <= 16384 else 3
     return route + permute + 2 + 1 + 1 + 1
 
@@ -600,6 +596,223 @@ def run_dsa(args, world, rank, dist, dev):
 
 # ------------------------------------------------------------------ our arm
 
+STAGES = ["route", "permute", "gather_tokens", "expert_up", "expert_down", "combine"]
+
+
+def build_step(cfg, blk, x_dev, dense, stream):
+    """One pass of the hot path on `stream`; with `ev` (7 events) it records the
+    stage boundaries.  xin / yout replace the block's input and output buffers."""
+    from sigmoid_routed_mixture_b200 import moe
+
+    def step(ev=None, xin=None, yout=None):
+        xin = x_dev if xin is None else xin
+        yout = blk.y if yout is None else yout
+        if dense:
+            # one stage: the dense MLP (identity rows, up, down, combine)
+            if ev is not None:
+                for j in range(4):
+                    ev[j].record(stream)
+            moe.dense_mlp(cfg, blk.weights, xin, blk.ws, y=yout)
+            if ev is not None:
+                for j in range(4, 7):
+                    ev[j].record(stream)
+            return
+        if ev is not None:
+            ev[0].record(stream)
+        moe.route_packed(cfg, xin, blk.router_packed, blk.bias, blk.ws, out=(blk.idx, blk.gate, blk.margin))
+        if ev is not None:
+            ev[1].record(stream)
+        moe.permute(cfg, blk.idx, blk.ws, out=(blk.counts, blk.offsets, blk.sorted))
+        if ev is not None:
+            ev[2].record(stream)
+        moe.gather_tokens(cfg, xin, blk.sorted, blk.ws)
+        if ev is not None:
+            ev[3].record(stream)
+        moe.expert_up(cfg, blk.weights, blk.offsets, blk.sorted, blk.ws)
+        if ev is not None:
+            ev[4].record(stream)
+        moe.expert_down(cfg, blk.weights, blk.gate, blk.offsets, blk.sorted, blk.ws)
+        if ev is not None:
+            ev[5].record(stream)
+        moe.combine(cfg, blk.ws, yout)
+        if ev is not None:
+            ev[6].record(stream)
+
+    return step
+
+
+def measure_block(step, ws, steps, warmup, eager, dist, stream):
+    """Warm-up, then EXACTLY `steps` timed steps (CUDA-graph replays, or host
+    launches with `eager`) between a barrier and device synchronisations, with
+    the SM clocks sampled meanwhile; then the same number of host-launched
+    steps with events at the stage boundaries (they only feed the stage shares
+    and the kernel roofline).  Returns a dict of the timings and the graph."""
+    import torch
+
+    from sigmoid_routed_mixture_b200 import moe
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if moe.device_error(ws) != 0:
+        raise RuntimeError("device error during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(torch.cuda.current_device())
+    graph = None
+    if not eager:
+        # the step captured once as a CUDA graph and replayed: every kernel of
+        # every step still runs; only the host launch gaps go away
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(warmup):
+            graph.replay()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    e_start.record(stream)
+    for i in range(steps):
+        if graph is not None:
+            graph.replay()
+        else:
+            step(evs[i])
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dist is not None:
+        dist.barrier()
+    total_ms = e_start.elapsed_time(e_end)
+    eager_ms = total_ms
+    if graph is not None:
+        e_start.record(stream)
+        for i in range(steps):
+            step(evs[i])
+        e_end.record(stream)
+        torch.cuda.synchronize()
+        eager_ms = e_start.elapsed_time(e_end)
+    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(6)] for i in range(steps)])
+    if moe.device_error(ws) != 0:
+        raise RuntimeError("device error during the timed steps")
+    return dict(graph=graph, total_ms=total_ms, eager_ms=eager_ms, stage_ms=stage_ms, clocks=clocks)
+
+
+def block_record(w, cfg, blk, meas, t_max, steps, pk, dense):
+    """Roofline of the dominant kernel, the block roofline and the routing
+    statistics of one measured block (the algorithmic work of the method, from
+    this run's own expert counts)."""
+    counts = blk.counts.cpu().numpy()
+    touched = (int((counts[: w.E] > 0).sum()) if not dense else 0) + int(w.has_shared)
+    rows = cfg.rows
+    H, I = w.H, w.I
+    f_router = 2.0 * w.T * H * w.E
+    f_up = 2.0 * rows * H * 2 * I
+    f_down = 2.0 * rows * I * H
+    # algorithmic bytes: weights of the touched groups plus the block's own
+    # input (x) or output (y); intermediates (gathered rows, h, slot outputs)
+    # are implementation choices and are not counted
+    b_up = touched * 2 * I * H * 2 + w.T * H * 2
+    b_down = touched * H * I * 2 + w.T * H * 2
+    mean_stage = meas["stage_ms"].mean(axis=0)
+    names = list(STAGES)
+    if dense:
+        names[3] = "dense_mlp"
+    dom = int(np.argmax(mean_stage))
+    tpk, tpk_kind = tensor_peak(pk, meas["total_ms"])
+    ridge = tpk * 1e12 / (pk["hbm"] * 1e9)
+    work = {"expert_up": (f_up, b_up), "expert_down": (f_down, b_down),
+            "route": (f_router, w.T * H * 2 + w.E * H * 4 + w.T * w.K * 8),
+            "permute": (0.0, w.T * w.K * 4 * 3 + rows * 4),
+            "gather_tokens": (0.0, w.T * H * 2 + rows * H * 2),
+            "combine": (0.0, rows * H * 2 + w.T * H * 2),
+            "dense_mlp": (f_up + f_down, 3 * H * I * 2 + 2 * w.T * H * 2)}
+    f, by = work[names[dom]]
+    dur_s = mean_stage[dom] / 1e3
+    if f > 0 and f / by > ridge:
+        roof = {"kernel": names[dom], "bound": "tensor", "achieved": f / dur_s / 1e12,
+                "peak": tpk, "unit": "TFLOP/s", "peak_kind": tpk_kind,
+                "frac_of_burst": f / dur_s / 1e12 / pk["tflops"]}
+    else:
+        roof = {"kernel": names[dom], "bound": "hbm", "achieved": by / dur_s / 1e9, "peak": pk["hbm"],
+                "unit": "GB/s", "peak_kind": "copy bandwidth, " + pk["source"]}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = measured_traffic(w.name, names[dom])
+    roof["algorithmic_per_launch"] = f if roof["bound"] == "tensor" else by
+    f_alg = f_router + f_up + f_down
+    b_alg = touched * 3 * H * I * 2 + w.E * H * 4 + w.E * 4 + 2 * w.T * H * 2
+    step_s = t_max / 1e3 / steps
+    t_roof = max(f_alg / (tpk * 1e12), b_alg / (pk["hbm"] * 1e9))
+    return {
+        "roofline": roof,
+        "block_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof / step_s,
+                           "bound": "tensor" if f_alg / (tpk * 1e12) >= b_alg / (pk["hbm"] * 1e9) else "hbm",
+                           "f_alg_tflop": f_alg / 1e12, "b_alg_gb": b_alg / 1e9},
+        "stage_ms": {n: float(v) for n, v in zip(names, mean_stage)},
+        "routing": None if dense else {
+            "touched_groups": touched, "zero_count_experts": int((counts[: w.E] == 0).sum()),
+            "max_count": int(counts[: w.E].max()), "min_count": int(counts[: w.E].min()),
+            "near_ties": int((blk.margin <= 1e-4).sum().item())},
+    }
+
+
+def steps_for(step, stream, target_ms=250.0, lo=20, hi=4000):
+    """Steps whose timed loop lasts about target_ms (estimated from 5 host-launched steps)."""
+    import torch
+
+    a = torch.cuda.Event(enable_timing=True)
+    z = torch.cuda.Event(enable_timing=True)
+    step()
+    a.record(stream)
+    for _ in range(5):
+        step()
+    z.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(z) / 5
+    return int(min(hi, max(lo, -(-target_ms // max(ms, 1e-3)))))
+
+
+def also_records(args, dev, stream, pk, packed):
+    """The other block configurations, each timed like the headline (CUDA-graph
+    replays, >= 0.25 s of timed loop, clocks sampled): the 64-token decode block
+    and the 8192-token skewed block on the headline's packed GLM-5 expert weights
+    (same shapes and distribution), and the GLM-4.7-Flash-shaped block on its own."""
+    import torch
+
+    from sigmoid_routed_mixture_b200 import moe
+
+    out = {}
+    for name in ("glm5_decode", "glm5_skewed", "glm47flash"):
+        w = W.WORKLOADS[name]
+        x, w_r, b = W.router_inputs(w)
+        cfg = moe.Config.of(w)
+        w_r_dev, b_dev = torch.from_numpy(w_r).to(dev), torch.from_numpy(b).to(dev)
+        if name == "glm47flash":
+            blk = moe.MoeBlock(cfg, w_r_dev, b_dev, **W.expert_weights(w, dev))
+            weights_note = "its own seeded weights"
+        else:
+            blk = moe.MoeBlock(cfg, w_r_dev, b_dev, None, None, None, packed=packed)
+            weights_note = "the headline block's packed GLM-5 expert weights (same shapes and distribution)"
+        torch.cuda.empty_cache()
+        x_dev = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        step = build_step(cfg, blk, x_dev, False, stream)
+        steps = steps_for(step, stream)
+        meas = measure_block(step, blk.ws, steps, args.warmup, args.eager, None, stream)
+        rec = {"value": w.T * steps / (meas["total_ms"] / 1e3), "unit": UNIT,
+               "ms_per_step": meas["total_ms"] / steps, "steps": steps, "warmup": args.warmup,
+               "tokens": w.T, "weights": weights_note,
+               "launch": "cuda graph replay" if meas["graph"] is not None else "eager",
+               "gpu_launches": kernels_per_step(w) * steps, "clocks": meas["clocks"]}
+        rec.update(block_record(w, cfg, blk, meas, meas["total_ms"], steps, pk, False))
+        out[name] = rec
+        del meas, blk, step, x_dev
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -611,6 +824,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=0)
     ap.add_argument("--cpu-tokens", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-also", action="store_true",
+                    help="glm5_prefill at N = 1: skip timing the decode, skewed and GLM-4.7-Flash blocks")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--tokens", type=int, default=0, help="run the workload at this many tokens")
     ap.add_argument("--eager", action="store_true",
@@ -670,90 +885,10 @@ def main():
     torch.cuda.empty_cache()
     x_dev = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
     stream = torch.cuda.current_stream()
-
-    def step(ev=None, xin=None, yout=None):
-        xin = x_dev if xin is None else xin
-        yout = blk.y if yout is None else yout
-        if dense:
-            # one stage: the dense MLP (identity rows, up, down, combine)
-            if ev is not None:
-                for j in range(4):
-                    ev[j].record(stream)
-            moe.dense_mlp(cfg, blk.weights, xin, blk.ws, y=yout)
-            if ev is not None:
-                for j in range(4, 7):
-                    ev[j].record(stream)
-            return
-        if ev is not None:
-            ev[0].record(stream)
-        moe.route(cfg, xin, blk.w_router, blk.bias, blk.ws, out=(blk.idx, blk.gate, blk.margin))
-        if ev is not None:
-            ev[1].record(stream)
-        moe.permute(cfg, blk.idx, blk.ws, out=(blk.counts, blk.offsets, blk.sorted))
-        if ev is not None:
-            ev[2].record(stream)
-        moe.gather_tokens(cfg, xin, blk.sorted, blk.ws)
-        if ev is not None:
-            ev[3].record(stream)
-        moe.expert_up(cfg, blk.weights, blk.offsets, blk.sorted, blk.ws)
-        if ev is not None:
-            ev[4].record(stream)
-        moe.expert_down(cfg, blk.weights, blk.gate, blk.offsets, blk.sorted, blk.ws)
-        if ev is not None:
-            ev[5].record(stream)
-        moe.combine(cfg, blk.ws, yout)
-        if ev is not None:
-            ev[6].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if moe.device_error(blk.ws) != 0:
-        raise RuntimeError("device error during warm-up")
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
-    e_start = torch.cuda.Event(enable_timing=True)
-    e_end = torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(torch.cuda.current_device())
-    graph = None
-    if not args.eager:
-        # the step captured once as a CUDA graph and replayed: every kernel of
-        # every step still runs; only the host launch gaps go away
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            step()
-        for _ in range(args.warmup):
-            graph.replay()
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.3)
-    # the timed steps (value): graph replays, or host launches with --eager
-    e_start.record(stream)
-    for i in range(args.steps):
-        if graph is not None:
-            graph.replay()
-        else:
-            step(evs[i])
-    e_end.record(stream)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    if dist is not None:
-        dist.barrier()
-    total_ms = e_start.elapsed_time(e_end)
-    eager_ms = total_ms
-    if graph is not None:
-        # per-stage breakdown from the same number of host-launched steps, after
-        # the timed ones (it only feeds the stage shares and the kernel roofline)
-        e_start.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        e_end.record(stream)
-        torch.cuda.synchronize()
-        eager_ms = e_start.elapsed_time(e_end)
-    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(6)]
-                         for i in range(args.steps)])
+    step = build_step(cfg, blk, x_dev, dense, stream)
+    meas = measure_block(step, blk.ws, args.steps, args.warmup, args.eager, dist, stream)
+    graph = meas["graph"]
+    total_ms = meas["total_ms"]
     t_max = max_over_ranks(total_ms, dist, dev)
     value = aggregate_tokens_per_s(w.T, world, args.steps, t_max)
 
@@ -767,6 +902,7 @@ def main():
     ys = [blk.y, torch.empty_like(blk.y)]
     y_host = [torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     replays = [graph.replay if graph is not None else (lambda: step(xin=xs[0], yout=ys[0]))]
+    graph1 = None
     if graph is not None:
         step(xin=xs[1], yout=ys[1])
         torch.cuda.synchronize()
@@ -802,73 +938,27 @@ def main():
         cublas_ms = {"up": loop(lambda: torch.matmul(x_dev, w13_t.t())),
                      "down": loop(lambda: torch.matmul(h_t, w2_t.t()))}
 
-    # ---- algorithmic work and the roofline of the dominant kernel
-    counts = blk.counts.cpu().numpy()
-    touched = (int((counts[: w.E] > 0).sum()) if not dense else 0) + int(w.has_shared)
-    rows = cfg.rows
-    H, I = w.H, w.I
-    f_router = 2.0 * w.T * H * w.E
-    f_up = 2.0 * rows * H * 2 * I
-    f_down = 2.0 * rows * I * H
-    # algorithmic bytes: weights of the touched groups plus the block's own
-    # input (x) or output (y); intermediates (gathered rows, h, slot outputs)
-    # are implementation choices and are not counted
-    b_up = touched * 2 * I * H * 2 + w.T * H * 2
-    b_down = touched * H * I * 2 + w.T * H * 2
     pk = peaks()
-    mean_stage = stage_ms.mean(axis=0)
-    names = ["route", "permute", "gather_tokens", "expert_up", "expert_down", "combine"]
-    if dense:
-        names[3] = "dense_mlp"
-    dom = int(np.argmax(mean_stage))
-    tpk, tpk_kind = tensor_peak(pk, total_ms)
-    ridge = tpk * 1e12 / (pk["hbm"] * 1e9)
-    work = {"expert_up": (f_up, b_up), "expert_down": (f_down, b_down),
-            "route": (f_router, w.T * H * 2 + w.E * H * 4 + w.T * w.K * 8),
-            "permute": (0.0, w.T * w.K * 4 * 3 + rows * 4),
-            "gather_tokens": (0.0, w.T * H * 2 + rows * H * 2),
-            "combine": (0.0, rows * H * 2 + w.T * H * 2),
-            "dense_mlp": (f_up + f_down, 3 * H * I * 2 + 2 * w.T * H * 2)}
-    f, by = work[names[dom]]
-    dur_s = mean_stage[dom] / 1e3
-    if f > 0 and f / by > ridge:
-        roof = {"kernel": names[dom], "bound": "tensor", "achieved": f / dur_s / 1e12,
-                "peak": tpk, "unit": "TFLOP/s", "peak_kind": tpk_kind,
-                "frac_of_burst": f / dur_s / 1e12 / pk["tflops"]}
-    else:
-        roof = {"kernel": names[dom], "bound": "hbm", "achieved": by / dur_s / 1e9, "peak": pk["hbm"],
-                "unit": "GB/s", "peak_kind": "copy bandwidth, " + pk["source"]}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = measured_traffic(w.name, names[dom])
-    roof["algorithmic_per_launch"] = f if roof["bound"] == "tensor" else by
-    f_alg = f_router + f_up + f_down
-    b_alg = touched * 3 * H * I * 2 + w.E * H * 4 + w.E * 4 + 2 * w.T * H * 2
-    step_s = t_max / 1e3 / args.steps
-    t_roof = max(f_alg / (tpk * 1e12), b_alg / (pk["hbm"] * 1e9))
-
+    rec = block_record(w, cfg, blk, meas, t_max, args.steps, pk, dense)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init weights of the GLM-5 MoE block shapes)",
         "config": workload_config(w, argparse.Namespace(gpus=world)),
-        "roofline": roof,
-        "block_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof / step_s,
-                           "f_alg_tflop": f_alg / 1e12, "b_alg_gb": b_alg / 1e9},
-        "stage_ms": {n: float(v) for n, v in zip(names, mean_stage)},
+        "roofline": rec["roofline"],
+        "block_roofline": rec["block_roofline"],
+        "stage_ms": rec["stage_ms"],
         "launch": "cuda graph replay" if graph is not None else "eager",
-        "eager_ms_per_step": eager_ms / args.steps,
-        "routing": None if dense else {
-            "touched_groups": touched, "zero_count_experts": int((counts[: w.E] == 0).sum()),
-            "max_count": int(counts[: w.E].max()), "min_count": int(counts[: w.E].min()),
-            "near_ties": int((blk.margin <= 1e-4).sum().item())},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(w.T * H * 2),
-                "d2h_bytes_per_step": int(w.T * H * 2), "steps": args.e2e_steps,
+        "eager_ms_per_step": meas["eager_ms"] / args.steps,
+        "routing": rec["routing"],
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(w.T * w.H * 2),
+                "d2h_bytes_per_step": int(w.T * w.H * 2), "steps": args.e2e_steps,
                 "copies": "pinned host buffers, H2D and D2H on their own streams overlapping the compute of the "
                           "neighbouring steps (two device buffer sets)"},
         "gpu_launches": (KERNELS_PER_DENSE_STEP if dense else kernels_per_step(w)) * args.steps,
         "cublas_same_gemms_ms": cublas_ms,
-        "clocks": clocks,
+        "clocks": meas["clocks"],
     }
 
     # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N = 1 only
@@ -882,14 +972,14 @@ def main():
         tokens = oracle_sample_tokens(w, idx, n)
         experts = set(np.unique(idx[tokens]).tolist())
         w13, w2p = blk.weights
+        H, I = w.H, w.I
 
         def getter(name, e):
-            if name == "w1":
-                rows_ = [w13[(e * 2 * I + j * 256): (e * 2 * I + j * 256 + 128)] for j in range(2 * I // 256)]
-                return W.torch_bf16_to_bits(torch.cat(rows_))
-            if name == "w3":
-                rows_ = [w13[(e * 2 * I + j * 256 + 128): (e * 2 * I + (j + 1) * 256)] for j in range(2 * I // 256)]
-                return W.torch_bf16_to_bits(torch.cat(rows_))
+            # packed W13 of group e: units of 32 rows, 16 W1 rows then the matching 16 W3 rows
+            if name in ("w1", "w3"):
+                units = w13[e * 2 * I:(e + 1) * 2 * I].view(I // 16, 32, H)
+                part = units[:, :16] if name == "w1" else units[:, 16:]
+                return W.torch_bf16_to_bits(part.reshape(I, H))
             return W.torch_bf16_to_bits(w2p[e * H:(e + 1) * H].to(torch.bfloat16))
 
         tables = host_expert_tables(w, experts, getter)
@@ -904,6 +994,13 @@ def main():
             "cores": int(os.environ["OMP_NUM_THREADS"]), "kind": "oracle",
             "sample": "route+permute+forward of %d of the %d tokens, %d times (double-precision C oracle, "
                       "OpenMP), %.1f s" % (len(tokens), w.T, len(times), sum(times))}
+
+    # ---- the other block configurations (after every timed region of the
+    # headline, so they cannot disturb it), rank 0 at N = 1 only
+    if world == 1 and not args.no_also and w.name == "glm5_prefill" and not args.tokens:
+        packed = blk.weights
+        del replays, graph, graph1, meas, step
+        line["also"] = also_records(args, dev, stream, pk, packed)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -71,7 +71,10 @@ size_t dsa_workspace_size(const dsa_cfg_t *cfg);
  *   scores  fp32 [B][T][S]       out: S[t,s] for every key query t sees; the
  *                                entries s > S - T + t are not written
  * Errors: MOE_ERR_ARG (NULL pointer), MOE_ERR_UNSUPPORTED, MOE_ERR_ALIGN,
- * MOE_ERR_WORKSPACE, MOE_ERR_CUDA; device: MOE_ERR_TIMEOUT. */
+ * MOE_ERR_WORKSPACE, MOE_ERR_CUDA; device: MOE_ERR_TIMEOUT.
+ * Test-only switch: SRM_MOE_INJECT_STALL=1 in the environment makes the
+ * score kernel issue no key copies, so its bounded waits run out and the
+ * call reports MOE_ERR_TIMEOUT (failure-detection tests; leave it unset). */
 moe_status_t dsa_scores(const dsa_cfg_t *cfg, const void *q, const void *k, const float *w,
                         float *scores, void *ws, size_t ws_bytes, void *stream);
 

@@ -49,7 +49,9 @@ typedef enum {
     MOE_ERR_UNSUPPORTED = 2,  /* shape outside the supported set listed above */
     MOE_ERR_ALIGN = 3,        /* pointer misaligned (see above) */
     MOE_ERR_WORKSPACE = 4,    /* ws_bytes < moe_workspace_size(cfg) */
-    MOE_ERR_BAD_INDEX = 5,    /* device: an expert id outside [0, E) in topk_idx */
+    MOE_ERR_BAD_INDEX = 5,    /* device: an expert id outside [0, E) in topk_idx, a row id
+                                 outside the rows in sorted, or a group range in offsets
+                                 that is not 0 = offsets[0] <= o_g <= o_g+1 <= rows */
     MOE_ERR_TIMEOUT = 6,      /* device: a pipeline wait exceeded its time limit */
     MOE_ERR_CUDA = 7,         /* a CUDA runtime or driver call failed */
     MOE_ERR_RANGE = 8         /* device: an fp16 intermediate (h or a slot output) exceeded
@@ -71,9 +73,9 @@ typedef struct {
 
 /* Expert weights after moe_pack_weights (device, bf16):
  *   w13: [(E+1) * 2I][H]  per group g (g = E is the shared expert), rows in
- *        blocks of 256: block j holds rows 128j..128j+127 of W1_g (gate
- *        projection) followed by rows 128j..128j+127 of W3_g (up projection);
- *        the gate-then-up order is the fused gate_up_proj order of the nnterp
+ *        units of 32: unit j holds rows 16j..16j+15 of W1_g (gate projection)
+ *        followed by rows 16j..16j+15 of W3_g (up projection); the
+ *        gate-then-up order is the fused gate_up_proj order of the nnterp
  *        GLM-4 page (section 03, "The MLP is GLM's fused one").
  *   w2:  [(E+1) * H][I]  W2_g (down projection) for g = 0..E, shared last,
  *        stored as IEEE fp16 (see moe_pack_weights). */
@@ -86,6 +88,21 @@ typedef struct {
  * `cfg` (one buffer serves all three).  Returns 0 for an invalid cfg. */
 size_t moe_workspace_size(const moe_cfg_t *cfg);
 
+/* Staging buffers inside a workspace, for moe_workspace_offset. */
+typedef enum {
+    MOE_WS_TOKEN_ROWS = 0,   /* bf16 [T*K + T*has_shared][H]: token rows in expert-sorted
+                                order (moe_gather_tokens writes, moe_expert_up reads) */
+    MOE_WS_SLOT_OUTPUTS = 1  /* fp16 [T*K + T*has_shared][H]: weighted per-slot outputs,
+                                row t*K + slot, shared rows T*K + t (moe_expert_down
+                                writes, moe_combine reads) */
+} moe_ws_region_t;
+
+/* Byte offset of a staging buffer in a workspace laid out for cfg (16-byte
+ * aligned when the workspace is); (size_t)-1 for an invalid cfg or region.
+ * Lets a caller fill or read those buffers directly (the expert-parallel
+ * calls of srm_ep.h do). */
+size_t moe_workspace_offset(const moe_cfg_t *cfg, int32_t region);
+
 /* Pack per-expert weights into the moe_weights_t layout.
  *   w1, w3: bf16 [E][I][H];  w2: bf16 [E][H][I];
  *   ws1, ws3: bf16 [I][H];  ws2: bf16 [H][I] (shared expert; ignored and may
@@ -95,10 +112,15 @@ size_t moe_workspace_size(const moe_cfg_t *cfg);
  * magnitudes in [2^-17, 65504] (smaller ones keep fp16's subnormal spacing of
  * 2^-24, larger ones saturate).  The down projection multiplies fp16 h by
  * fp16 W2: fp16 holds h with three more mantissa bits than bf16 at the same
- * tensor-core rate.  cfg->T is not used. */
+ * tensor-core rate.
+ *   w2_inexact: int32 [1] device counter or NULL; out: the number of W2
+ *   values (routed and shared) whose fp16 copy differs from the bf16 value
+ *   (beyond +-65504, saturated; or too small for fp16's 2^-24 spacing,
+ *   rounded).  0 means the packed W2 is exact.  The call zeroes it first.
+ * cfg->T is not used. */
 moe_status_t moe_pack_weights(const moe_cfg_t *cfg, const void *w1, const void *w3, const void *w2,
                               const void *ws1, const void *ws3, const void *ws2, void *w13_out,
-                              void *w2_out, void *stream);
+                              void *w2_out, int32_t *w2_inexact, void *stream);
 
 /* Router ("Mixture of experts" equations z = x W_r, s = sigmoid(z),
  * E_sel = top_K(s + b), G = scale * s E_sel / sum s E_sel).
@@ -113,12 +135,37 @@ moe_status_t moe_pack_weights(const moe_cfg_t *cfg, const void *w1, const void *
  *   logits:    fp32 [T][E] or NULL; out: z, the router logits before the
  *              sigmoid and the bias (the pages' router_logits value).
  *   ws, ws_bytes: workspace of at least moe_workspace_size(cfg) bytes (holds
- *              the bf16 split of W_r and the partial logits).
+ *              the bf16 split of W_r and, for small T, the partial logits).
  * z is computed on the tensor cores from an exact three-part bf16 split of
- * W_r (each product exact, fp32 accumulation): fp32-accurate logits. */
+ * W_r (each product exact, fp32 accumulation): fp32-accurate logits.  This
+ * call makes the split into the workspace every time (one small extra
+ * kernel); moe_pack_router + moe_route_packed make it once. */
 moe_status_t moe_route(const moe_cfg_t *cfg, const void *x, const float *w_router, const float *bias,
                        int32_t *topk_idx, float *topk_gate, float *margin, float *logits, void *ws,
                        size_t ws_bytes, void *stream);
+
+/* Bytes of the packed router weights for cfg (2 * 3 * E_pad * H, E_pad = E
+ * rounded up to 64).  0 for an invalid cfg. */
+size_t moe_router_packed_size(const moe_cfg_t *cfg);
+
+/* The exact three-part bf16 split of the router weights, made once:
+ *   w_router_packed: [3][E_pad][H] bf16, part p row e = the p-th bf16 term of
+ *   W_r[e] (hi = bf16(W), mid = bf16(W - hi), lo = bf16(W - hi - mid); the
+ *   remainder is below 2^-24 |W|), rows E..E_pad-1 zero.  16-byte aligned,
+ *   moe_router_packed_size(cfg) bytes.  cfg->T is not used. */
+moe_status_t moe_pack_router(const moe_cfg_t *cfg, const float *w_router, void *w_router_packed,
+                             void *stream);
+
+/* moe_route with pre-packed router weights: logits, scores, biased top-K,
+ * margin and gates in ONE kernel (for large T one CTA per 128 tokens selects
+ * from the logits it holds, which reach global memory only if `logits` is
+ * given; for small T the H range is split over several CTAs that meet at a
+ * grid barrier bounded in time, MOE_ERR_TIMEOUT if it runs out, and sum their
+ * partials in a fixed order).  Arguments as moe_route, with w_router_packed
+ * from moe_pack_router in place of w_router.  Deterministic. */
+moe_status_t moe_route_packed(const moe_cfg_t *cfg, const void *x, const void *w_router_packed,
+                              const float *bias, int32_t *topk_idx, float *topk_gate, float *margin,
+                              float *logits, void *ws, size_t ws_bytes, void *stream);
 
 /* Expert-sorted permutation of the T*K assignments (deterministic).
  *   topk_idx: int32 [T][K] (as written by moe_route, or by the caller)
@@ -149,6 +196,16 @@ moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *weights, con
  * caller can time or overlap them.  They communicate through the workspace
  * (token rows in expert-sorted order, the intermediate h and the per-slot
  * outputs), so the same ws, cfg, offsets and sorted must be used for all four.
+ * offsets and sorted are checked on the device as they are read: a group whose
+ * range is malformed (first offset not 0, an end before its start or past the
+ * T*K + T*has_shared rows) is skipped and a row id outside the rows is ignored,
+ * both flagged MOE_ERR_BAD_INDEX; nothing outside the buffers is accessed.
+ *
+ * Test-only switch: with the environment variable SRM_MOE_INJECT_STALL=1 at
+ * the time of the call, moe_expert_up (and dsa_scores) issue no operand loads,
+ * so their bounded pipeline waits run out and the call reports MOE_ERR_TIMEOUT
+ * through the error word.  It exists for failure-detection tests; leave it
+ * unset in production.
  *
  * moe_gather_tokens: copies the token rows of x into expert-sorted order in
  *   the workspace (row p = x of the token of sorted[p]; each row of x is read
@@ -191,8 +248,10 @@ moe_status_t moe_combine(const moe_cfg_t *cfg, void *y, void *ws, size_t ws_byte
  *   Memory: every GPU that loads the library holds the array (about 256 KB)
  *   until the process exits.
  *   Set-up: the first call on each device looks up the array's device address
- *   (with that device current); make that first call before any stream
- *   capture.
+ *   (with that device current) and keeps it until the process exits; make that
+ *   first call before any stream capture.  Resetting the device
+ *   (cudaDeviceReset) after that is not supported.  Device ordinals 0-63 are
+ *   supported (MOE_ERR_UNSUPPORTED otherwise).
  *   Sharing: all calls use the same array and it keeps the last call's
  *   contents (each call clears its error word first); calls that overlap on
  *   the GPU (unordered streams) race on it.

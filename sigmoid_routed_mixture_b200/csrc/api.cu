@@ -10,6 +10,7 @@
 
 #include <mutex>
 
+#include "../../include/srm_ep.h"
 #include "../../include/srm_moe.h"
 #include "host_util.h"
 #include "kernels.h"
@@ -84,6 +85,14 @@ size_t moe_workspace_size(const moe_cfg_t *cfg) {
   return layout(*cfg).total;
 }
 
+size_t moe_workspace_offset(const moe_cfg_t *cfg, int32_t region) {
+  if (check_cfg(cfg, true) != MOE_OK) return static_cast<size_t>(-1);
+  const WsLayout L = layout(*cfg);
+  if (region == MOE_WS_TOKEN_ROWS) return L.xs;
+  if (region == MOE_WS_SLOT_OUTPUTS) return L.ybuf;
+  return static_cast<size_t>(-1);
+}
+
 const char *moe_status_string(moe_status_t s) {
   switch (s) {
     case MOE_OK: return "ok";
@@ -101,48 +110,103 @@ const char *moe_status_string(moe_status_t s) {
 
 moe_status_t moe_pack_weights(const moe_cfg_t *cfg, const void *w1, const void *w3, const void *w2,
                               const void *ws1, const void *ws3, const void *ws2, void *w13_out,
-                              void *w2_out, void *stream) {
+                              void *w2_out, int32_t *w2_inexact, void *stream) {
   moe_status_t st = check_cfg(cfg, true);
   if (st != MOE_OK) return st;
   if (!w13_out || !w2_out || (cfg->E > 0 && (!w1 || !w3 || !w2))) return MOE_ERR_ARG;
+  if (w2_inexact && !aligned(w2_inexact, 4)) return MOE_ERR_ALIGN;
   if (cfg->has_shared && (!ws1 || !ws3 || !ws2)) return MOE_ERR_ARG;
   const void *ptrs[] = {w1, w3, w2, w13_out, w2_out};
   for (const void *p : ptrs)
     if (p && !aligned(p, 16)) return MOE_ERR_ALIGN;
   if (cfg->has_shared && (!aligned(ws1, 16) || !aligned(ws3, 16) || !aligned(ws2, 16)))
     return MOE_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (w2_inexact && cudaMemsetAsync(w2_inexact, 0, sizeof(int32_t), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return cuda_status(srm::launch_pack(
       static_cast<const uint16_t *>(w1), static_cast<const uint16_t *>(w3),
       static_cast<const uint16_t *>(w2), static_cast<const uint16_t *>(ws1),
       static_cast<const uint16_t *>(ws3), static_cast<const uint16_t *>(ws2), cfg->H, cfg->I,
       cfg->E, cfg->has_shared, static_cast<uint16_t *>(w13_out), static_cast<uint16_t *>(w2_out),
-      num_sms(), static_cast<cudaStream_t>(stream)));
+      w2_inexact, num_sms(), s));
+}
+
+size_t moe_router_packed_size(const moe_cfg_t *cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return 2ull * 3 * static_cast<size_t>(srm::router_e_pad(cfg->E)) * cfg->H;
+}
+
+moe_status_t moe_pack_router(const moe_cfg_t *cfg, const float *w_router, void *w_router_packed,
+                             void *stream) {
+  moe_status_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!w_router || !w_router_packed) return MOE_ERR_ARG;
+  if (!aligned(w_router, 16) || !aligned(w_router_packed, 16)) return MOE_ERR_ALIGN;
+  return cuda_status(srm::launch_router_split(w_router, cfg->E, cfg->H,
+                                              static_cast<uint16_t *>(w_router_packed), num_sms(),
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Host validation shared by moe_route and moe_route_packed (w = the fp32 or
+// the packed router weights); everything is checked before the first launch.
+moe_status_t check_route_args(const moe_cfg_t *cfg, const void *x, const void *w, const float *bias,
+                              const int32_t *topk_idx, const float *topk_gate, const float *margin,
+                              const float *logits, const void *ws, size_t ws_bytes) {
+  moe_status_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !w || !bias || !topk_idx || !topk_gate || !ws) return MOE_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(w, 16) || !aligned(bias, 4) || !aligned(topk_idx, 4) ||
+      !aligned(topk_gate, 4) || (margin && !aligned(margin, 4)) || (logits && !aligned(logits, 4)) ||
+      !aligned(ws, 256))
+    return MOE_ERR_ALIGN;
+  if (ws_bytes < layout(*cfg).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_route_packed(const moe_cfg_t *cfg, const void *x, const void *w_router_packed,
+                              const float *bias, int32_t *topk_idx, float *topk_gate, float *margin,
+                              float *logits, void *ws, size_t ws_bytes, void *stream) {
+  moe_status_t st = check_route_args(cfg, x, w_router_packed, bias, topk_idx, topk_gate, margin, logits,
+                                     ws, ws_bytes);
+  if (st != MOE_OK || cfg->T == 0) return st;
+  const WsLayout L = layout(*cfg);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int e_pad = srm::router_e_pad(cfg->E);
+  CUtensorMap tm_x, tm_w;
+  if (!make_tmap(&tm_x, x, cfg->H, static_cast<uint64_t>(cfg->T), 64, 128) ||
+      !make_tmap(&tm_w, w_router_packed, cfg->H, 3ull * e_pad, 64, static_cast<uint32_t>(e_pad)))
+    return MOE_ERR_CUDA;
+  int *grid_counter = reinterpret_cast<int *>(wsb + L.err + 64);
+  if (cudaMemsetAsync(grid_counter, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(srm::launch_route(
+      tm_x, tm_w, bias, static_cast<int>(cfg->T), cfg->H, cfg->E, cfg->K, cfg->routed_scale,
+      reinterpret_cast<float *>(wsb + L.zp), grid_counter, topk_idx, topk_gate, margin, logits,
+      reinterpret_cast<int *>(wsb + L.err), num_sms(), s));
 }
 
 moe_status_t moe_route(const moe_cfg_t *cfg, const void *x, const float *w_router, const float *bias,
                        int32_t *topk_idx, float *topk_gate, float *margin, float *logits, void *ws,
                        size_t ws_bytes, void *stream) {
-  moe_status_t st = check_cfg(cfg);
-  if (st != MOE_OK) return st;
-  if (cfg->T == 0) return MOE_OK;
-  if (!x || !w_router || !bias || !topk_idx || !topk_gate || !ws) return MOE_ERR_ARG;
-  if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(bias, 4) || !aligned(topk_idx, 4) ||
-      !aligned(topk_gate, 4) || (margin && !aligned(margin, 4)) || (logits && !aligned(logits, 4)) ||
-      !aligned(ws, 256))
-    return MOE_ERR_ALIGN;
+  moe_status_t st = check_route_args(cfg, x, w_router, bias, topk_idx, topk_gate, margin, logits, ws,
+                                     ws_bytes);
+  if (st != MOE_OK || cfg->T == 0) return st;
   const WsLayout L = layout(*cfg);
-  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  uint8_t *wsb = static_cast<uint8_t *>(ws);
-  const int e_pad = srm::router_e_pad(cfg->E);
-  CUtensorMap tm_x, tm_w;
-  if (!make_tmap(&tm_x, x, cfg->H, static_cast<uint64_t>(cfg->T), 64, 128) ||
-      !make_tmap(&tm_w, wsb + L.wsplit, cfg->H, 3ull * e_pad, 64, static_cast<uint32_t>(e_pad)))
-    return MOE_ERR_CUDA;
-  return cuda_status(srm::launch_route(
-      tm_x, tm_w, w_router, bias, static_cast<int>(cfg->T), cfg->H, cfg->E, cfg->K,
-      cfg->routed_scale, reinterpret_cast<uint16_t *>(wsb + L.wsplit),
-      reinterpret_cast<float *>(wsb + L.zp), topk_idx, topk_gate, margin, logits,
-      reinterpret_cast<int *>(wsb + L.err), num_sms(), static_cast<cudaStream_t>(stream)));
+  void *wsplit = static_cast<uint8_t *>(ws) + L.wsplit;
+  st = moe_pack_router(cfg, w_router, wsplit, stream);
+  if (st != MOE_OK) return st;
+  return moe_route_packed(cfg, x, wsplit, bias, topk_idx, topk_gate, margin, logits, ws, ws_bytes,
+                          stream);
 }
 
 moe_status_t moe_permute(const moe_cfg_t *cfg, const int32_t *topk_idx, int32_t *counts,
@@ -232,9 +296,10 @@ moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool pair = srm::gemm_use_pairs(cfg->T, cfg->K, cfg->E);
   CUtensorMap tm_x, tm_w13;
-  if (!make_tmap(&tm_x, wsb + L.xs, H, static_cast<uint64_t>(rows_y(*cfg)), 64, 128) ||
+  if (!make_tmap(&tm_x, wsb + L.xs, H, static_cast<uint64_t>(rows_y(*cfg)), 64,
+                 static_cast<uint32_t>(srm::gemm_tok_box_rows())) ||
       !make_tmap(&tm_w13, weights->w13, H, static_cast<uint64_t>(E + 1) * 2 * I, 64,
-                 static_cast<uint32_t>(srm::gemm_b_box_rows(pair))))
+                 static_cast<uint32_t>(srm::gemm_w_box_rows())))
     return MOE_ERR_CUDA;
   GemmArgs p = gemm_args(*cfg, offsets, sorted, nullptr, wsb, L);
   // Failure-detection tests set SRM_MOE_INJECT_STALL=1: the up projection's
@@ -265,10 +330,11 @@ moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
   const int H = cfg->H, I = cfg->I, E = cfg->E;
   const bool pair = srm::gemm_use_pairs(cfg->T, cfg->K, cfg->E);
   CUtensorMap tm_h, tm_w2;
-  if (!make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(rows_y(*cfg)), 64, 128,
+  if (!make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(rows_y(*cfg)), 64,
+                 static_cast<uint32_t>(srm::gemm_tok_box_rows()),
                  CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
       !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(E + 1) * H, 64,
-                 static_cast<uint32_t>(srm::gemm_b_box_rows(pair)), CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+                 static_cast<uint32_t>(srm::gemm_w_box_rows()), CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_CUDA;
   GemmArgs p = gemm_args(*cfg, offsets, sorted, topk_gate, wsb, L);
   p.out = wsb + L.ybuf;
@@ -357,13 +423,15 @@ moe_status_t moe_dense_mlp(const moe_cfg_t *cfg, const moe_weights_t *weights, c
     return MOE_ERR_CUDA;
   const bool pair = cfg->T >= 512;
   CUtensorMap tm_x, tm_w13, tm_h, tm_w2;
-  if (!make_tmap(&tm_x, x, H, static_cast<uint64_t>(T), 64, 128) ||
+  if (!make_tmap(&tm_x, x, H, static_cast<uint64_t>(T), 64,
+                 static_cast<uint32_t>(srm::gemm_tok_box_rows())) ||
       !make_tmap(&tm_w13, weights->w13, H, 2ull * I, 64,
-                 static_cast<uint32_t>(srm::gemm_b_box_rows(pair))) ||
-      !make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(T), 64, 128,
+                 static_cast<uint32_t>(srm::gemm_w_box_rows())) ||
+      !make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(T), 64,
+                 static_cast<uint32_t>(srm::gemm_tok_box_rows()),
                  CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
       !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(H), 64,
-                 static_cast<uint32_t>(srm::gemm_b_box_rows(pair)), CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+                 static_cast<uint32_t>(srm::gemm_w_box_rows()), CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_CUDA;
   GemmArgs p = gemm_args(*cfg, offsets, sorted, nullptr, wsb, L);
   p.out = wsb + L.h;
@@ -383,6 +451,58 @@ moe_status_t moe_dense_mlp(const moe_cfg_t *cfg, const moe_weights_t *weights, c
   return cuda_status(srm::launch_combine(reinterpret_cast<const uint16_t *>(wsb + L.ybuf),
                                          static_cast<const uint16_t *>(residual),
                                          static_cast<uint16_t *>(y), T, H, 0, 1, num_sms(), s));
+}
+
+moe_status_t moe_ep_shared(const moe_cfg_t *cfg, const moe_weights_t *shared, const void *x, void *ws,
+                           size_t ws_bytes, void *stream) {
+  moe_status_t st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->has_shared != 1) return MOE_ERR_ARG;
+  if (cfg->T == 0) return MOE_OK;
+  if (!shared || !shared->w13 || !shared->w2 || !x || !ws) return MOE_ERR_ARG;
+  if (!aligned(shared->w13, 16) || !aligned(shared->w2, 16) || !aligned(x, 16) || !aligned(ws, 256))
+    return MOE_ERR_ALIGN;
+  const WsLayout L = layout(*cfg);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  const int T = static_cast<int>(cfg->T), H = cfg->H, I = cfg->I;
+  // one group (the shared expert) holding every token in order; its rows are
+  // the shared row ids T*K + t, so the down projection writes them where the
+  // single-GPU path does (gate 1, past the routed rows)
+  int32_t *offsets = reinterpret_cast<int32_t *>(wsb + L.err + 192);
+  int32_t *sorted = reinterpret_cast<int32_t *>(wsb + L.pos);
+  if (srm::launch_identity_rows(offsets, sorted, T, num_sms(), s, T * cfg->K) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  // the tile shape the single-GPU path would use for this block
+  const bool pair = srm::gemm_use_pairs(cfg->T, cfg->K, cfg->E);
+  CUtensorMap tm_x, tm_w13, tm_h, tm_w2;
+  if (!make_tmap(&tm_x, x, H, static_cast<uint64_t>(T), 64,
+                 static_cast<uint32_t>(srm::gemm_tok_box_rows())) ||
+      !make_tmap(&tm_w13, shared->w13, H, 2ull * I, 64,
+                 static_cast<uint32_t>(srm::gemm_w_box_rows())) ||
+      !make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(T), 64,
+                 static_cast<uint32_t>(srm::gemm_tok_box_rows()),
+                 CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_tmap(&tm_w2, shared->w2, I, static_cast<uint64_t>(H), 64,
+                 static_cast<uint32_t>(srm::gemm_w_box_rows()), CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    return MOE_ERR_CUDA;
+  GemmArgs p = gemm_args(*cfg, offsets, sorted, nullptr, wsb, L);
+  p.groups = 1;
+  p.out = wsb + L.h;
+  p.n_total = 2 * I;
+  p.k_total = H;
+  p.out_ld = I;
+  if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s) != cudaSuccess ||
+      srm::launch_grouped_gemm(srm::kUp, pair, tm_x, tm_w13, p, num_sms(), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  p.out = wsb + L.ybuf;
+  p.n_total = H;
+  p.k_total = I;
+  p.out_ld = H;
+  if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cuda_status(srm::launch_grouped_gemm(srm::kDown, pair, tm_h, tm_w2, p, num_sms(), s));
 }
 
 moe_status_t moe_get_device_error(void *ws, moe_status_t *device_status, void *stream) {

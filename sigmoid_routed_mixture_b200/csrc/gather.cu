@@ -75,21 +75,21 @@ __global__ void __launch_bounds__(256)
 }
 
 __global__ void identity_rows_kernel(int32_t *__restrict__ offsets, int32_t *__restrict__ sorted,
-                                     int T) {
+                                     int T, int base) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i == 0) {
     offsets[0] = 0;
     offsets[1] = T;
   }
-  for (int t = i; t < T; t += gridDim.x * blockDim.x) sorted[t] = t;
+  for (int t = i; t < T; t += gridDim.x * blockDim.x) sorted[t] = base + t;
 }
 
 cudaError_t launch_identity_rows(int32_t *offsets, int32_t *sorted, int T, int num_sms,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, int base) {
   int blocks = (T + 255) / 256;
   if (blocks > num_sms * 4) blocks = num_sms * 4;
   if (blocks < 1) blocks = 1;
-  identity_rows_kernel<<<blocks, 256, 0, stream>>>(offsets, sorted, T);
+  identity_rows_kernel<<<blocks, 256, 0, stream>>>(offsets, sorted, T, base);
   return cudaGetLastError();
 }
 

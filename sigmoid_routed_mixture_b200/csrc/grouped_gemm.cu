@@ -1,7 +1,7 @@
 // grouped_gemm.cu -- the two expert contractions of the mixture on the
 // 5th-generation tensor cores (tcgen05.mma, accumulators in tensor memory),
 // fed by TMA, as one persistent, warp-specialised kernel template that runs
-// on CTA pairs.
+// on CTA pairs (or single CTAs for small batches).
 //
 // Definition ("GLM-5 . MoE transformer block", "All 43 steps", Mixture of
 // experts): per expert i and token row x,
@@ -10,35 +10,45 @@
 // weighted by G_i ("expert_outputs: each routing slot's weighted expert
 // output", nnterp GLM-5 page, The API table).
 //
-//   kUp   : for every group g (routed experts 0..E-1, shared expert E) and its
-//           rows, [g | u] = xs_rows . W13_g^T where xs holds the token rows in
-//           expert-sorted order (gather.cu); epilogue h = silu(g) * u -> fp16
-//           h[row][I] (three more mantissa bits than bf16 at the same
-//           tensor-core rate; |h| saturates at 65504, flagged MOE_ERR_RANGE).
-//   kDown : Y[a] = G[a] * (h_rows . W2_g^T) in fp16 x fp16 (W2 packed as
-//           fp16, an exact conversion of bf16 weights in fp16's normal
-//           range), rows of h contiguous, epilogue multiplies by the routing
-//           gate (1 for the shared expert) and scatters fp16 rows to their
-//           (token, slot) position a (fp16: 8x finer rounding than bf16 in
-//           the same two bytes; saturation at 65504 is flagged MOE_ERR_RANGE).
+// Operand roles: the WEIGHTS are the MMA's M side and the TOKENS its N side,
+// D^T[weight row][token] = W_g[weight rows] . X[tokens]^T.  M is fixed (256
+// weight rows per CTA pair, 128 per single CTA), and N, the tile's token
+// count, can be any multiple of 16 up to 256: a group whose row count is not a
+// multiple of 256 pads its last tile to 16 rows, not to 256 (with tokens on
+// the M side, 16.8% of the rows of the 16384-token GLM-5 block were padding).
 //
-// Tiling: a cluster of two CTAs (a CTA pair) owns one work tile of 256 rows x
-// 256 output columns: each CTA loads its 128 rows of A and 128 of the 256
-// rows of B (so every B byte crosses L2 once per pair, not once per CTA), and
-// the leader CTA issues tcgen05.mma.cta_group::2 with M = 256 that reads both
-// CTAs' shared memory and leaves each CTA's 128 x 256 fp32 accumulator in its
-// own tensor memory.  K loop in steps of 64 (one 128-byte swizzle atom), a
-// 6-stage TMA ring per CTA, two accumulators per CTA (512 TMEM columns) so the
-// epilogue of one tile overlaps the main loop of the next.
+//   kUp   : for every group g (routed experts 0..E-1, shared expert E), the
+//           packed W13_g rows against its token rows (xs: token rows in
+//           expert-sorted order, gather.cu).  W13 is packed in units of 32
+//           rows, 16 gate rows then the 16 matching up rows, so TMEM lanes
+//           l and l + 16 of a warp hold gate and up of one feature: one
+//           shuffle pairs them, epilogue h = silu(g) * u -> fp16 h[row][I]
+//           (three more mantissa bits than bf16 at the same tensor-core rate;
+//           |h| saturates at 65504, flagged MOE_ERR_RANGE).
+//   kDown : W2_g rows (output features, fp16; an exact conversion of bf16
+//           weights in fp16's normal range) against the token rows of h
+//           (fp16); epilogue multiplies by the routing gate (1 for the shared
+//           expert) and stores fp16 to the row's (token, slot) position
+//           (saturation at 65504 flagged MOE_ERR_RANGE).
+//
+// Tiling: a work tile is (group, weight block of 256 rows, token block of up
+// to 256 rows).  On a CTA pair each CTA loads 128 of the weight rows and half
+// of the tile's token rows (N/2, in TMA boxes of 32 rows), the leader issues
+// tcgen05.mma.cta_group::2 with M = 256 and N = the tile's token count
+// rounded up to 16, and each CTA receives its 128 weight rows x N tokens in
+// its own tensor memory.  K loop in steps of 64 (one 128-byte swizzle atom), a
+// 6-stage TMA ring per CTA (4 for single CTAs), two accumulators of 256
+// columns so the epilogue of one tile overlaps the main loop of the next.
 // Warp roles (6 warps per CTA):
-//   warp 0: TMA producer (one lane issues the CTA's A and B tile loads)
+//   warp 0: TMA producer (one lane issues the CTA's weight and token loads)
 //   warp 1: tensor-memory allocation; in the leader also single-thread MMA issue
 //   warps 2-5: epilogue (tensor memory -> registers -> global)
-// Work tiles are (group, 256-column block, row block), row block fastest; a
-// unit (CTA pair or single CTA) takes its next tile from a global atomic
-// counter when it is ready for one, so tiles that share a weight tile start
-// together; the per-group row-block counts come from the group offsets on the
-// device, so the host never synchronises.
+// Work tiles are ordered (group, weight block, token block), token block
+// fastest; a unit (CTA pair or single CTA) takes its next tile from a global
+// atomic counter when it is ready for one, so the tiles that share a weight
+// block start together and read it from DRAM once; the per-group token-block
+// counts come from the group offsets on the device, so the host never
+// synchronises.
 //
 // Barrier protocol of a pair (no TMA multicast anywhere):
 //   full[s]   (leader's)  producer of the leader arms it with both CTAs' bytes;
@@ -60,26 +70,26 @@
 namespace srm {
 
 namespace gg {
-constexpr int BM = 128;        // rows per CTA
-constexpr int BN = 256;        // output columns per tile
+constexpr int BM = 128;        // weight rows per CTA (tensor-memory lanes)
+constexpr int BT = 256;        // tokens per tile (largest MMA N)
 constexpr int BK = 64;
+constexpr int TOK_BOX = 32;    // token rows per TMA box
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
+constexpr uint32_t TMEM_COLS = 2 * BT;  // two accumulators
 constexpr int MAX_GROUPS = 257;
 constexpr int MAX_STAGES = 6;
 constexpr int TILE_RING = 4;  // tile ids in flight between the scheduler and the roles
 
-// kPair: a CTA pair shares each 256-row tile (M = 256, each CTA loads half of
-// B); solo: one CTA per 128-row tile (M = 128, the CTA loads all of B).
+// kPair: a CTA pair shares each tile (M = 256 weight rows, each CTA loads 128
+// of them and half of the tokens); solo: one CTA per tile (M = 128, all tokens).
 template <bool kPair>
 struct Cfg {
-  static constexpr int TILE_M = kPair ? 2 * BM : BM;
-  static constexpr int B_ROWS = kPair ? BN / 2 : BN;     // B rows loaded per CTA
+  static constexpr int W_BLOCK = kPair ? 2 * BM : BM;   // weight rows per tile (MMA M)
+  static constexpr int TOK_ROWS = kPair ? BT / 2 : BT;  // token rows one CTA holds at most
   static constexpr int STAGES = kPair ? 6 : 4;
-  static constexpr int A_BYTES = BM * BK * 2;            // 16 KB
-  static constexpr int B_BYTES = B_ROWS * BK * 2;        // 16 or 32 KB
+  static constexpr int A_BYTES = BM * BK * 2;           // 16 KB of weights
+  static constexpr int B_BYTES = TOK_ROWS * BK * 2;     // 16 or 32 KB of token rows at most
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t TX_BYTES = (kPair ? 2 : 1) * STAGE_BYTES;
   static constexpr uint32_t EPI_ARRIVALS = kPair ? 8 : 4;
 };
 
@@ -107,23 +117,24 @@ constexpr size_t smem_bytes() {
 
 struct TileCoord {
   int g;          // group
-  int row_base;   // first row of this CTA's half of the tile (expert-sorted order)
-  int rows;       // valid rows of this CTA's half (0..128)
-  int n0;         // first output column
+  int row_base;   // first token row of the tile (expert-sorted order)
+  int rows;       // valid token rows (1..256)
+  int n;          // MMA N: rows rounded up to 16
+  int w0;         // first weight row of the tile within the group
 };
 
 // Tiles of group g occupy [tile_start[g] * n_tiles, tile_start[g+1] * n_tiles)
-// and inside a group the row block runs fastest: the units working at the same
-// moment share each 256-column weight tile (one DRAM read serves all the
-// group's row blocks) instead of spreading over many weight tiles that evict
-// one another from L2.  A group with more than m_chunk row blocks (the shared
-// expert at large batches) is walked in chunks of m_chunk row blocks, each
-// chunk through all column blocks, so that the chunk's rows stay in L2 while
-// every column block reads them (a whole 16384-token group would not fit and
-// would be re-read from DRAM once per column block).
+// and inside a group the token block runs fastest: the units working at the
+// same moment share each 256-row weight block (one DRAM read serves all the
+// group's token blocks) instead of spreading over many weight blocks that
+// evict one another from L2.  A group with more than m_chunk token blocks (the
+// shared expert at large batches) is walked in chunks of m_chunk token blocks,
+// each chunk through all weight blocks, so that the chunk's token rows stay in
+// L2 while every weight block reads them (a whole 16384-token group would not
+// fit and would be re-read from DRAM once per weight block).
 template <bool kPair>
 __device__ __forceinline__ TileCoord decode_tile(const gg::Smem &s, int groups, int n_tiles,
-                                                 int m_chunk, int tile, int rank) {
+                                                 int m_chunk, int tile) {
   const int mt_flat = tile / n_tiles;
   int lo = 0, hi = groups - 1;  // last g with tile_start[g] <= mt_flat
   while (lo < hi) {
@@ -137,32 +148,39 @@ __device__ __forceinline__ TileCoord decode_tile(const gg::Smem &s, int groups, 
   const int local = tile - s.tile_start[lo] * n_tiles;
   const int chunk = local / (m_chunk * n_tiles);
   const int m0 = chunk * m_chunk;
-  const int cm = min(m_chunk, mblocks - m0);  // row blocks in this chunk
+  const int cm = min(m_chunk, mblocks - m0);  // token blocks in this chunk
   const int r = local - m0 * n_tiles;
   const int nt = r / cm;
   const int mt = m0 + (r - nt * cm);
   TileCoord c;
   c.g = lo;
-  c.row_base = s.grp_off[lo] + mt * gg::Cfg<kPair>::TILE_M + rank * gg::BM;
-  c.rows = max(0, min(gg::BM, s.grp_off[lo + 1] - c.row_base));
-  c.n0 = nt * gg::BN;
+  c.row_base = s.grp_off[lo] + mt * gg::BT;
+  c.rows = max(0, min(gg::BT, s.grp_off[lo + 1] - c.row_base));
+  c.n = max(16, (c.rows + 15) & ~15);
+  c.w0 = nt * gg::Cfg<kPair>::W_BLOCK;
   return c;
 }
 
+// fp32 -> fp16 bits (round to nearest even), saturating at +-65504 (sets sat)
+__device__ __forceinline__ uint16_t f16_sat(float v, bool &sat) {
+  sat |= !(fabsf(v) <= 65504.f);
+  return __half_as_ushort(__float2half_rn(fminf(fmaxf(v, -65504.f), 65504.f)));
+}
+
 template <int kMode, bool kPair>
-__device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b,
+__device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, const CUtensorMap &tmap_w,
                                                   const GemmArgs &p) {
   using namespace gg;
   using C = Cfg<kPair>;
   constexpr int STAGES = C::STAGES;
   constexpr int A_BYTES = C::A_BYTES;
   constexpr int B_BYTES = C::B_BYTES;
-  constexpr int TILE_M = C::TILE_M;
+  constexpr int TOK_BOX_BYTES = TOK_BOX * BK * 2;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   uint8_t *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t *sA = base;
-  uint8_t *sB = base + STAGES * A_BYTES;
+  uint8_t *sA = base;                   // weights
+  uint8_t *sB = base + STAGES * A_BYTES;  // token rows
   Smem &s = *reinterpret_cast<Smem *>(base + STAGES * C::STAGE_BYTES);
 
   const int warp = threadIdx.x >> 5;
@@ -170,12 +188,12 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
   const uint32_t rank = kPair ? cluster_ctarank() : 0;
   const bool leader = rank == 0;
   const int groups = p.groups;
-  const int n_tiles = p.n_total / BN;
+  const int n_tiles = p.n_total / C::W_BLOCK;
   const int kblocks = p.k_total / BK;
-  // row blocks per chunk: about 48 MB of A rows (16-bit operands)
-  const int m_chunk = max(1, (48 << 20) / (TILE_M * p.k_total * 2));
-  // up: bf16 x times bf16 W13; down: fp16 h times fp16 W2
-  constexpr uint32_t IDESC = umma_idesc_f32acc(TILE_M, BN, kMode == kUp ? 1u : 0u);
+  // token blocks per chunk: about 48 MB of token rows (16-bit operands)
+  const int m_chunk = max(1, (48 << 20) / (BT * p.k_total * 2));
+  // up: bf16 W13 times bf16 x; down: fp16 W2 times fp16 h
+  constexpr uint32_t AB_BF16 = kMode == kUp ? 1u : 0u;
 
   // ---- prologue: barriers, tensor memory, per-group tile starts
   if (threadIdx.x == 0) {
@@ -195,8 +213,8 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
     s.abort_flag = 0;
     s.mma_consumed = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&tmap_a);
-    tma_prefetch_desc(&tmap_b);
+    tma_prefetch_desc(&tmap_tok);
+    tma_prefetch_desc(&tmap_w);
   }
   if (warp == 1) {
     if (kPair) {
@@ -208,14 +226,27 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
     }
   }
   if (warp == 0) {
-    // group offsets and an exclusive scan of ceil(count / TILE_M) over the groups
+    // group offsets and an exclusive scan of ceil(count / BT) over the
+    // groups.  Offsets come from the caller: a group whose range is not
+    // 0 <= o0 <= o1 <= n_rows_y (or a first offset other than 0, which is how
+    // the allocation-free permutation flags a bad id) gets no tiles and is
+    // flagged MOE_ERR_BAD_INDEX, so no row outside the buffers is touched.
+    // A group's end is the next group's raw start, so a valid group keeps its
+    // own bounds even when its neighbour is rejected.
+    auto token_blocks = [&](int g) {
+      const int o0 = p.offsets[g], o1 = p.offsets[g + 1];
+      if (o0 < 0 || o1 < o0 || o1 > p.n_rows_y || (g == 0 && o0 != 0)) {
+        record_error(p.err, MOE_ERR_BAD_INDEX);
+        return 0;
+      }
+      return (o1 - o0 + BT - 1) / BT;
+    };
     const int per = (groups + 31) / 32;
     const int g0 = lane * per;
     int local = 0;
     for (int g = g0; g < min(g0 + per, groups); ++g) {
-      const int o0 = p.offsets[g], o1 = p.offsets[g + 1];
-      s.grp_off[g] = o0;
-      local += (o1 - o0 + TILE_M - 1) / TILE_M;
+      s.grp_off[g] = p.offsets[g];
+      local += token_blocks(g);
     }
     int incl = local;
 #pragma unroll
@@ -226,7 +257,7 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
     int run = incl - local;
     for (int g = g0; g < min(g0 + per, groups); ++g) {
       s.tile_start[g] = run;
-      run += (p.offsets[g + 1] - p.offsets[g] + TILE_M - 1) / TILE_M;
+      run += token_blocks(g);
     }
     if (lane == 31) {
       s.total_mtiles = incl;
@@ -249,8 +280,8 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // The leader's producer is also the tile scheduler: it takes the next
-    // tile from the global counter, so tiles sharing a weight tile (one
-    // group's row blocks) start at nearly the same moment on whichever units
+    // tile from the global counter, so tiles sharing a weight block (one
+    // group's token blocks) start at nearly the same moment on whichever units
     // are free, and publishes the id to its own CTA and to the peer through
     // the tile ring.
     uint32_t stage = 0, phase = 0, ts = 0, tph = 0;
@@ -276,8 +307,12 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
         tph ^= 1u;
       }
       if (tile < 0 || p.stall) break;
-      const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, m_chunk, tile, rank);
-      const int b_row = c.g * p.n_total + c.n0 + rank * C::B_ROWS;
+      const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, m_chunk, tile);
+      const int w_row = c.g * p.n_total + c.w0 + rank * BM;   // this CTA's weight rows
+      const int tok_rows = kPair ? c.n / 2 : c.n;             // this CTA's token rows
+      const int tok_row0 = c.row_base + rank * tok_rows;
+      const int nb = (tok_rows + TOK_BOX - 1) / TOK_BOX;
+      const uint32_t tx = (kPair ? 2u : 1u) * static_cast<uint32_t>(A_BYTES + nb * TOK_BOX_BYTES);
       bool ok = true;
       for (int kb = 0; kb < kblocks; ++kb) {
         if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, p.err)) {
@@ -285,14 +320,19 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
           break;
         }
         if (lane == 0) {
-          if (leader) mbar_arrive_expect_tx(&s.full[stage], C::TX_BYTES);
+          if (leader) mbar_arrive_expect_tx(&s.full[stage], tx);
+          uint8_t *b_dst = sB + stage * B_BYTES;
           if (kPair) {
             const uint32_t full_leader = cluster_map(&s.full[stage], 0);
-            tma_load_2d_pair(sA + stage * A_BYTES, &tmap_a, full_leader, kb * BK, c.row_base);
-            tma_load_2d_pair(sB + stage * B_BYTES, &tmap_b, full_leader, kb * BK, b_row);
+            tma_load_2d_pair(sA + stage * A_BYTES, &tmap_w, full_leader, kb * BK, w_row);
+            for (int j = 0; j < nb; ++j)
+              tma_load_2d_pair(b_dst + j * TOK_BOX_BYTES, &tmap_tok, full_leader, kb * BK,
+                               tok_row0 + j * TOK_BOX);
           } else {
-            tma_load_2d(sA + stage * A_BYTES, &tmap_a, &s.full[stage], kb * BK, c.row_base);
-            tma_load_2d(sB + stage * B_BYTES, &tmap_b, &s.full[stage], kb * BK, b_row);
+            tma_load_2d(sA + stage * A_BYTES, &tmap_w, &s.full[stage], kb * BK, w_row);
+            for (int j = 0; j < nb; ++j)
+              tma_load_2d(b_dst + j * TOK_BOX_BYTES, &tmap_tok, &s.full[stage], kb * BK,
+                          tok_row0 + j * TOK_BOX);
           }
         }
         __syncwarp();
@@ -317,9 +357,11 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
           tph ^= 1u;
         }
         if (tile < 0) break;
+        const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, m_chunk, tile);
+        const uint32_t idesc = umma_idesc_f32acc(C::W_BLOCK, c.n, AB_BF16);
         if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag, p.err)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
+        const uint32_t d_tmem = tmem_base + acc * BT;
         bool ok = true;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&s.full[stage], phase, abort_flag, p.err)) {
@@ -335,10 +377,10 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
             for (int k = 0; k < BK / 16; ++k) {
               if (kPair)
                 umma_pair(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32),
-                          IDESC, (kb | k) != 0 ? 1u : 0u);
+                          idesc, (kb | k) != 0 ? 1u : 0u);
               else
                 umma_bf16(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32),
-                          IDESC, (kb | k) != 0 ? 1u : 0u);
+                          idesc, (kb | k) != 0 ? 1u : 0u);
             }
             if (kPair)
               umma_commit_pair(&s.empty[stage], 0x3);
@@ -366,8 +408,10 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // tensor-memory lane quarter this warp may access
-    const int row = q * 32 + lane;
+    // Warp q = warp % 4 may read tensor-memory lanes 32q .. 32q+31: this
+    // CTA's weight rows w0 + rank*128 + 32q + lane, one lane per weight row,
+    // the tile's tokens along the columns.
+    const int q = warp & 3;
     uint32_t acc = 0, acc_phase = 0, ts = 0, tph = 0;
     while (true) {
       if (!mbar_wait(&s.tile_full[ts], tph, abort_flag, p.err, kPair)) break;
@@ -378,60 +422,64 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
         tph ^= 1u;
       }
       if (tile < 0) break;
-      const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, m_chunk, tile, rank);
+      const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, m_chunk, tile);
+      const int wr = c.w0 + static_cast<int>(rank) * BM + q * 32;  // this warp's first weight row
       if (!mbar_wait(&s.tfull[acc], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
-      bool valid = row < c.rows;
-      int a = valid ? p.sorted[c.row_base + row] : 0;
-      if (valid && (a < 0 || a >= p.n_rows_y)) {
-        record_error(p.err, MOE_ERR_BAD_INDEX);
-        valid = false;
-      }
-      const uint32_t taddr = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t taddr = tmem_base + acc * BT + (static_cast<uint32_t>(q * 32) << 16);
       bool sat = false;
       if (kMode == kUp) {
-        // columns 0..127 of the tile are gate rows, 128..255 the matching up rows
-        uint16_t *hrow = reinterpret_cast<uint16_t *>(p.out) +
-                         static_cast<size_t>(c.row_base + row) * p.out_ld + c.n0 / 2;
+        // lanes 0-15 hold gate rows of features j0 .. j0+15, lanes 16-31 the
+        // matching up rows (the 32-row packing unit); after one exchange lane l
+        // has (g, u) of feature j0 + (l % 16) for tokens half*16 .. half*16+15
+        // of each 32-token chunk, half = l / 16
+        const int half = lane >> 4;
+        const int j = wr / 2 + (lane & 15);
+        __half *h = reinterpret_cast<__half *>(p.out);
 #pragma unroll 1
-        for (int ch = 0; ch < BN / 2 / 32; ++ch) {
-          uint32_t gr[32], ur[32];
-          tmem_ld32(taddr + ch * 32, gr);
-          tmem_ld32(taddr + BN / 2 + ch * 32, ur);
+        for (int c0 = 0; c0 < c.n; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c0, v);
           tmem_ld_wait();
-          if (valid) {
-            uint32_t packed[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float g0 = __uint_as_float(gr[2 * j]), g1 = __uint_as_float(gr[2 * j + 1]);
-              const float u0 = __uint_as_float(ur[2 * j]), u1 = __uint_as_float(ur[2 * j + 1]);
-              packed[j] = pack_f16x2_sat(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1, sat);
-            }
-            uint4 *dst = reinterpret_cast<uint4 *>(hrow + ch * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
-                                  packed[4 * v + 3]);
+          for (int k = 0; k < 16; ++k) {
+            const float mine = __uint_as_float(v[half ? k + 16 : k]);
+            const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(v[half ? k : k + 16]), 16);
+            const float g = half ? other : mine;
+            const float u = half ? mine : other;
+            const int t = c0 + half * 16 + k;
+            if (t < c.rows)
+              h[static_cast<size_t>(c.row_base + t) * p.out_ld + j] =
+                  __ushort_as_half(f16_sat(g * sigmoidf_(g) * u, sat));
           }
         }
       } else {
-        const float gv = (a < p.tk) ? p.gate[valid ? a : 0] : 1.0f;
-        uint16_t *yrow = reinterpret_cast<uint16_t *>(p.out) + static_cast<size_t>(a) * p.out_ld + c.n0;
+        // lane = output feature f; the tokens' destinations and gates are
+        // loaded one per lane per 32-token chunk and broadcast by shuffles
+        const int f = wr + lane;
+        __half *y = reinterpret_cast<__half *>(p.out);
 #pragma unroll 1
-        for (int ch = 0; ch < BN / 32; ++ch) {
-          uint32_t r[32];
-          tmem_ld32(taddr + ch * 32, r);
+        for (int c0 = 0; c0 < c.n; c0 += 32) {
+          int my_a = -1;
+          float my_g = 0.f;
+          if (c0 + lane < c.rows) {
+            const int a = p.sorted[c.row_base + c0 + lane];
+            if (a < 0 || a >= p.n_rows_y) {
+              record_error(p.err, MOE_ERR_BAD_INDEX);
+            } else {
+              my_a = a;
+              my_g = a < p.tk ? p.gate[a] : 1.0f;
+            }
+          }
+          uint32_t v[32];
+          tmem_ld32(taddr + c0, v);
           tmem_ld_wait();
-          if (valid) {
-            uint32_t packed[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              packed[j] = pack_f16x2_sat(gv * __uint_as_float(r[2 * j]), gv * __uint_as_float(r[2 * j + 1]), sat);
-            uint4 *dst = reinterpret_cast<uint4 *>(yrow + ch * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
-                                  packed[4 * v + 3]);
+          for (int k = 0; k < 32; ++k) {
+            const int a = __shfl_sync(0xffffffffu, my_a, k);
+            const float gv = __shfl_sync(0xffffffffu, my_g, k);
+            if (a >= 0)
+              y[static_cast<size_t>(a) * p.out_ld + f] = __ushort_as_half(f16_sat(gv * __uint_as_float(v[k]), sat));
           }
         }
       }
@@ -501,21 +549,24 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_a, con
 
 template <int kMode>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
-    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                             const __grid_constant__ CUtensorMap tmap_b, GemmArgs p) {
-  grouped_gemm_body<kMode, true>(tmap_a, tmap_b, p);
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_tok,
+                             const __grid_constant__ CUtensorMap tmap_w, GemmArgs p) {
+  grouped_gemm_body<kMode, true>(tmap_tok, tmap_w, p);
 }
 
 template <int kMode>
 __global__ void __launch_bounds__(gg::THREADS, 1)
-    grouped_gemm_solo_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                             const __grid_constant__ CUtensorMap tmap_b, GemmArgs p) {
-  grouped_gemm_body<kMode, false>(tmap_a, tmap_b, p);
+    grouped_gemm_solo_kernel(const __grid_constant__ CUtensorMap tmap_tok,
+                             const __grid_constant__ CUtensorMap tmap_w, GemmArgs p) {
+  grouped_gemm_body<kMode, false>(tmap_tok, tmap_w, p);
 }
 
-bool gemm_use_pairs(int64_t T, int K, int E) { return T * K >= 512LL * E; }
+// CTA pairs unless the experts average fewer than 8 rows each (decode), where
+// single CTAs keep more weight bytes in flight per SM
+bool gemm_use_pairs(int64_t T, int K, int E) { return T * K >= 8LL * (E > 0 ? E : 1); }
 
-int gemm_b_box_rows(bool pair) { return pair ? gg::Cfg<true>::B_ROWS : gg::Cfg<false>::B_ROWS; }
+int gemm_tok_box_rows() { return gg::TOK_BOX; }
+int gemm_w_box_rows() { return gg::BM; }
 
 template <int kMode>
 static cudaError_t launch_mode(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p,

@@ -31,25 +31,32 @@ struct GemmArgs {
                            // the MMA warp's bounded wait runs out (MOE_ERR_TIMEOUT)
 };
 
-// Tile shape of the grouped GEMMs: CTA pairs with 256-row tiles when the
-// experts get many rows each (T*K >= 512*E), single CTAs with 128-row tiles
-// otherwise (less padding of each expert's last tile, more weight bytes in
-// flight per SM for small batches).  A tiles are 128 rows; the B box has
-// gemm_b_box_rows(pair) rows.
+// Tile shape of the grouped GEMMs: the weights are the MMA's M side (256 rows
+// per CTA pair, 128 per single CTA), the tokens its N side (up to 256 per
+// tile, rounded up to 16).  CTA pairs unless the experts average fewer than 8
+// rows each.  Tensor maps: tokens [rows][K] with boxes of gemm_tok_box_rows()
+// rows, weights [rows][K] with boxes of gemm_w_box_rows() rows, 64 K-elements
+// wide, 128-byte swizzle.
 bool gemm_use_pairs(int64_t T, int K, int E);
-int gemm_b_box_rows(bool pair);
-cudaError_t launch_grouped_gemm(int mode, bool pair, const CUtensorMap &ta, const CUtensorMap &tb,
-                                const GemmArgs &p, int num_sms, cudaStream_t stream);
+int gemm_tok_box_rows();
+int gemm_w_box_rows();
+cudaError_t launch_grouped_gemm(int mode, bool pair, const CUtensorMap &tmap_tok,
+                                const CUtensorMap &tmap_w, const GemmArgs &p, int num_sms,
+                                cudaStream_t stream);
 
 // router: W_r split into bf16 parts [3][e_pad][H] (wsplit), fp32 partial logits
-// zp [splits][T][e_pad]; tmap_x: x [T][H] box 64 x 128, tmap_w: wsplit [3*e_pad][H]
-// box 64 x e_pad
+// zp [splits][T][e_pad] (split-K only); tmap_x: x [T][H] box 64 x 128,
+// tmap_w: wsplit [3*e_pad][H] box 64 x e_pad; grid_counter: an int zeroed
+// before the launch (split-K grid barrier)
 int router_e_pad(int E);
-int router_splits(int T, int H);
-cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, const float *w_r,
-                         const float *bias, int T, int H, int E, int K, float scale,
-                         uint16_t *wsplit, float *zp, int32_t *idx, float *gate, float *margin,
-                         float *logits, int *err, int num_sms, cudaStream_t stream);
+int router_splits(int T, int H);  // upper bound of the split count (workspace sizing)
+int router_grid_splits(int T, int H, int num_sms);
+cudaError_t launch_router_split(const float *w_r, int E, int H, uint16_t *wsplit, int num_sms,
+                                cudaStream_t stream);
+cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, const float *bias, int T,
+                         int H, int E, int K, float scale, float *zp, int *grid_counter,
+                         int32_t *idx, float *gate, float *margin, float *logits, int *err,
+                         int num_sms, cudaStream_t stream);
 
 // chunk scratch: int32 [E * nchunks]
 int permute_num_chunks(int64_t n_assign);
@@ -67,17 +74,42 @@ cudaError_t launch_gather_rows(const uint16_t *x, const int32_t *sorted, int T, 
 cudaError_t launch_combine(const uint16_t *Y, const uint16_t *residual, uint16_t *y, int T, int H,
                            int K, int has_shared, int num_sms, cudaStream_t stream);
 
-// offsets = {0, T}, sorted[t] = t: every token in one group, in order
+// offsets = {0, T}, sorted[t] = base + t: every token in one group, in order
 cudaError_t launch_identity_rows(int32_t *offsets, int32_t *sorted, int T, int num_sms,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, int base = 0);
+
+// expert-parallel dispatch / return (ep.cu); peers: one device pointer per rank
+constexpr int kEpMaxRanks = 8;
+struct EpPtrs {
+  void *p[kEpMaxRanks];
+};
+struct EpInts {
+  int v[kEpMaxRanks + 1];
+};
+struct EpI64 {
+  int64_t v[kEpMaxRanks];
+};
+cudaError_t launch_ep_plan(int n_ranks, int rank, int E, const EpInts &expert_first,
+                           const int32_t *counts_all, int32_t *dst_row, int32_t *recv_offsets,
+                           int32_t *recv_sorted, int64_t max_rows, int *err, int num_sms,
+                           cudaStream_t stream);
+cudaError_t launch_ep_dispatch(int n_ranks, int rank, int T, int H, int E, int K,
+                               const EpInts &expert_first, const EpI64 &capacity,
+                               const int32_t *dst_row, const uint16_t *x, const float *gate,
+                               const int32_t *offsets, const int32_t *sorted, const EpPtrs &recv_x,
+                               const EpPtrs &recv_gate, const EpPtrs &recv_src, int *err,
+                               int num_sms, cudaStream_t stream);
+cudaError_t launch_ep_return(int n_ranks, int rows, int H, const int32_t *recv_src,
+                             const uint16_t *y_local, const EpPtrs &dst_y, const EpInts &dst_rows,
+                             int *err, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_rmsnorm(const uint16_t *x, const uint16_t *gamma, float eps, int T, int H,
                            uint16_t *out, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_pack(const uint16_t *w1, const uint16_t *w3, const uint16_t *w2,
                         const uint16_t *ws1, const uint16_t *ws3, const uint16_t *ws2, int H, int I,
-                        int E, int has_shared, uint16_t *w13_out, uint16_t *w2_out, int num_sms,
-                        cudaStream_t stream);
+                        int E, int has_shared, uint16_t *w13_out, uint16_t *w2_out,
+                        int32_t *w2_inexact, int num_sms, cudaStream_t stream);
 
 // ---- sparse-attention key selection (dsa.cu)
 constexpr int kDsaMaxKeys = 32768;  // keys per sequence the top-k kernel holds in registers

@@ -39,12 +39,16 @@ static __device__ __align__(256) int32_t g_permute_scratch[kErrWords + kMaxE * k
 
 // Address of g_permute_scratch on each device, looked up once per device with
 // that device current (in host code the symbol is only a host-side handle).
+// The address is kept for the life of the process: a cudaDeviceReset after the
+// first call may move the array, so resetting a device that this entry point
+// has used is not supported.
 std::mutex g_mutex;
 int32_t *g_scratch_ptr[kDevices] = {nullptr};
 
 moe_status_t scratch_for_current_device(int32_t **out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return MOE_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return MOE_ERR_CUDA;
+  if (dev >= kDevices) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!g_scratch_ptr[dev]) {
     void *p = nullptr;

@@ -1,5 +1,5 @@
-// router.cu -- the router: logits on the tensor cores, then sigmoid scores,
-// biased top-K selection and renormalised, scaled gates.
+// router.cu -- the router in one kernel: logits on the tensor cores, then
+// sigmoid scores, biased top-K selection and renormalised, scaled gates.
 //
 // Definition ("GLM-5 . MoE transformer block", "All 43 steps", Mixture of
 // experts):  z = x W_r;  s = sigmoid(z);  E_sel_i = [i in top_K(s + b)];
@@ -15,18 +15,22 @@
 // product exact and fp32 accumulation: fp32-accurate logits at bf16 tensor-
 // core speed.
 //   1) router_split_kernel: W_r -> [3][E_pad][H] bf16 (E_pad = E rounded up
-//      to 64, padding rows zero), once per call (6 MB read, 9 MB written at
-//      the GLM-5 shape).
-//   2) router_logits_kernel: 128 tokens x E_pad experts per CTA, tcgen05.mma
+//      to 64, padding rows zero).  A property of the weights: moe_pack_router
+//      runs it once; moe_route (fp32 W_r given per call) runs it every call.
+//   2) router_kernel: 128 tokens x E_pad experts per CTA, tcgen05.mma
 //      kind::f16 (bf16) into tensor memory, TMA-fed ring, short accumulation
-//      chains promoted to fp32 registers (see below); the H range may be split
-//      over S CTAs (S > 1 when there are few 128-token tiles) and each CTA
-//      writes fp32 partial logits zp[s][t][e].
-//   2b) router_reduce_kernel (S > 1): one thread per (token, expert) sums the
-//      S partials in a fixed order (deterministic).
-//   3) router_select_kernel: one warp per token: s, keys, K rounds of a warp
-//      arg-max (key descending, index ascending), one more round for the
-//      margin, gates.
+//      chains promoted to fp32 registers (see below), then the selection in
+//      the same kernel:
+//        - one CTA per 128 tokens (no split of H): the epilogue warps stage
+//          their fp32 z rows in shared memory (the drained operand ring) and
+//          each warp selects for its tokens: s, keys, K rounds of a warp
+//          arg-max (key descending, index ascending), one more round for the
+//          margin, gates.  z never reaches global memory unless asked for.
+//        - few 128-token tiles (decode): the H range is split over S CTAs;
+//          each writes fp32 partial logits, all CTAs of the grid (at most one
+//          per SM, so all resident together) meet at a bounded grid barrier,
+//          then every CTA takes some tokens, sums the S partials in a fixed
+//          order (deterministic) and selects.
 #include <cuda.h>
 #include <math.h>
 
@@ -106,7 +110,7 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// ---------------------------------------------------------------- 2) logits
+// ---------------------------------------------------------------- 2) logits + selection
 
 // The tensor core's fp32 accumulator loses precision over long chains of
 // MMAs (measured on B200: max |dz| 1.5e-4 after 1152 chained MMAs against
@@ -125,22 +129,132 @@ struct RouterSmem {
   int mma_consumed;
 };
 
+struct RouteOut {
+  const float *bias;
+  int32_t *idx;
+  float *gate;
+  float *margin;  // may be null
+  float *logits;  // may be null: [T][E]
+  float scale;
+  int T, E, K;
+};
+
+// Selection for one token by one warp from its E logits zrow[e] (shared or
+// global memory, e < E read): s = sigmoid(z), key = s + b, K rounds of a warp
+// arg-max (key descending, equal keys to the lower index), one more round for
+// the margin; gates = scale * s / sum of the selected s.  bias_r[j] holds
+// bias[lane + 32 j] (this lane's experts).
+template <int NE>
+__device__ __forceinline__ void select_token(const float *zrow, const float (&bias_r)[NE], int t,
+                                             const RouteOut &o, int lane) {
+  float key[NE], sv[NE];
+#pragma unroll
+  for (int j = 0; j < NE; ++j) {
+    const int e = lane + 32 * j;
+    float z = 0.f;
+    if (e < o.E) {
+      z = zrow[e];
+      if (o.logits) o.logits[static_cast<size_t>(t) * o.E + e] = z;
+    }
+    const float sj = sigmoidf_(z);
+    sv[j] = sj;
+    key[j] = e < o.E ? sj + bias_r[j] : -INFINITY;
+  }
+  int my_e = 0;
+  float my_s = 0.f, kth_key = 0.f, next_key = -INFINITY;
+  const int K = o.K;
+  const int rounds = K < o.E ? K + 1 : K;
+  for (int k = 0; k < rounds; ++k) {
+    float bk = -INFINITY, bs = 0.f;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NE; ++j) {
+      if (key[j] > bk) {  // j ascending = expert index ascending: strict > keeps the lower
+        bk = key[j];
+        be = lane + 32 * j;
+        bs = sv[j];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+      if (ok > bk || (ok == bk && oe < be)) {
+        bk = ok;
+        be = oe;
+        bs = os;
+      }
+    }
+    if (k == K) {
+      next_key = bk;
+      break;
+    }
+    if (lane == k) {
+      my_e = be;
+      my_s = bs;
+    }
+    if (k == K - 1) kth_key = bk;
+#pragma unroll
+    for (int j = 0; j < NE; ++j)
+      if (be == lane + 32 * j) key[j] = -INFINITY;
+  }
+  float denom = 0.f;
+  for (int k = 0; k < K; ++k) denom += __shfl_sync(0xffffffffu, my_s, k);
+  if (lane < K) {
+    o.idx[static_cast<size_t>(t) * K + lane] = my_e;
+    o.gate[static_cast<size_t>(t) * K + lane] = o.scale * my_s / denom;
+  }
+  if (o.margin && lane == 0) o.margin[t] = K < o.E ? kth_key - next_key : INFINITY;
+}
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Grid barrier of a launch whose CTAs are all resident together (the grid is
+// at most one CTA per SM): one arrival per CTA on a counter that is zero
+// before the launch, then a wait bounded by kWaitLimitNs.  Returns false (and
+// records MOE_ERR_TIMEOUT) if the wait ran out.
+__device__ __forceinline__ bool grid_barrier(int *counter, int n_ctas, int *err) {
+  __shared__ int ok;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(counter, 1);
+    const uint64_t t0 = global_timer_ns();
+    int seen = 0;
+    while (true) {
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(seen) : "l"(counter) : "memory");
+      if (seen >= n_ctas) break;
+      if (global_timer_ns() - t0 > kWaitLimitNs) break;
+    }
+    ok = seen >= n_ctas;
+    if (!ok) record_error(err, MOE_ERR_TIMEOUT);
+  }
+  __syncthreads();
+  return ok != 0;
+}
+
 // NH = e_pad / 64: each epilogue thread keeps half a row (e_pad / 2 columns).
-template <int NH>
+// kSplit: the H range is split over gridDim.y CTAs (partials + grid barrier).
+template <int NH, bool kSplit>
 __global__ void __launch_bounds__(rt::THREADS, 1)
-    router_logits_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                         const __grid_constant__ CUtensorMap tmap_w, int T, int kb_per_split,
-                         int kblocks, int stages, uint32_t tmem_cols, float *__restrict__ zp,
-                         int *err) {
+    router_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                  int kb_per_split, int kblocks, int stages, uint32_t tmem_cols,
+                  float *__restrict__ zp, int *grid_counter, RouteOut o, int *err) {
   using namespace rt;
   constexpr int e_pad = NH * 64;
   constexpr int HALF = e_pad / 2;
+  constexpr int NE = e_pad / 32;         // experts per lane in the selection
+  constexpr int ZS = e_pad + 4;          // shared-memory row stride of staged z (floats)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   uint8_t *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   constexpr int stage_bytes = A_BYTES + 3 * e_pad * BK * 2;
   RouterSmem &s = *reinterpret_cast<RouterSmem *>(base + stages * stage_bytes);
+  float *zs = reinterpret_cast<float *>(base);  // staged z rows, over the drained ring
 
+  const int T = o.T;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * BM;
   const int split = blockIdx.y;
@@ -270,12 +384,36 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.tempty[slot]);
     }
-    if (ok && t < T) {
-      float4 *d4 = reinterpret_cast<float4 *>(zp + (static_cast<size_t>(split) * T + t) * e_pad +
-                                              hf * HALF);
+    if (kSplit) {
+      if (ok && t < T) {
+        float4 *d4 = reinterpret_cast<float4 *>(zp + (static_cast<size_t>(split) * T + t) * e_pad +
+                                                hf * HALF);
 #pragma unroll
-      for (int v = 0; v < HALF / 4; ++v)
-        d4[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+        for (int v = 0; v < HALF / 4; ++v)
+          d4[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+      }
+    } else {
+      // Every MMA has completed (its tfull arrived) and so has every copy it
+      // read: the operand ring is free.  Stage the 128 x e_pad tile of z there
+      // (row stride ZS floats: the 8 rows of one 16-byte store phase fall in
+      // distinct banks), then each epilogue warp selects for 16 tokens.
+      if (ok) {
+        float4 *d4 = reinterpret_cast<float4 *>(zs + row * ZS + hf * HALF);
+#pragma unroll
+        for (int v = 0; v < HALF / 4; ++v)
+          d4[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+      }
+      named_barrier(1, 32 * EPI_WARPS);
+      if (!*abort_flag) {
+        float bias_r[NE];
+#pragma unroll
+        for (int j = 0; j < NE; ++j) {
+          const int e = lane + 32 * j;
+          bias_r[j] = e < o.E ? o.bias[e] : 0.f;
+        }
+        for (int r = warp - 2; r < BM && m0 + r < T; r += EPI_WARPS)
+          select_token<NE>(zs + r * ZS, bias_r, m0 + r, o, lane);
+      }
     }
   }
 
@@ -304,6 +442,43 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
   }
+
+  if (kSplit) {
+    // Every CTA's partials are written; after the grid barrier each CTA takes
+    // tokens t = cta, cta + n_ctas, ...: warp j sums the S partials of experts
+    // 32j .. 32j+31 in split order (eight interleaved accumulators combined in
+    // a fixed tree: deterministic, whichever CTA does it), stages z in shared
+    // memory, and one warp selects.
+    const int n_ctas = gridDim.x * gridDim.y;
+    const int cta = blockIdx.y * gridDim.x + blockIdx.x;
+    const int splits = gridDim.y;
+    if (!grid_barrier(grid_counter, n_ctas, err)) return;
+    float bias_r[NE];
+#pragma unroll
+    for (int j = 0; j < NE; ++j) {
+      const int e = lane + 32 * j;
+      bias_r[j] = e < o.E ? o.bias[e] : 0.f;
+    }
+    const size_t plane = static_cast<size_t>(T) * e_pad;
+    for (int tt = cta; tt < T; tt += n_ctas) {
+      if (warp < NE) {
+        const float *src = zp + static_cast<size_t>(tt) * e_pad + warp * 32 + lane;
+        float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        int sp = 0;
+        for (; sp + 8 <= splits; sp += 8) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) a8[u] += __ldcg(src + (sp + u) * plane);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (sp + u < splits) a8[u] += __ldcg(src + (sp + u) * plane);
+        zs[warp * 32 + lane] = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+      }
+      __syncthreads();
+      if (warp == 0) select_token<NE>(zs, bias_r, tt, o, lane);
+      __syncthreads();
+    }
+  }
 }
 
 int router_stages(int e_pad) {
@@ -311,161 +486,80 @@ int router_stages(int e_pad) {
   return s > 4 ? 4 : s;
 }
 
-// ---------------------------------------------------------------- 2b) split-K sum
-
-// z[t][e] = sum over the S partials, written over partial 0.  One thread per
-// (token, expert); eight independent accumulators (split s goes to s mod 8)
-// added in a fixed order at the end: deterministic, and eight loads in flight.
-__global__ void __launch_bounds__(256)
-    router_reduce_kernel(float *__restrict__ zp, int splits, int T, int e_pad) {
-  const int64_t n = static_cast<int64_t>(T) * e_pad;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    int sp = 0;
-    for (; sp + 8 <= splits; sp += 8) {
-#pragma unroll
-      for (int u = 0; u < 8; ++u) acc[u] += zp[(sp + u) * n + i];
-    }
-    for (int u = 0; sp < splits; ++sp, ++u) acc[u] += zp[sp * n + i];
-    zp[i] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-  }
-}
-
-// ---------------------------------------------------------------- 3) select
-
-template <int NE>
-__global__ void __launch_bounds__(256)
-    router_select_kernel(const float *__restrict__ zp, int splits, const float *__restrict__ bias,
-                         int T, int E, int e_pad, int K, float scale, int32_t *__restrict__ idx,
-                         float *__restrict__ gate, float *__restrict__ margin,
-                         float *__restrict__ logits) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;  // whole warp
-  float key[NE], sv[NE];
-#pragma unroll
-  for (int j = 0; j < NE; ++j) {
-    const int e = lane + 32 * j;
-    float z = 0.f;
-    if (e < E) {
-      z = zp[static_cast<size_t>(t) * e_pad + e];
-      if (logits) logits[static_cast<size_t>(t) * E + e] = z;
-    }
-    const float sj = sigmoidf_(z);
-    sv[j] = sj;
-    key[j] = e < E ? sj + bias[e] : -INFINITY;
-  }
-  int my_e = 0;
-  float my_s = 0.f, kth_key = 0.f, next_key = -INFINITY;
-  const int rounds = K < E ? K + 1 : K;
-  for (int k = 0; k < rounds; ++k) {
-    float bk = -INFINITY, bs = 0.f;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < NE; ++j) {
-      if (key[j] > bk) {  // j ascending = expert index ascending: strict > keeps the lower
-        bk = key[j];
-        be = lane + 32 * j;
-        bs = sv[j];
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-      if (ok > bk || (ok == bk && oe < be)) {
-        bk = ok;
-        be = oe;
-        bs = os;
-      }
-    }
-    if (k == K) {
-      next_key = bk;
-      break;
-    }
-    if (lane == k) {
-      my_e = be;
-      my_s = bs;
-    }
-    if (k == K - 1) kth_key = bk;
-#pragma unroll
-    for (int j = 0; j < NE; ++j)
-      if (be == lane + 32 * j) key[j] = -INFINITY;
-  }
-  float denom = 0.f;
-  for (int k = 0; k < K; ++k) denom += __shfl_sync(0xffffffffu, my_s, k);
-  if (lane < K) {
-    idx[static_cast<size_t>(t) * K + lane] = my_e;
-    gate[static_cast<size_t>(t) * K + lane] = scale * my_s / denom;
-  }
-  if (margin && lane == 0) margin[t] = K < E ? kth_key - next_key : INFINITY;
-}
-
 // ---------------------------------------------------------------- launch
 
-template <int NH>
-static cudaError_t launch_logits(dim3 grid, size_t smem, const CUtensorMap &tmap_x,
-                                 const CUtensorMap &tmap_w, int T, int kb_per, int kblocks,
-                                 int stages, uint32_t cols, float *zp, int *err,
-                                 cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<NH>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  router_logits_kernel<NH><<<grid, rt::THREADS, smem, stream>>>(tmap_x, tmap_w, T, kb_per, kblocks,
-                                                                stages, cols, zp, err);
-  return cudaGetLastError();
-}
-
-size_t router_logits_smem_bytes(int e_pad) {
+size_t router_smem_bytes(int e_pad) {
   return 1024 + static_cast<size_t>(router_stages(e_pad)) * router_stage_bytes(e_pad) +
          sizeof(RouterSmem);
 }
 
-cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, const float *w_r,
-                         const float *bias, int T, int H, int E, int K, float scale,
-                         uint16_t *wsplit, float *zp, int32_t *idx, float *gate, float *margin,
-                         float *logits, int *err, int num_sms, cudaStream_t stream) {
-  const int e_pad = router_e_pad(E);
-  router_split_kernel<<<num_sms * 4, 256, 0, stream>>>(w_r, E, e_pad, H, wsplit);
-  const int kblocks = H / rt::BK;
-  const int splits = router_splits(T, H);
-  const int kb_per = (kblocks + splits - 1) / splits;
+template <int NH, bool kSplit>
+static cudaError_t launch_router_kernel(dim3 grid, const CUtensorMap &tmap_x, const CUtensorMap &tmap_w,
+                                        int kb_per, int kblocks, float *zp, int *grid_counter,
+                                        const RouteOut &o, int *err, cudaStream_t stream) {
+  constexpr int e_pad = NH * 64;
+  const size_t smem = router_smem_bytes(e_pad);
   const int stages = router_stages(e_pad);
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(2 * e_pad)) cols <<= 1;  // two ping-pong accumulators
-  const size_t smem = router_logits_smem_bytes(e_pad);
-  dim3 grid((T + rt::BM - 1) / rt::BM, (kblocks + kb_per - 1) / kb_per);
-  cudaError_t e = cudaSuccess;
-  switch (e_pad / 64) {
-    case 1: e = launch_logits<1>(grid, smem, tmap_x, tmap_w, T, kb_per, kblocks, stages, cols, zp, err, stream); break;
-    case 2: e = launch_logits<2>(grid, smem, tmap_x, tmap_w, T, kb_per, kblocks, stages, cols, zp, err, stream); break;
-    case 3: e = launch_logits<3>(grid, smem, tmap_x, tmap_w, T, kb_per, kblocks, stages, cols, zp, err, stream); break;
-    default: e = launch_logits<4>(grid, smem, tmap_x, tmap_w, T, kb_per, kblocks, stages, cols, zp, err, stream); break;
-  }
+  cudaError_t e = cudaFuncSetAttribute(router_kernel<NH, kSplit>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int used_splits = static_cast<int>(grid.y);
-  if (used_splits > 1) {
-    const int64_t n = static_cast<int64_t>(T) * e_pad;
-    int rb = static_cast<int>((n + 255) / 256);
-    if (rb > num_sms * 8) rb = num_sms * 8;
-    router_reduce_kernel<<<rb, 256, 0, stream>>>(zp, used_splits, T, e_pad);
-  }
-  const int blocks = (T + 7) / 8;
-  if (E <= 32)
-    router_select_kernel<1><<<blocks, 256, 0, stream>>>(zp, 1, bias, T, E, e_pad, K, scale,
-                                                        idx, gate, margin, logits);
-  else if (E <= 64)
-    router_select_kernel<2><<<blocks, 256, 0, stream>>>(zp, 1, bias, T, E, e_pad, K, scale,
-                                                        idx, gate, margin, logits);
-  else if (E <= 128)
-    router_select_kernel<4><<<blocks, 256, 0, stream>>>(zp, 1, bias, T, E, e_pad, K, scale,
-                                                        idx, gate, margin, logits);
-  else
-    router_select_kernel<8><<<blocks, 256, 0, stream>>>(zp, 1, bias, T, E, e_pad, K, scale,
-                                                        idx, gate, margin, logits);
+  router_kernel<NH, kSplit><<<grid, rt::THREADS, smem, stream>>>(tmap_x, tmap_w, kb_per, kblocks, stages,
+                                                                 cols, zp, grid_counter, o, err);
   return cudaGetLastError();
+}
+
+cudaError_t launch_router_split(const float *w_r, int E, int H, uint16_t *wsplit, int num_sms,
+                                cudaStream_t stream) {
+  router_split_kernel<<<num_sms * 4, 256, 0, stream>>>(w_r, E, router_e_pad(E), H, wsplit);
+  return cudaGetLastError();
+}
+
+int router_grid_splits(int T, int H, int num_sms) {
+  const int m_tiles = (T + rt::BM - 1) / rt::BM;
+  int s = router_splits(T, H);
+  const int fit = num_sms / (m_tiles > 0 ? m_tiles : 1);  // the whole grid resident at once
+  if (s > fit) s = fit;
+  if (s < 1) s = 1;
+  const int kblocks = H / rt::BK;
+  const int kb_per = (kblocks + s - 1) / s;
+  return (kblocks + kb_per - 1) / kb_per;  // splits that get at least one k-block
+}
+
+cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, const float *bias, int T,
+                         int H, int E, int K, float scale, float *zp, int *grid_counter,
+                         int32_t *idx, float *gate, float *margin, float *logits, int *err,
+                         int num_sms, cudaStream_t stream) {
+  const int kblocks = H / rt::BK;
+  const int splits = router_grid_splits(T, H, num_sms);
+  const int kb_per = (kblocks + splits - 1) / splits;
+  dim3 grid((T + rt::BM - 1) / rt::BM, splits);
+  RouteOut o;
+  o.bias = bias;
+  o.idx = idx;
+  o.gate = gate;
+  o.margin = margin;
+  o.logits = logits;
+  o.scale = scale;
+  o.T = T;
+  o.E = E;
+  o.K = K;
+  const int nh = router_e_pad(E) / 64;
+  if (splits > 1) {
+    switch (nh) {
+      case 1: return launch_router_kernel<1, true>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
+      case 2: return launch_router_kernel<2, true>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
+      case 3: return launch_router_kernel<3, true>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
+      default: return launch_router_kernel<4, true>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
+    }
+  }
+  switch (nh) {
+    case 1: return launch_router_kernel<1, false>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
+    case 2: return launch_router_kernel<2, false>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
+    case 3: return launch_router_kernel<3, false>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
+    default: return launch_router_kernel<4, false>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
+  }
 }
 
 }  // namespace srm

@@ -27,6 +27,9 @@ SYMBOLS = (
     "moe_workspace_size",
     "moe_pack_weights",
     "moe_route",
+    "moe_router_packed_size",
+    "moe_pack_router",
+    "moe_route_packed",
     "moe_permute",
     "moe_forward",
     "moe_gather_tokens",
@@ -117,9 +120,15 @@ def lib():
         L.moe_workspace_size.restype = ctypes.c_size_t
         L.moe_workspace_size.argtypes = [P(_Cfg)]
         L.moe_pack_weights.restype = ctypes.c_int
-        L.moe_pack_weights.argtypes = [P(_Cfg)] + [vp] * 9
+        L.moe_pack_weights.argtypes = [P(_Cfg)] + [vp] * 10
         L.moe_route.restype = ctypes.c_int
         L.moe_route.argtypes = [P(_Cfg)] + [vp] * 8 + [ctypes.c_size_t, vp]
+        L.moe_router_packed_size.restype = ctypes.c_size_t
+        L.moe_router_packed_size.argtypes = [P(_Cfg)]
+        L.moe_pack_router.restype = ctypes.c_int
+        L.moe_pack_router.argtypes = [P(_Cfg), vp, vp, vp]
+        L.moe_route_packed.restype = ctypes.c_int
+        L.moe_route_packed.argtypes = [P(_Cfg)] + [vp] * 8 + [ctypes.c_size_t, vp]
         L.moe_permute.restype = ctypes.c_int
         L.moe_permute.argtypes = [P(_Cfg), vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.moe_forward.restype = ctypes.c_int
@@ -196,8 +205,11 @@ def workspace(cfg: Config, device=None) -> torch.Tensor:
     return torch.empty(workspace_bytes(cfg), dtype=torch.uint8, device=device or "cuda")
 
 
-def pack_weights(cfg: Config, w1, w3, w2, ws1=None, ws3=None, ws2=None, stream=None):
-    """Returns (w13 bf16 [(E+1)*2I, H], w2p fp16 [(E+1)*H, I]) in the kernels' layout."""
+def pack_weights(cfg: Config, w1, w3, w2, ws1=None, ws3=None, ws2=None, stream=None, inexact=None):
+    """Returns (w13 bf16 [(E+1)*2I, H], w2p fp16 [(E+1)*H, I]) in the kernels' layout.
+    inexact: optional int32 [1] device tensor; receives the number of W2 values
+    whose fp16 copy is not exact (saturated beyond 65504, or rounded below fp16's
+    2^-24 spacing)."""
     E, I, H = cfg.E, cfg.I, cfg.H
     bf = torch.bfloat16
     if E > 0 or w1 is not None:
@@ -211,28 +223,65 @@ def pack_weights(cfg: Config, w1, w3, w2, ws1=None, ws3=None, ws2=None, stream=N
     dev = (w1 if w1 is not None else ws1).device
     w13 = torch.empty(((E + 1) * 2 * I, H), dtype=bf, device=dev)
     w2p = torch.empty(((E + 1) * H, I), dtype=torch.float16, device=dev)
+    if inexact is not None:
+        _req(inexact, torch.int32, (1,), "inexact")
     _check(lib().moe_pack_weights(ctypes.byref(cfg.c()), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(ws1),
-                                  _ptr(ws3), _ptr(ws2), _ptr(w13), _ptr(w2p), _stream(stream)),
+                                  _ptr(ws3), _ptr(ws2), _ptr(w13), _ptr(w2p), _ptr(inexact),
+                                  _stream(stream)),
            "moe_pack_weights")
     return w13, w2p
+
+
+def _route_outputs(cfg, x, want_margin, out):
+    T, K = cfg.T, cfg.K
+    if out is None:
+        idx = torch.empty((T, K), dtype=torch.int32, device=x.device)
+        gate = torch.empty((T, K), dtype=torch.float32, device=x.device)
+        margin = torch.empty((T,), dtype=torch.float32, device=x.device) if want_margin else None
+        return idx, gate, margin
+    return out
 
 
 def route(cfg: Config, x, w_router, bias, ws, want_margin=True, out=None, logits=None, stream=None):
     """Router: returns (topk_idx int32 [T,K], topk_gate fp32 [T,K], margin fp32 [T] or None).
     ``logits``: optional fp32 [T, E] tensor that receives z (router_logits)."""
-    T, H, E, K = cfg.T, cfg.H, cfg.E, cfg.K
+    T, H, E = cfg.T, cfg.H, cfg.E
     _req(x, torch.bfloat16, (T, H), "x")
     _req(w_router, torch.float32, (E, H), "w_router")
     _req(bias, torch.float32, (E,), "bias")
-    if out is None:
-        idx = torch.empty((T, K), dtype=torch.int32, device=x.device)
-        gate = torch.empty((T, K), dtype=torch.float32, device=x.device)
-        margin = torch.empty((T,), dtype=torch.float32, device=x.device) if want_margin else None
-    else:
-        idx, gate, margin = out
+    idx, gate, margin = _route_outputs(cfg, x, want_margin, out)
     _check(lib().moe_route(ctypes.byref(cfg.c()), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(idx),
                            _ptr(gate), _ptr(margin), _ptr(logits), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_route")
+    return idx, gate, margin
+
+
+def pack_router(cfg: Config, w_router, stream=None):
+    """The exact three-part bf16 split of W_r (fp32 [E, H]) as a uint8 device
+    tensor of moe_router_packed_size bytes, for route_packed."""
+    _req(w_router, torch.float32, (cfg.E, cfg.H), "w_router")
+    n = lib().moe_router_packed_size(ctypes.byref(cfg.c()))
+    if n == 0:
+        raise MoeError(1, "moe_router_packed_size")
+    packed = torch.empty((n,), dtype=torch.uint8, device=w_router.device)
+    _check(lib().moe_pack_router(ctypes.byref(cfg.c()), _ptr(w_router), _ptr(packed), _stream(stream)),
+           "moe_pack_router")
+    return packed
+
+
+def route_packed(cfg: Config, x, w_router_packed, bias, ws, want_margin=True, out=None, logits=None,
+                 stream=None):
+    """route() with the router weights from pack_router: one kernel."""
+    T, H, E = cfg.T, cfg.H, cfg.E
+    _req(x, torch.bfloat16, (T, H), "x")
+    n = lib().moe_router_packed_size(ctypes.byref(cfg.c()))
+    _req(w_router_packed, torch.uint8, (n,), "w_router_packed")
+    _req(bias, torch.float32, (E,), "bias")
+    idx, gate, margin = _route_outputs(cfg, x, want_margin, out)
+    _check(lib().moe_route_packed(ctypes.byref(cfg.c()), _ptr(x), _ptr(w_router_packed), _ptr(bias),
+                                  _ptr(idx), _ptr(gate), _ptr(margin), _ptr(logits), _ptr(ws), ws.numel(),
+                                  _stream(stream)),
+           "moe_route_packed")
     return idx, gate, margin
 
 
@@ -363,11 +412,15 @@ def device_error(ws, stream=None) -> int:
 class MoeBlock:
     """One MoE block with packed weights and a workspace: ``y = block(x)``."""
 
-    def __init__(self, cfg: Config, w_router, bias, w1, w3, w2, ws1=None, ws3=None, ws2=None):
+    def __init__(self, cfg: Config, w_router, bias, w1, w3, w2, ws1=None, ws3=None, ws2=None,
+                 packed=None):
         self.cfg = cfg
         self.w_router = w_router
         self.bias = bias
-        self.weights = pack_weights(cfg, w1, w3, w2, ws1, ws3, ws2)
+        # packed: (w13, w2) from pack_weights for this block's H, I and E, shared
+        # with another block of the same shapes instead of packing again
+        self.weights = packed if packed is not None else pack_weights(cfg, w1, w3, w2, ws1, ws3, ws2)
+        self.router_packed = pack_router(cfg, w_router)
         self.ws = workspace(cfg, device=w_router.device)
         dev = w_router.device
         T, K, E = cfg.T, cfg.K, cfg.E
@@ -383,8 +436,8 @@ class MoeBlock:
         """The decoder block's FFN sublayer: x' + MoE(RMSNorm(x')) (bf16 [T, H])."""
         cfg = self.cfg
         x_ffn = rmsnorm(cfg, x_resid, gamma, eps, stream=stream)
-        route(cfg, x_ffn, self.w_router, self.bias, self.ws, out=(self.idx, self.gate, self.margin),
-              logits=logits, stream=stream)
+        route_packed(cfg, x_ffn, self.router_packed, self.bias, self.ws,
+                     out=(self.idx, self.gate, self.margin), logits=logits, stream=stream)
         permute(cfg, self.idx, self.ws, out=(self.counts, self.offsets, self.sorted), stream=stream)
         gather_tokens(cfg, x_ffn, self.sorted, self.ws, stream=stream)
         expert_up(cfg, self.weights, self.offsets, self.sorted, self.ws, stream=stream)
@@ -393,8 +446,8 @@ class MoeBlock:
         return self.y, x_ffn
 
     def __call__(self, x, stream=None, logits=None):
-        route(self.cfg, x, self.w_router, self.bias, self.ws, out=(self.idx, self.gate, self.margin),
-              logits=logits, stream=stream)
+        route_packed(self.cfg, x, self.router_packed, self.bias, self.ws,
+                     out=(self.idx, self.gate, self.margin), logits=logits, stream=stream)
         permute(self.cfg, self.idx, self.ws, out=(self.counts, self.offsets, self.sorted), stream=stream)
         return forward(self.cfg, self.weights, x, self.gate, self.offsets, self.sorted, self.ws, y=self.y,
                        stream=stream)

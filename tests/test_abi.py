@@ -1,6 +1,6 @@
 """Host-side checks of the C ABI (no GPU needed): the library loads, exports
-every entry point include/srm_moe.h and include/srm_dsa.h declare, sizes its
-workspaces and rejects invalid arguments before any launch."""
+every entry point include/srm_moe.h, include/srm_dsa.h and include/srm_ep.h
+declare, sizes its workspaces and rejects invalid arguments before any launch."""
 import ctypes
 import os
 import re
@@ -9,6 +9,7 @@ import pytest
 
 from sigmoid_routed_mixture_b200 import build as B
 from sigmoid_routed_mixture_b200 import dsa
+from sigmoid_routed_mixture_b200 import ep
 from sigmoid_routed_mixture_b200 import moe
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -37,6 +38,9 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
     assert set(moe.SYMBOLS) <= declared
     assert set(dsa.SYMBOLS) <= declared and "dsa_select" in declared
+    assert {"moe_ep_plan", "moe_ep_dispatch", "moe_ep_return", "moe_ep_shared", "moe_workspace_offset",
+            "moe_pack_router", "moe_route_packed"} <= declared
+    ep.lib()  # the expert-parallel entry points resolve and take their types
 
 
 def test_status_strings(L):
@@ -78,7 +82,7 @@ def test_null_pointers_rejected_before_launch(L):
     assert L.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None, 0, None) == 1
     assert L.moe_permute(ctypes.byref(c), None, None, None, None, None, 0, None) == 1
     assert L.moe_forward(ctypes.byref(c), None, None, None, None, None, None, None, 0, None) == 1
-    assert L.moe_pack_weights(ctypes.byref(c), None, None, None, None, None, None, None, None, None) == 1
+    assert L.moe_pack_weights(ctypes.byref(c), None, None, None, None, None, None, None, None, None, None) == 1
     st = ctypes.c_int(0)
     assert L.moe_get_device_error(None, ctypes.byref(st), None) == 1
 
@@ -91,6 +95,37 @@ def test_misaligned_and_small_workspace_rejected(L):
                        None) == 3
     need = L.moe_workspace_size(ctypes.byref(c))
     assert L.moe_permute(ctypes.byref(c), aligned, aligned, aligned, aligned, aligned, need - 1, None) == 4
+
+
+def test_router_packing_and_ep_calls_validate_before_launch(L):
+    c = cfg().c()
+    fake = ctypes.c_void_p(0x10001)
+    aligned = ctypes.c_void_p(0x100000)
+    assert L.moe_router_packed_size(ctypes.byref(c)) == 2 * 3 * 64 * 256
+    assert L.moe_router_packed_size(ctypes.byref(cfg(K=0).c())) == 0
+    assert L.moe_pack_router(ctypes.byref(c), None, None, None) == 1
+    assert L.moe_pack_router(ctypes.byref(c), fake, aligned, None) == 3
+    assert L.moe_route_packed(ctypes.byref(c), aligned, fake, aligned, aligned, aligned, None, None, aligned,
+                              1 << 40, None) == 3
+    need = L.moe_workspace_size(ctypes.byref(c))
+    assert L.moe_route_packed(ctypes.byref(c), aligned, aligned, aligned, aligned, aligned, None, None, aligned,
+                              need - 1, None) == 4
+    # the fp32 router path checks everything before its split kernel
+    assert L.moe_route(ctypes.byref(c), aligned, aligned, aligned, aligned, aligned, None, None, aligned,
+                       need - 1, None) == 4
+    assert ep.workspace_offset(cfg(), ep.WS_SLOT_OUTPUTS) > ep.workspace_offset(cfg(), ep.WS_TOKEN_ROWS) > 0
+    assert L.moe_workspace_offset(ctypes.byref(c), 7) == ctypes.c_size_t(-1).value
+    first = (ctypes.c_int32 * 3)(0, 8, 16)
+    bad_first = (ctypes.c_int32 * 3)(0, 8, 15)
+    assert L.moe_ep_plan(ctypes.byref(c), 2, 0, bad_first, aligned, aligned, aligned, aligned, 16, aligned,
+                         None) == 1
+    assert L.moe_ep_plan(ctypes.byref(c), 2, 2, first, aligned, aligned, aligned, aligned, 16, aligned, None) == 1
+    assert L.moe_ep_plan(ctypes.byref(c), 9, 0, first, aligned, aligned, aligned, aligned, 16, aligned, None) == 1
+    assert L.moe_ep_plan(ctypes.byref(c), 2, 0, first, fake, aligned, aligned, aligned, 16, aligned, None) == 3
+    owner = cfg(K=1, has_shared=False).c()
+    assert L.moe_ep_return(ctypes.byref(c), 2, aligned, None, None, aligned, 1 << 40, None) == 1  # K != 1
+    assert L.moe_ep_return(ctypes.byref(owner), 2, None, None, None, aligned, 1 << 40, None) == 1
+    assert L.moe_ep_shared(ctypes.byref(cfg(has_shared=False).c()), None, None, None, 0, None) == 1
 
 
 def test_zero_tokens_is_a_no_op(L):
@@ -159,6 +194,7 @@ C_CLIENT = r"""
 #include <stdio.h>
 #include "srm_moe.h"
 #include "srm_dsa.h"
+#include "srm_ep.h"
 
 int main(void) {
     moe_cfg_t cfg = {16384, 6144, 2048, 256, 8, 2.5f, 1};

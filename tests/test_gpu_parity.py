@@ -197,6 +197,108 @@ def test_out_of_range_expert_id_is_flagged():
     assert moe.device_error(ws) == 0  # read clears it
 
 
+@pytest.mark.parametrize("T", [64, 4096])  # single-CTA tiles, CTA-pair tiles
+def test_malformed_offsets_are_rejected_by_the_expert_stages(T):
+    """The expert stages take offsets from the caller.  A first offset other than
+    0 (the allocation-free permutation's in-band flag for a bad id), a group that
+    ends before it starts, or an end past the rows gives that group no tiles and
+    MOE_ERR_BAD_INDEX, with no access outside the buffers; the next call with
+    good offsets is exact."""
+    w = W.WORKLOADS["tiny"].replace(T=T, seed=2900 + T)
+    case = MH.Case(w)
+    blk = case.block()
+    cfg = case.cfg
+    moe.route(cfg, case.x_dev, blk.w_router, blk.bias, blk.ws, out=(blk.idx, blk.gate, blk.margin))
+    moe.permute(cfg, blk.idx, blk.ws, out=(blk.counts, blk.offsets, blk.sorted))
+    moe.gather_tokens(cfg, case.x_dev, blk.sorted, blk.ws)
+    torch.cuda.synchronize()
+    assert moe.device_error(blk.ws) == 0
+    bad_idx = blk.idx.clone()
+    bad_idx[3, 1] = w.E + 5
+    _, flagged, _ = moe.permute_noalloc(cfg, bad_idx)
+    torch.cuda.synchronize()
+    assert int(flagged[0]) == -1
+    good = blk.offsets.clone()
+    backwards = good.clone()
+    backwards[5] = backwards[4] - 1
+    past_end = good.clone()
+    past_end[w.E + 1] = cfg.rows + 128
+    for off in (flagged, backwards, past_end):
+        moe.expert_up(cfg, blk.weights, off, blk.sorted, blk.ws)
+        torch.cuda.synchronize()
+        assert moe.device_error(blk.ws) == 5
+        moe.expert_down(cfg, blk.weights, blk.gate, off, blk.sorted, blk.ws)
+        torch.cuda.synchronize()
+        assert moe.device_error(blk.ws) == 5
+    res = case.run()
+    assert res["err"] == 0
+    MH.check_forward(case, res, np.arange(w.T))
+
+
+@pytest.mark.parametrize("T", [5, 300, 9600])  # split-K paths (5, 300) and one CTA per 128 tokens (9600)
+def test_route_fp32_and_packed_router_agree_bit_exact(T):
+    """moe_route (fp32 W_r, split into the workspace on every call) and
+    moe_pack_router + moe_route_packed run the same router kernel on the same
+    split: selections, gates, margins and logits are identical."""
+    w = W.WORKLOADS["glm47flash"].replace(T=T, seed=3300 + T)
+    cfg = moe.Config.of(w)
+    x, w_r, b = W.router_inputs(w)
+    x_dev = MH.to_dev_bf16(x)
+    w_r, b = torch.from_numpy(w_r).cuda(), torch.from_numpy(b).cuda()
+    ws = moe.workspace(cfg)
+    z1 = torch.empty((T, w.E), dtype=torch.float32, device="cuda")
+    z2 = torch.empty_like(z1)
+    r1 = moe.route(cfg, x_dev, w_r, b, ws, logits=z1)
+    r1 = [t.clone() for t in r1]
+    packed = moe.pack_router(cfg, w_r)
+    r2 = moe.route_packed(cfg, x_dev, packed, b, ws, logits=z2)
+    torch.cuda.synchronize()
+    assert moe.device_error(ws) == 0
+    for a, bb in zip(r1, r2):
+        assert torch.equal(a, bb)
+    assert torch.equal(z1, z2)
+    case = MH.Case(w, x=x, w_r=w_r.cpu().numpy(), b=b.cpu().numpy(), weights={})
+    res = dict(idx=r2[0].cpu().numpy(), gate=r2[1].cpu().numpy(), margin=r2[2].cpu().numpy(),
+               logits=z2.cpu().numpy())
+    tok = np.arange(T) if T <= 512 else np.random.default_rng(T).choice(T, 512, replace=False)
+    MH.check_route(case, res, tok)
+
+
+def test_pack_reports_w2_values_fp16_cannot_hold():
+    """moe_pack_weights stores W2 as fp16.  bf16 weights beyond +-65504 saturate
+    and ones finer than fp16's 2^-24 spacing are rounded; the call counts them.
+    The expected count is the host's own bf16 -> fp16 -> float round trip of
+    every routed and shared W2 value; planted 1e5 (saturates), 1e-8 (rounds to
+    0) and 3 * 2^-26 (between fp16 subnormals) must each add one, while 2^-20
+    (a multiple of 2^-24) must not."""
+    w = W.WORKLOADS["tiny"]
+    cfg = moe.Config.of(w)
+    wts = W.expert_weights(w, "cuda")
+
+    def host_count(w2, ws2):
+        a = torch.cat([w2.reshape(-1), ws2.reshape(-1)]).float().cpu()
+        return int((a.half().float() != a).sum())
+
+    n = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    moe.pack_weights(cfg, wts["w1"], wts["w3"], wts["w2"], wts["ws1"], wts["ws3"], wts["ws2"], inexact=n)
+    torch.cuda.synchronize()
+    base = host_count(wts["w2"], wts["ws2"])
+    assert int(n) == base
+    w2, ws2 = wts["w2"].clone(), wts["ws2"].clone()
+    w2[3, 17, 5] = 1e5
+    w2[0, 0, 0] = 1e-8
+    ws2[9, 100] = 3 * 2.0 ** -26
+    w2[5, 2, 64] = 2.0 ** -20
+    expect = host_count(w2, ws2)
+    planted = torch.tensor([1e5, 1e-8, 3 * 2.0 ** -26, 2.0 ** -20], dtype=torch.bfloat16).float()
+    assert (planted.half().float() != planted).tolist() == [True, True, True, False]
+    w13, w2p = moe.pack_weights(cfg, wts["w1"], wts["w3"], w2, wts["ws1"], wts["ws3"], ws2, inexact=n)
+    torch.cuda.synchronize()
+    assert int(n) == expect
+    assert float(w2p[3 * w.H + 17, 5]) == 65504.0 and float(w2p[0, 0]) == 0.0
+    assert float(w2p[5 * w.H + 2, 64]) == 2.0 ** -20
+
+
 def test_timeout_is_reported_and_context_survives(monkeypatch):
     """Failure detection without a GPU fault: with SRM_MOE_INJECT_STALL=1 the up
     projection's producer issues no loads, so the MMA warp waits on a barrier

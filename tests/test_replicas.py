@@ -111,14 +111,14 @@ def test_tensor_peak_follows_the_timed_loop_length():
 
 
 def test_launches_per_step_match_the_kernel_structure():
-    """The bench's gpu_launches claim: decode runs W_r split, split-K logits,
-    their reduction, selection, the one-CTA permutation, invert, gather, up,
-    down, combine (10 kernels, as the ncu launch list shows); prefill runs the
-    router without split-K and the three-kernel permutation (11)."""
+    """The bench's gpu_launches claim: one router kernel (logits, selection and
+    gates; the router weights are split once at pack time), the one-CTA
+    permutation for small batches or histogram + scan + scatter, invert,
+    gather, up, down, combine: 7 kernels at decode, 9 at prefill."""
     sys.path.insert(0, ROOT)
     import bench
     from sigmoid_routed_mixture_b200 import workloads as W
 
-    assert bench.kernels_per_step(W.WORKLOADS["glm5_decode"]) == 10
-    assert bench.kernels_per_step(W.WORKLOADS["glm5_prefill"]) == 11
+    assert bench.kernels_per_step(W.WORKLOADS["glm5_decode"]) == 7
+    assert bench.kernels_per_step(W.WORKLOADS["glm5_prefill"]) == 9
     assert bench.DSA_KERNELS_PER_STEP == 3  # plan, scores, top-k

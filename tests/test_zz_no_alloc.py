@@ -37,7 +37,11 @@ def call_noalloc(cfg, idx, counts, offsets, sorted_):
 
 @pytest.mark.parametrize("has_shared", [True, False])
 def test_noalloc_matches_workspace_permute_on_two_calls(has_shared):
-    for T, E, K, seed in [(32768, 256, 8, 11), (1000, 64, 4, 12)]:
+    # both calls above 16384 assignments, so both take the chunked path whose
+    # per-chunk counts live in the static array; the second has fewer chunks and
+    # another expert count, so leftovers of the first would show; the third is
+    # the one-CTA path for small batches
+    for T, E, K, seed in [(32768, 256, 8, 11), (3000, 64, 8, 12), (1000, 64, 4, 14)]:
         cfg = moe.Config(T=T, H=256, I=128, E=E, K=K, has_shared=has_shared)
         idx = topk_ids(T, E, K, seed)
         ref = moe.permute(cfg, idx, moe.workspace(cfg))
@@ -51,19 +55,20 @@ def test_noalloc_matches_workspace_permute_on_two_calls(has_shared):
         assert int(out[1][0]) == 0
 
 
-def test_noalloc_limits_and_bad_ids():
+@pytest.mark.parametrize("T,E,K", [(300, 16, 4), (3000, 64, 8)])  # one-CTA path, chunked path
+def test_noalloc_limits_and_bad_ids(T, E, K):
     L = moe.lib()
     big = moe.Config(T=262144 // 8 + 1, H=256, I=128, E=256, K=8)
     assert L.moe_permute_noalloc(ctypes.byref(big.c()), None, None, None, None, None) == 2
-    cfg = moe.Config(T=300, H=256, I=128, E=16, K=4)
-    idx = topk_ids(300, 16, 4, 13)
-    idx[5, 1] = 99  # out of range: skipped and flagged in offsets[0]
+    cfg = moe.Config(T=T, H=256, I=128, E=E, K=K)
+    idx = topk_ids(T, E, K, 13)
+    idx[5, 1] = 999  # out of range: skipped and flagged in offsets[0]
     counts, offsets, sorted_ = moe.permute_noalloc(cfg, idx)
     torch.cuda.synchronize()
     assert int(offsets[0]) == -1
-    idx[5, 1] = next(v for v in range(16) if v not in idx[5].tolist())
+    idx[5, 1] = next(v for v in range(E) if v not in idx[5].tolist())
     counts, offsets, sorted_ = moe.permute_noalloc(cfg, idx)  # the next call starts clean
     ref = moe.permute(cfg, idx, moe.workspace(cfg))
     torch.cuda.synchronize()
-    assert torch.equal(offsets, ref[1]) and torch.equal(sorted_, ref[2])
+    assert torch.equal(counts, ref[0]) and torch.equal(offsets, ref[1]) and torch.equal(sorted_, ref[2])
     assert np.all(np.diff(offsets.cpu().numpy()) >= 0)

@@ -183,9 +183,11 @@ moe_status_t moe_route_packed(const moe_cfg_t *cfg, const void *x, const void *w
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int e_pad = srm::router_e_pad(cfg->E);
+  const bool pair = srm::router_use_pairs(static_cast<int>(cfg->T), cfg->H, num_sms());
   CUtensorMap tm_x, tm_w;
   if (!make_tmap(&tm_x, x, cfg->H, static_cast<uint64_t>(cfg->T), 64, 128) ||
-      !make_tmap(&tm_w, w_router_packed, cfg->H, 3ull * e_pad, 64, static_cast<uint32_t>(e_pad)))
+      !make_tmap(&tm_w, w_router_packed, cfg->H, 3ull * e_pad, 64,
+                 static_cast<uint32_t>(srm::router_w_box_rows(cfg->E, pair))))
     return MOE_ERR_CUDA;
   int *grid_counter = reinterpret_cast<int *>(wsb + L.err + 64);
   if (cudaMemsetAsync(grid_counter, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;

@@ -46,11 +46,14 @@ cudaError_t launch_grouped_gemm(int mode, bool pair, const CUtensorMap &tmap_tok
 
 // router: W_r split into bf16 parts [3][e_pad][H] (wsplit), fp32 partial logits
 // zp [splits][T][e_pad] (split-K only); tmap_x: x [T][H] box 64 x 128,
-// tmap_w: wsplit [3*e_pad][H] box 64 x e_pad; grid_counter: an int zeroed
+// tmap_w: wsplit [3*e_pad][H] box 64 x router_w_box_rows; grid_counter: an int zeroed
 // before the launch (split-K grid barrier)
 int router_e_pad(int E);
 int router_splits(int T, int H);  // upper bound of the split count (workspace sizing)
 int router_grid_splits(int T, int H, int num_sms);
+// without a split, CTA pairs: tmap_w's box is then e_pad / 2 rows (router_w_box_rows)
+bool router_use_pairs(int T, int H, int num_sms);
+int router_w_box_rows(int E, bool pair);
 cudaError_t launch_router_split(const float *w_r, int E, int H, uint16_t *wsplit, int num_sms,
                                 cudaStream_t stream);
 cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, const float *bias, int T,

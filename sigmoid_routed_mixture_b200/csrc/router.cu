@@ -54,7 +54,7 @@ int router_e_pad(int E) { return (E + 63) / 64 * 64; }
 int router_stage_bytes(int e_pad) { return rt::A_BYTES + 3 * e_pad * rt::BK * 2; }
 
 struct RouterSmem;
-int router_stages(int e_pad);
+int router_stages(int e_pad, bool pair);
 
 int router_splits(int T, int H) {
   const int m_tiles = (T + rt::BM - 1) / rt::BM;
@@ -237,31 +237,39 @@ __device__ __forceinline__ bool grid_barrier(int *counter, int n_ctas, int *err)
 
 // NH = e_pad / 64: each epilogue thread keeps half a row (e_pad / 2 columns).
 // kSplit: the H range is split over gridDim.y CTAs (partials + grid barrier).
-template <int NH, bool kSplit>
+// kPair (large T, no split): clusters of two CTAs run tcgen05.mma.cta_group::2
+// with M = 256 tokens; each CTA loads its 128 token rows and half of every
+// part's expert rows, so each byte of the split W_r crosses L2 once per 256
+// tokens instead of once per 128, and a stage is small enough for 3 of them.
+template <int NH, bool kSplit, bool kPair>
 __global__ void __launch_bounds__(rt::THREADS, 1)
     router_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                   int kb_per_split, int kblocks, int stages, uint32_t tmem_cols,
                   float *__restrict__ zp, int *grid_counter, RouteOut o, int *err) {
+  static_assert(!(kSplit && kPair), "the split-K router runs on single CTAs");
   using namespace rt;
   constexpr int e_pad = NH * 64;
   constexpr int HALF = e_pad / 2;
   constexpr int NE = e_pad / 32;         // experts per lane in the selection
   constexpr int ZS = e_pad + 4;          // shared-memory row stride of staged z (floats)
+  constexpr int W_ROWS = kPair ? e_pad / 2 : e_pad;  // expert rows of each part this CTA loads
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   uint8_t *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  constexpr int stage_bytes = A_BYTES + 3 * e_pad * BK * 2;
+  constexpr int stage_bytes = A_BYTES + 3 * W_ROWS * BK * 2;
   RouterSmem &s = *reinterpret_cast<RouterSmem *>(base + stages * stage_bytes);
   float *zs = reinterpret_cast<float *>(base);  // staged z rows, over the drained ring
 
   const int T = o.T;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * BM;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0;
+  const bool leader = rank == 0;
+  const int m0 = blockIdx.x * BM;  // a pair's two CTAs are x = 2p, 2p + 1: tokens 256p, 256p + 128
   const int split = blockIdx.y;
   const int kb0 = split * kb_per_split;
   const int kb1 = min(kblocks, kb0 + kb_per_split);
   const int nchunks = (kb1 - kb0 + CHUNK - 1) / CHUNK;
-  constexpr uint32_t part_bytes = static_cast<uint32_t>(e_pad) * BK * 2;
+  constexpr uint32_t part_bytes = static_cast<uint32_t>(W_ROWS) * BK * 2;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < stages; ++i) {
@@ -270,7 +278,7 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.tfull[i], 1);
-      mbar_init(&s.tempty[i], EPI_WARPS);
+      mbar_init(&s.tempty[i], (kPair ? 2 : 1) * EPI_WARPS);
     }
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
@@ -280,11 +288,19 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
     tma_prefetch_desc(&tmap_w);
   }
   if (warp == 1) {
-    tmem_alloc(&s.tmem_base, tmem_cols);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(&s.tmem_base, tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&s.tmem_base, tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (kPair)
+    cluster_sync();  // the peer's barriers are initialised before any remote use
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   volatile int *abort_flag = &s.abort_flag;
@@ -297,11 +313,21 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
       if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, err)) break;
       if (lane == 0) {
         uint8_t *st = base + stage * stage_bytes;
-        mbar_arrive_expect_tx(&s.full[stage], stage_bytes);
-        tma_load_2d(st, &tmap_x, &s.full[stage], kb * BK, m0);
-        for (int part = 0; part < 3; ++part)
-          tma_load_2d(st + A_BYTES + part * part_bytes, &tmap_w, &s.full[stage], kb * BK,
-                      part * e_pad);
+        if (kPair) {
+          // both CTAs' copies complete on the leader's barrier
+          if (leader) mbar_arrive_expect_tx(&s.full[stage], 2 * stage_bytes);
+          const uint32_t full_leader = cluster_map(&s.full[stage], 0);
+          tma_load_2d_pair(st, &tmap_x, full_leader, kb * BK, m0);
+          for (int part = 0; part < 3; ++part)
+            tma_load_2d_pair(st + A_BYTES + part * part_bytes, &tmap_w, full_leader, kb * BK,
+                             part * e_pad + static_cast<int>(rank) * W_ROWS);
+        } else {
+          mbar_arrive_expect_tx(&s.full[stage], stage_bytes);
+          tma_load_2d(st, &tmap_x, &s.full[stage], kb * BK, m0);
+          for (int part = 0; part < 3; ++part)
+            tma_load_2d(st + A_BYTES + part * part_bytes, &tmap_w, &s.full[stage], kb * BK,
+                        part * e_pad);
+        }
       }
       __syncwarp();
       ++issued;
@@ -311,8 +337,11 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    const uint32_t idesc = umma_idesc_f32acc(BM, e_pad, 1u);
+    // ---------------------------------------------------------- MMA issuer (the leader of a pair)
+    if (kPair && !leader) {
+      // nothing to issue: the leader's MMAs read this CTA's shared memory
+    } else {
+    const uint32_t idesc = umma_idesc_f32acc(kPair ? 2 * BM : BM, e_pad, 1u);
     uint32_t stage = 0, phase = 0;
     int consumed = 0;
     bool ok = true;
@@ -335,11 +364,20 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
           for (int part = 0; part < 3; ++part) {
             const uint32_t b_addr = a_addr + A_BYTES + part * part_bytes;
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k)
-              umma_bf16(d, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), idesc,
-                        (kb > ka || part > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k) {
+              const uint32_t accum = (kb > ka || part > 0 || k > 0) ? 1u : 0u;
+              if (kPair)
+                umma_pair(d, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), idesc,
+                          accum);
+              else
+                umma_bf16(d, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), idesc,
+                          accum);
+            }
           }
-          umma_commit(&s.empty[stage]);
+          if (kPair)
+            umma_commit_pair(&s.empty[stage], 0x3);
+          else
+            umma_commit(&s.empty[stage]);
         }
         __syncwarp();
         if (++stage == static_cast<uint32_t>(stages)) {
@@ -347,10 +385,16 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
           phase ^= 1u;
         }
       }
-      if (ok && lane == 0) umma_commit(&s.tfull[slot]);
+      if (ok && lane == 0) {
+        if (kPair)
+          umma_commit_pair(&s.tfull[slot], 0x3);
+        else
+          umma_commit(&s.tfull[slot]);
+      }
       __syncwarp();
     }
     if (lane == 0) s.mma_consumed = consumed;
+    }
   } else {
     // ---------------------------------------------------------- epilogue
     // warps 2..9: lane quarter q = warp % 4 (the TMEM lanes this warp may
@@ -382,7 +426,12 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.tempty[slot]);
+      if (lane == 0) {
+        if (!kPair || leader)
+          mbar_arrive(&s.tempty[slot]);
+        else
+          mbar_arrive_remote(cluster_map(&s.tempty[slot], 0));
+      }
     }
     if (kSplit) {
       if (ok && t < T) {
@@ -420,16 +469,25 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
   __syncthreads();
   if (s.abort_flag) {  // error path: let copies and MMAs in flight land first
     if (warp == 0 && lane == 0) {
-      for (int i = s.mma_consumed; i < issued; ++i) {
-        const uint32_t a = smem_addr(&s.full[i % stages]);
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(a, static_cast<uint32_t>((i / stages) & 1)) &&
-               global_timer_ns() - t0 < kWaitLimitNs) {
+      const uint64_t t0 = global_timer_ns();
+      if (leader) {
+        // (a pair's leader barriers count both CTAs' copies)
+        for (int i = s.mma_consumed; i < issued; ++i) {
+          const uint32_t a = smem_addr(&s.full[i % stages]);
+          while (!mbar_try_wait(a, static_cast<uint32_t>((i / stages) & 1)) &&
+                 global_timer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      } else {  // the peer gives its own copies a bounded time to land
+        while (global_timer_ns() - t0 < 1000000ull) {
         }
       }
     }
-    if (warp == 1 && lane == 0) {
-      umma_commit(&s.drain);
+    if (warp == 1 && lane == 0 && leader) {
+      if (kPair)
+        umma_commit_pair(&s.drain, 0x1);
+      else
+        umma_commit(&s.drain);
       const uint32_t a = smem_addr(&s.drain);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(a, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
@@ -438,9 +496,13 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (kPair) cluster_sync();  // neither CTA leaves while the other may touch its shared memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, tmem_cols);
+    if (kPair)
+      tmem_dealloc_pair(tmem, tmem_cols);
+    else
+      tmem_dealloc(tmem, tmem_cols);
   }
 
   if (kSplit) {
@@ -481,33 +543,51 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
   }
 }
 
-int router_stages(int e_pad) {
-  int s = static_cast<int>((rt::MAX_SMEM - 1024 - sizeof(RouterSmem)) / router_stage_bytes(e_pad));
+int router_stages(int e_pad, bool pair = false) {
+  const int stage = rt::A_BYTES + 3 * (pair ? e_pad / 2 : e_pad) * rt::BK * 2;
+  int s = static_cast<int>((rt::MAX_SMEM - 1024 - sizeof(RouterSmem)) / stage);
   return s > 4 ? 4 : s;
 }
 
 // ---------------------------------------------------------------- launch
 
-size_t router_smem_bytes(int e_pad) {
-  return 1024 + static_cast<size_t>(router_stages(e_pad)) * router_stage_bytes(e_pad) +
-         sizeof(RouterSmem);
+size_t router_smem_bytes(int e_pad, bool pair) {
+  const int stage = rt::A_BYTES + 3 * (pair ? e_pad / 2 : e_pad) * rt::BK * 2;
+  return 1024 + static_cast<size_t>(router_stages(e_pad, pair)) * stage + sizeof(RouterSmem);
 }
 
-template <int NH, bool kSplit>
+
+template <int NH, bool kSplit, bool kPair>
 static cudaError_t launch_router_kernel(dim3 grid, const CUtensorMap &tmap_x, const CUtensorMap &tmap_w,
                                         int kb_per, int kblocks, float *zp, int *grid_counter,
                                         const RouteOut &o, int *err, cudaStream_t stream) {
   constexpr int e_pad = NH * 64;
-  const size_t smem = router_smem_bytes(e_pad);
-  const int stages = router_stages(e_pad);
+  const size_t smem = router_smem_bytes(e_pad, kPair);
+  const int stages = router_stages(e_pad, kPair);
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(2 * e_pad)) cols <<= 1;  // two ping-pong accumulators
-  cudaError_t e = cudaFuncSetAttribute(router_kernel<NH, kSplit>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = router_kernel<NH, kSplit, kPair>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  router_kernel<NH, kSplit><<<grid, rt::THREADS, smem, stream>>>(tmap_x, tmap_w, kb_per, kblocks, stages,
-                                                                 cols, zp, grid_counter, o, err);
-  return cudaGetLastError();
+  if (!kPair) {
+    kern<<<grid, rt::THREADS, smem, stream>>>(tmap_x, tmap_w, kb_per, kblocks, stages, cols, zp,
+                                              grid_counter, o, err);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(rt::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmap_x, tmap_w, kb_per, kblocks, stages, cols, zp, grid_counter,
+                            o, err);
 }
 
 cudaError_t launch_router_split(const float *w_r, int E, int H, uint16_t *wsplit, int num_sms,
@@ -527,6 +607,10 @@ int router_grid_splits(int T, int H, int num_sms) {
   return (kblocks + kb_per - 1) / kb_per;  // splits that get at least one k-block
 }
 
+int router_w_box_rows(int E, bool pair) { return pair ? router_e_pad(E) / 2 : router_e_pad(E); }
+
+bool router_use_pairs(int T, int H, int num_sms) { return router_grid_splits(T, H, num_sms) == 1; }
+
 cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, const float *bias, int T,
                          int H, int E, int K, float scale, float *zp, int *grid_counter,
                          int32_t *idx, float *gate, float *margin, float *logits, int *err,
@@ -534,7 +618,9 @@ cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, c
   const int kblocks = H / rt::BK;
   const int splits = router_grid_splits(T, H, num_sms);
   const int kb_per = (kblocks + splits - 1) / splits;
-  dim3 grid((T + rt::BM - 1) / rt::BM, splits);
+  const bool pair = splits == 1;  // must match router_use_pairs (the tensor map's box)
+  const int m_tiles = (T + rt::BM - 1) / rt::BM;
+  dim3 grid(pair ? (m_tiles + 1) / 2 * 2 : m_tiles, splits);
   RouteOut o;
   o.bias = bias;
   o.idx = idx;
@@ -546,20 +632,22 @@ cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, c
   o.E = E;
   o.K = K;
   const int nh = router_e_pad(E) / 64;
+#define SRM_ROUTER_CASES(SPLIT, PAIR)                                                                       \
+  switch (nh) {                                                                                            \
+    case 1: return launch_router_kernel<1, SPLIT, PAIR>(grid, tmap_x, tmap_w, kb_per, kblocks, zp,         \
+                                                        grid_counter, o, err, stream);                     \
+    case 2: return launch_router_kernel<2, SPLIT, PAIR>(grid, tmap_x, tmap_w, kb_per, kblocks, zp,         \
+                                                        grid_counter, o, err, stream);                     \
+    case 3: return launch_router_kernel<3, SPLIT, PAIR>(grid, tmap_x, tmap_w, kb_per, kblocks, zp,         \
+                                                        grid_counter, o, err, stream);                     \
+    default: return launch_router_kernel<4, SPLIT, PAIR>(grid, tmap_x, tmap_w, kb_per, kblocks, zp,        \
+                                                         grid_counter, o, err, stream);                    \
+  }
   if (splits > 1) {
-    switch (nh) {
-      case 1: return launch_router_kernel<1, true>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
-      case 2: return launch_router_kernel<2, true>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
-      case 3: return launch_router_kernel<3, true>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
-      default: return launch_router_kernel<4, true>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
-    }
+    SRM_ROUTER_CASES(true, false)
   }
-  switch (nh) {
-    case 1: return launch_router_kernel<1, false>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
-    case 2: return launch_router_kernel<2, false>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
-    case 3: return launch_router_kernel<3, false>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
-    default: return launch_router_kernel<4, false>(grid, tmap_x, tmap_w, kb_per, kblocks, zp, grid_counter, o, err, stream);
-  }
+  SRM_ROUTER_CASES(false, true)
+#undef SRM_ROUTER_CASES
 }
 
 }  // namespace srm

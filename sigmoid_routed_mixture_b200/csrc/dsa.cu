@@ -568,15 +568,20 @@ __global__ void __launch_bounds__(NT)
     prefix |= static_cast<uint32_t>(digit) << shift;
     pmask |= 255u << shift;
     __syncthreads();
+    // every key of the chosen bin is taken: the keys to keep are exactly those
+    // whose bits so far are >= prefix, and no lower digit is needed (the same
+    // value for the whole CTA, so the exit is uniform)
+    if (n_eq == k_rem) break;
   }
-  // prefix is the n_sel-th largest key: take every key above it and the first
-  // k_rem of the n_eq keys equal to it (lowest indices), listed by index
+  // (v & pmask) vs prefix orders the keys by the digits decided so far (all 32
+  // bits unless the passes stopped early).  Take every key above prefix and the
+  // first k_rem of the n_eq keys equal to it (lowest indices), listed by index
   const unsigned lt = (1u << lane) - 1u;
   uint64_t eq_take = ~uint64_t(0);  // bit j: this thread's key j, if equal, is taken
   if (n_eq > k_rem) {  // ties across the threshold: rank the equal keys by index
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && v[j] == prefix);
+      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && (v[j] & pmask) == prefix);
       if (lane == 0) cnt[j * NW + warp] = __popc(m);
     }
     __syncthreads();
@@ -585,7 +590,7 @@ __global__ void __launch_bounds__(NT)
     eq_take = 0;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && v[j] == prefix);
+      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && (v[j] & pmask) == prefix);
       if (cnt[j * NW + warp] + __popc(m & lt) < k_rem) eq_take |= uint64_t(1) << j;
     }
     __syncthreads();
@@ -593,7 +598,8 @@ __global__ void __launch_bounds__(NT)
   uint64_t take_bits = 0;
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
-    const bool take = j * NT + tid < n_vis && (v[j] > prefix || (v[j] == prefix && ((eq_take >> j) & 1u)));
+    const uint32_t vm = v[j] & pmask;
+    const bool take = j * NT + tid < n_vis && (vm > prefix || (vm == prefix && ((eq_take >> j) & 1u)));
     const unsigned m = __ballot_sync(0xffffffffu, take);
     if (take) take_bits |= uint64_t(1) << j;
     if (lane == 0) cnt[j * NW + warp] = __popc(m);

@@ -27,7 +27,8 @@
  *     on a non-OK status nothing was launched.  Problems only the device can
  *     see (a corrupt expert id, a pipeline wait that ran out) are recorded in
  *     the workspace's error word and read by moe_get_device_error; outputs of
- *     such a call are unspecified.  No kernel traps or asserts.
+ *     such a call are unspecified.  The first error is kept until read, so one
+ *     read after a step covers all of its calls.  No kernel traps or asserts.
  *   - Supported shapes: 1 <= K <= E <= 256, K <= 16, H % 256 == 0,
  *     I % 128 == 0, T >= 0 (T == 0 is a no-op), T * (K + 1) < 2^31.
  *     Pointers that feed the tensor-memory-access engine (x, packed weights,
@@ -85,7 +86,11 @@ typedef struct {
 } moe_weights_t;
 
 /* Bytes of device workspace moe_route, moe_permute and moe_forward need for
- * `cfg` (one buffer serves all three).  Returns 0 for an invalid cfg. */
+ * `cfg` (one buffer serves all three).  Returns 0 for an invalid cfg.
+ * The first 256 bytes of a workspace hold the device error word and other
+ * control words: zero them once when the workspace is allocated (e.g.
+ * cudaMemset); from then on the library keeps them (a device-side error stays
+ * recorded until moe_get_device_error reads and clears it). */
 size_t moe_workspace_size(const moe_cfg_t *cfg);
 
 /* Staging buffers inside a workspace, for moe_workspace_offset. */

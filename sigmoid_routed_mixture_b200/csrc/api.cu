@@ -224,7 +224,6 @@ moe_status_t moe_permute(const moe_cfg_t *cfg, const int32_t *topk_idx, int32_t 
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t *wsb = static_cast<uint8_t *>(ws);
-  if (cudaMemsetAsync(wsb + L.err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   if (cfg->T == 0) {
     if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * (cfg->E + 1), s) != cudaSuccess ||
         cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (cfg->E + 2), s) != cudaSuccess)
@@ -420,8 +419,7 @@ moe_status_t moe_dense_mlp(const moe_cfg_t *cfg, const moe_weights_t *weights, c
   // one group holding every token in order: offsets {0, T}, sorted = identity
   int32_t *offsets = reinterpret_cast<int32_t *>(wsb + L.err + 192);
   int32_t *sorted = reinterpret_cast<int32_t *>(wsb + L.pos);
-  if (cudaMemsetAsync(wsb + L.err, 0, sizeof(int32_t), s) != cudaSuccess ||
-      srm::launch_identity_rows(offsets, sorted, T, num_sms(), s) != cudaSuccess)
+  if (srm::launch_identity_rows(offsets, sorted, T, num_sms(), s) != cudaSuccess)
     return MOE_ERR_CUDA;
   const bool pair = cfg->T >= 512;
   CUtensorMap tm_x, tm_w13, tm_h, tm_w2;

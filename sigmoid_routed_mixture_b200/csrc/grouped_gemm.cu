@@ -424,62 +424,69 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
       if (tile < 0) break;
       const TileCoord c = decode_tile<kPair>(s, groups, n_tiles, m_chunk, tile);
       const int wr = c.w0 + static_cast<int>(rank) * BM + q * 32;  // this warp's first weight row
+      constexpr int CHUNKS = BT / 32;
+      // kDown: each token's destination row and gate, lane holding tokens
+      // lane + 32m.  They do not depend on the accumulator, so they are read
+      // while the tile's MMAs still run.
+      int my_a[CHUNKS];
+      float my_g[CHUNKS];
+      if (kMode == kDown) {
+#pragma unroll
+        for (int m = 0; m < CHUNKS; ++m)
+          my_a[m] = 32 * m + lane < c.rows ? p.sorted[c.row_base + 32 * m + lane] : -1;
+#pragma unroll
+        for (int m = 0; m < CHUNKS; ++m) {
+          my_g[m] = 0.f;
+          if (32 * m + lane < c.rows) {
+            if (my_a[m] < 0 || my_a[m] >= p.n_rows_y) {
+              record_error(p.err, MOE_ERR_BAD_INDEX);
+              my_a[m] = -1;
+            } else {
+              my_g[m] = my_a[m] < p.tk ? p.gate[my_a[m]] : 1.0f;
+            }
+          }
+        }
+      }
       if (!mbar_wait(&s.tfull[acc], acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + acc * BT + (static_cast<uint32_t>(q * 32) << 16);
       bool sat = false;
-      if (kMode == kUp) {
-        // lanes 0-15 hold gate rows of features j0 .. j0+15, lanes 16-31 the
-        // matching up rows (the 32-row packing unit); after one exchange lane l
-        // has (g, u) of feature j0 + (l % 16) for tokens half*16 .. half*16+15
-        // of each 32-token chunk, half = l / 16
-        const int half = lane >> 4;
-        const int j = wr / 2 + (lane & 15);
-        __half *h = reinterpret_cast<__half *>(p.out);
-#pragma unroll 1
-        for (int c0 = 0; c0 < c.n; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(taddr + c0, v);
-          tmem_ld_wait();
+      // 32-token chunks (each read from tensor memory and waited for before use)
+#pragma unroll
+      for (int m = 0; m < CHUNKS; ++m) {
+        if (32 * m >= c.n) break;  // uniform across the warp
+        uint32_t cv[32];
+        tmem_ld32(taddr + 32 * m, cv);
+        tmem_ld_wait();
+        if (kMode == kUp) {
+          // lanes 0-15 hold gate rows of features j0 .. j0+15, lanes 16-31 the
+          // matching up rows (the 32-row packing unit); after one exchange lane
+          // l has (g, u) of feature j0 + (l % 16) for tokens half*16 ..
+          // half*16+15 of the chunk, half = l / 16
+          const int half = lane >> 4;
+          const int jf = wr / 2 + (lane & 15);
+          __half *h = reinterpret_cast<__half *>(p.out);
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
-            const float mine = __uint_as_float(v[half ? k + 16 : k]);
-            const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(v[half ? k : k + 16]), 16);
+            const float mine = __uint_as_float(cv[half ? k + 16 : k]);
+            const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(cv[half ? k : k + 16]), 16);
             const float g = half ? other : mine;
             const float u = half ? mine : other;
-            const int t = c0 + half * 16 + k;
+            const int t = 32 * m + half * 16 + k;
             if (t < c.rows)
-              h[static_cast<size_t>(c.row_base + t) * p.out_ld + j] =
+              h[static_cast<size_t>(c.row_base + t) * p.out_ld + jf] =
                   __ushort_as_half(f16_sat(g * sigmoidf_(g) * u, sat));
           }
-        }
-      } else {
-        // lane = output feature f; the tokens' destinations and gates are
-        // loaded one per lane per 32-token chunk and broadcast by shuffles
-        const int f = wr + lane;
-        __half *y = reinterpret_cast<__half *>(p.out);
-#pragma unroll 1
-        for (int c0 = 0; c0 < c.n; c0 += 32) {
-          int my_a = -1;
-          float my_g = 0.f;
-          if (c0 + lane < c.rows) {
-            const int a = p.sorted[c.row_base + c0 + lane];
-            if (a < 0 || a >= p.n_rows_y) {
-              record_error(p.err, MOE_ERR_BAD_INDEX);
-            } else {
-              my_a = a;
-              my_g = a < p.tk ? p.gate[a] : 1.0f;
-            }
-          }
-          uint32_t v[32];
-          tmem_ld32(taddr + c0, v);
-          tmem_ld_wait();
+        } else {
+          // lane = output feature f; destinations and gates broadcast by shuffles
+          const int f = wr + lane;
+          __half *y = reinterpret_cast<__half *>(p.out);
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            const int a = __shfl_sync(0xffffffffu, my_a, k);
-            const float gv = __shfl_sync(0xffffffffu, my_g, k);
+            const int a = __shfl_sync(0xffffffffu, my_a[m], k);
+            const float gv = __shfl_sync(0xffffffffu, my_g[m], k);
             if (a >= 0)
-              y[static_cast<size_t>(a) * p.out_ld + f] = __ushort_as_half(f16_sat(gv * __uint_as_float(v[k]), sat));
+              y[static_cast<size_t>(a) * p.out_ld + f] = __ushort_as_half(f16_sat(gv * __uint_as_float(cv[k]), sat));
           }
         }
       }

@@ -34,6 +34,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -139,13 +141,14 @@ struct RouteOut {
   int T, E, K;
 };
 
-// Selection for one token by one warp from its E logits zrow[e] (shared or
-// global memory, e < E read): s = sigmoid(z), key = s + b, K rounds of a warp
+// Selection for one token by one warp from its E logits (a row zrow[e] in
+// shared memory, or each lane's own z[j] = z[lane + 32j] in registers; e < E
+// read): s = sigmoid(z), key = s + b, K rounds of a warp
 // arg-max (key descending, equal keys to the lower index), one more round for
 // the margin; gates = scale * s / sum of the selected s.  bias_r[j] holds
 // bias[lane + 32 j] (this lane's experts).
-template <int NE>
-__device__ __forceinline__ void select_token(const float *zrow, const float (&bias_r)[NE], int t,
+template <int NE, typename Src>
+__device__ __forceinline__ void select_token(const Src &zsrc, const float (&bias_r)[NE], int t,
                                              const RouteOut &o, int lane) {
   float key[NE], sv[NE];
 #pragma unroll
@@ -153,7 +156,11 @@ __device__ __forceinline__ void select_token(const float *zrow, const float (&bi
     const int e = lane + 32 * j;
     float z = 0.f;
     if (e < o.E) {
-      z = zrow[e];
+      // a row in memory (pointer) or this lane's own values in registers (array)
+      if constexpr (std::is_pointer<Src>::value)
+        z = zsrc[lane + 32 * j];
+      else
+        z = zsrc[j];
       if (o.logits) o.logits[static_cast<size_t>(t) * o.E + e] = z;
     }
     const float sj = sigmoidf_(z);
@@ -461,7 +468,7 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
           bias_r[j] = e < o.E ? o.bias[e] : 0.f;
         }
         for (int r = warp - 2; r < BM && m0 + r < T; r += EPI_WARPS)
-          select_token<NE>(zs + r * ZS, bias_r, m0 + r, o, lane);
+          select_token<NE>(static_cast<const float *>(zs + r * ZS), bias_r, m0 + r, o, lane);
       }
     }
   }
@@ -506,15 +513,14 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
   }
 
   if (kSplit) {
-    // Every CTA's partials are written; after the grid barrier each CTA takes
-    // tokens t = cta, cta + n_ctas, ...: warp j sums the S partials of experts
-    // 32j .. 32j+31 in split order (eight interleaved accumulators combined in
-    // a fixed tree: deterministic, whichever CTA does it), stages z in shared
-    // memory, and one warp selects.
-    const int n_ctas = gridDim.x * gridDim.y;
-    const int cta = blockIdx.y * gridDim.x + blockIdx.x;
+    // Every CTA's partials are written; after the grid barrier each warp of
+    // the grid takes tokens t = w, w + W, ... (W = warps in the grid): its
+    // lanes sum the S partials of experts lane + 32j in split order, four
+    // splits at a time ((p0 + p1) + (p2 + p3), then into the running sum: a
+    // fixed order, deterministic whichever warp does it), and the warp selects
+    // from the sums held in its registers.  No barrier between tokens.
     const int splits = gridDim.y;
-    if (!grid_barrier(grid_counter, n_ctas, err)) return;
+    if (!grid_barrier(grid_counter, gridDim.x * gridDim.y, err)) return;
     float bias_r[NE];
 #pragma unroll
     for (int j = 0; j < NE; ++j) {
@@ -522,23 +528,29 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
       bias_r[j] = e < o.E ? o.bias[e] : 0.f;
     }
     const size_t plane = static_cast<size_t>(T) * e_pad;
-    for (int tt = cta; tt < T; tt += n_ctas) {
-      if (warp < NE) {
-        const float *src = zp + static_cast<size_t>(tt) * e_pad + warp * 32 + lane;
-        float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        int sp = 0;
-        for (; sp + 8 <= splits; sp += 8) {
+    const int warps_per_cta = blockDim.x >> 5;
+    const int n_warps = gridDim.x * gridDim.y * warps_per_cta;
+    const int gw = (blockIdx.y * gridDim.x + blockIdx.x) * warps_per_cta + warp;
+    for (int tt = gw; tt < T; tt += n_warps) {
+      const float *src = zp + static_cast<size_t>(tt) * e_pad + lane;
+      float z[NE];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) a8[u] += __ldcg(src + (sp + u) * plane);
+      for (int j = 0; j < NE; ++j) z[j] = 0.f;
+      int sp = 0;
+      for (; sp + 4 <= splits; sp += 4) {
+#pragma unroll
+        for (int j = 0; j < NE; ++j) {
+          const float *q = src + 32 * j + sp * plane;
+          const float a0 = __ldcg(q), a1 = __ldcg(q + plane), a2 = __ldcg(q + 2 * plane),
+                      a3 = __ldcg(q + 3 * plane);
+          z[j] += (a0 + a1) + (a2 + a3);
         }
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (sp + u < splits) a8[u] += __ldcg(src + (sp + u) * plane);
-        zs[warp * 32 + lane] = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
       }
-      __syncthreads();
-      if (warp == 0) select_token<NE>(zs, bias_r, tt, o, lane);
-      __syncthreads();
+      for (; sp < splits; ++sp) {
+#pragma unroll
+        for (int j = 0; j < NE; ++j) z[j] += __ldcg(src + 32 * j + sp * plane);
+      }
+      select_token<NE>(z, bias_r, tt, o, lane);
     }
   }
 }

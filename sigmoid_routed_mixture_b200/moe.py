@@ -201,8 +201,11 @@ def workspace_bytes(cfg: Config) -> int:
 
 
 def workspace(cfg: Config, device=None) -> torch.Tensor:
-    """A workspace tensor (uint8) of moe_workspace_size bytes."""
-    return torch.empty(workspace_bytes(cfg), dtype=torch.uint8, device=device or "cuda")
+    """A workspace tensor (uint8) of moe_workspace_size bytes, its control words
+    (the first 256 bytes: the device error word among them) zeroed."""
+    ws = torch.empty(workspace_bytes(cfg), dtype=torch.uint8, device=device or "cuda")
+    ws[:256].zero_()
+    return ws
 
 
 def pack_weights(cfg: Config, w1, w3, w2, ws1=None, ws3=None, ws2=None, stream=None, inexact=None):

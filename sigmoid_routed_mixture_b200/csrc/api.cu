@@ -76,6 +76,16 @@ WsLayout layout(const moe_cfg_t &c) {
 
 using namespace srm::host;
 
+// The token rows a grouped GEMM reads ([rows][inner], 16-bit), as its two
+// tensor maps: small boxes for tail tiles, big boxes for full tiles.
+bool make_tok_maps(srm::TokMaps *m, const void *ptr, uint64_t inner, uint64_t rows,
+                   CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  return make_tmap(&m->small, ptr, inner, rows, 64, static_cast<uint32_t>(srm::gemm_tok_box_rows()),
+                   dtype) &&
+         make_tmap(&m->big, ptr, inner, rows, 64, static_cast<uint32_t>(srm::gemm_tok_big_box_rows()),
+                   dtype);
+}
+
 }  // namespace
 
 extern "C" {
@@ -296,9 +306,9 @@ moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights,
   const int H = cfg->H, I = cfg->I, E = cfg->E;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool pair = srm::gemm_use_pairs(cfg->T, cfg->K, cfg->E);
-  CUtensorMap tm_x, tm_w13;
-  if (!make_tmap(&tm_x, wsb + L.xs, H, static_cast<uint64_t>(rows_y(*cfg)), 64,
-                 static_cast<uint32_t>(srm::gemm_tok_box_rows())) ||
+  srm::TokMaps tm_x;
+  CUtensorMap tm_w13;
+  if (!make_tok_maps(&tm_x, wsb + L.xs, H, static_cast<uint64_t>(rows_y(*cfg))) ||
       !make_tmap(&tm_w13, weights->w13, H, static_cast<uint64_t>(E + 1) * 2 * I, 64,
                  static_cast<uint32_t>(srm::gemm_w_box_rows())))
     return MOE_ERR_CUDA;
@@ -330,10 +340,10 @@ moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   const int H = cfg->H, I = cfg->I, E = cfg->E;
   const bool pair = srm::gemm_use_pairs(cfg->T, cfg->K, cfg->E);
-  CUtensorMap tm_h, tm_w2;
-  if (!make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(rows_y(*cfg)), 64,
-                 static_cast<uint32_t>(srm::gemm_tok_box_rows()),
-                 CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+  srm::TokMaps tm_h;
+  CUtensorMap tm_w2;
+  if (!make_tok_maps(&tm_h, wsb + L.h, I, static_cast<uint64_t>(rows_y(*cfg)),
+                     CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
       !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(E + 1) * H, 64,
                  static_cast<uint32_t>(srm::gemm_w_box_rows()), CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_CUDA;
@@ -422,14 +432,12 @@ moe_status_t moe_dense_mlp(const moe_cfg_t *cfg, const moe_weights_t *weights, c
   if (srm::launch_identity_rows(offsets, sorted, T, num_sms(), s) != cudaSuccess)
     return MOE_ERR_CUDA;
   const bool pair = cfg->T >= 512;
-  CUtensorMap tm_x, tm_w13, tm_h, tm_w2;
-  if (!make_tmap(&tm_x, x, H, static_cast<uint64_t>(T), 64,
-                 static_cast<uint32_t>(srm::gemm_tok_box_rows())) ||
+  srm::TokMaps tm_x, tm_h;
+  CUtensorMap tm_w13, tm_w2;
+  if (!make_tok_maps(&tm_x, x, H, static_cast<uint64_t>(T)) ||
       !make_tmap(&tm_w13, weights->w13, H, 2ull * I, 64,
                  static_cast<uint32_t>(srm::gemm_w_box_rows())) ||
-      !make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(T), 64,
-                 static_cast<uint32_t>(srm::gemm_tok_box_rows()),
-                 CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_tok_maps(&tm_h, wsb + L.h, I, static_cast<uint64_t>(T), CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
       !make_tmap(&tm_w2, weights->w2, I, static_cast<uint64_t>(H), 64,
                  static_cast<uint32_t>(srm::gemm_w_box_rows()), CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_CUDA;
@@ -476,14 +484,12 @@ moe_status_t moe_ep_shared(const moe_cfg_t *cfg, const moe_weights_t *shared, co
     return MOE_ERR_CUDA;
   // the tile shape the single-GPU path would use for this block
   const bool pair = srm::gemm_use_pairs(cfg->T, cfg->K, cfg->E);
-  CUtensorMap tm_x, tm_w13, tm_h, tm_w2;
-  if (!make_tmap(&tm_x, x, H, static_cast<uint64_t>(T), 64,
-                 static_cast<uint32_t>(srm::gemm_tok_box_rows())) ||
+  srm::TokMaps tm_x, tm_h;
+  CUtensorMap tm_w13, tm_w2;
+  if (!make_tok_maps(&tm_x, x, H, static_cast<uint64_t>(T)) ||
       !make_tmap(&tm_w13, shared->w13, H, 2ull * I, 64,
                  static_cast<uint32_t>(srm::gemm_w_box_rows())) ||
-      !make_tmap(&tm_h, wsb + L.h, I, static_cast<uint64_t>(T), 64,
-                 static_cast<uint32_t>(srm::gemm_tok_box_rows()),
-                 CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_tok_maps(&tm_h, wsb + L.h, I, static_cast<uint64_t>(T), CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
       !make_tmap(&tm_w2, shared->w2, I, static_cast<uint64_t>(H), 64,
                  static_cast<uint32_t>(srm::gemm_w_box_rows()), CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_CUDA;

@@ -73,7 +73,8 @@ namespace gg {
 constexpr int BM = 128;        // weight rows per CTA (tensor-memory lanes)
 constexpr int BT = 256;        // tokens per tile (largest MMA N)
 constexpr int BK = 64;
-constexpr int TOK_BOX = 32;    // token rows per TMA box
+constexpr int TOK_BOX = 32;    // token rows per TMA box of a tail tile
+constexpr int TOK_BOX_BIG = 128;  // token rows per TMA box when a CTA's rows are a multiple of it
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BT;  // two accumulators
 constexpr int MAX_GROUPS = 257;
@@ -108,6 +109,7 @@ struct Smem {
   int total_mtiles;
   int tile_start[MAX_GROUPS + 1];
   int grp_off[MAX_GROUPS + 1];
+  float epi[4][32][33];  // kDown: one 32 x 32 transpose buffer per epilogue warp (padded rows)
 };
 template <bool kPair>
 constexpr size_t smem_bytes() {
@@ -168,14 +170,13 @@ __device__ __forceinline__ uint16_t f16_sat(float v, bool &sat) {
 }
 
 template <int kMode, bool kPair>
-__device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, const CUtensorMap &tmap_w,
-                                                  const GemmArgs &p) {
+__device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, const CUtensorMap &tmap_tok_big,
+                                                  const CUtensorMap &tmap_w, const GemmArgs &p) {
   using namespace gg;
   using C = Cfg<kPair>;
   constexpr int STAGES = C::STAGES;
   constexpr int A_BYTES = C::A_BYTES;
   constexpr int B_BYTES = C::B_BYTES;
-  constexpr int TOK_BOX_BYTES = TOK_BOX * BK * 2;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   uint8_t *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -214,6 +215,7 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
     s.mma_consumed = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmap_tok);
+    tma_prefetch_desc(&tmap_tok_big);
     tma_prefetch_desc(&tmap_w);
   }
   if (warp == 1) {
@@ -311,8 +313,13 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
       const int w_row = c.g * p.n_total + c.w0 + rank * BM;   // this CTA's weight rows
       const int tok_rows = kPair ? c.n / 2 : c.n;             // this CTA's token rows
       const int tok_row0 = c.row_base + rank * tok_rows;
-      const int nb = (tok_rows + TOK_BOX - 1) / TOK_BOX;
-      const uint32_t tx = (kPair ? 2u : 1u) * static_cast<uint32_t>(A_BYTES + nb * TOK_BOX_BYTES);
+      // full tiles: one or two 128-row boxes (each TMA instruction costs issue
+      // time on the single producer lane); tails: 32-row boxes
+      const bool big = tok_rows % TOK_BOX_BIG == 0;
+      const int box_rows = big ? TOK_BOX_BIG : TOK_BOX;
+      const CUtensorMap *tmap_b = big ? &tmap_tok_big : &tmap_tok;
+      const int nb = (tok_rows + box_rows - 1) / box_rows;
+      const uint32_t tx = (kPair ? 2u : 1u) * static_cast<uint32_t>(A_BYTES + nb * box_rows * BK * 2);
       bool ok = true;
       for (int kb = 0; kb < kblocks; ++kb) {
         if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, p.err)) {
@@ -326,13 +333,13 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
             const uint32_t full_leader = cluster_map(&s.full[stage], 0);
             tma_load_2d_pair(sA + stage * A_BYTES, &tmap_w, full_leader, kb * BK, w_row);
             for (int j = 0; j < nb; ++j)
-              tma_load_2d_pair(b_dst + j * TOK_BOX_BYTES, &tmap_tok, full_leader, kb * BK,
-                               tok_row0 + j * TOK_BOX);
+              tma_load_2d_pair(b_dst + j * box_rows * BK * 2, tmap_b, full_leader, kb * BK,
+                               tok_row0 + j * box_rows);
           } else {
             tma_load_2d(sA + stage * A_BYTES, &tmap_w, &s.full[stage], kb * BK, w_row);
             for (int j = 0; j < nb; ++j)
-              tma_load_2d(b_dst + j * TOK_BOX_BYTES, &tmap_tok, &s.full[stage], kb * BK,
-                          tok_row0 + j * TOK_BOX);
+              tma_load_2d(b_dst + j * box_rows * BK * 2, tmap_b, &s.full[stage], kb * BK,
+                          tok_row0 + j * box_rows);
           }
         }
         __syncwarp();
@@ -478,16 +485,27 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
                   __ushort_as_half(f16_sat(g * sigmoidf_(g) * u, sat));
           }
         } else {
-          // lane = output feature f; destinations and gates broadcast by shuffles
-          const int f = wr + lane;
-          __half *y = reinterpret_cast<__half *>(p.out);
+          // transpose the 32 features x 32 tokens chunk through this warp's
+          // buffer (row stride 33: both passes conflict-free), so that lane l
+          // owns token 32m + l: its own destination and gate, and its 32
+          // features (64 contiguous bytes of the slot row) in four 16-byte stores
+          float(&buf)[32][33] = s.epi[warp - 2];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int a = __shfl_sync(0xffffffffu, my_a[m], k);
-            const float gv = __shfl_sync(0xffffffffu, my_g[m], k);
-            if (a >= 0)
-              y[static_cast<size_t>(a) * p.out_ld + f] = __ushort_as_half(f16_sat(gv * __uint_as_float(cv[k]), sat));
+          for (int k = 0; k < 32; ++k) buf[k][lane] = __uint_as_float(cv[k]);
+          __syncwarp();
+          if (my_a[m] >= 0) {
+            const float gv = my_g[m];
+            uint32_t packed[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              packed[j] = pack_f16x2_sat(gv * buf[lane][2 * j], gv * buf[lane][2 * j + 1], sat);
+            uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) +
+                                                   static_cast<size_t>(my_a[m]) * p.out_ld + wr);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(packed[4 * v4], packed[4 * v4 + 1], packed[4 * v4 + 2], packed[4 * v4 + 3]);
           }
+          __syncwarp();  // the buffer is read before the next chunk overwrites it
         }
       }
       if (sat) record_error(p.err, MOE_ERR_RANGE);
@@ -557,15 +575,17 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
 template <int kMode>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gg::THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_tok,
+                             const __grid_constant__ CUtensorMap tmap_tok_big,
                              const __grid_constant__ CUtensorMap tmap_w, GemmArgs p) {
-  grouped_gemm_body<kMode, true>(tmap_tok, tmap_w, p);
+  grouped_gemm_body<kMode, true>(tmap_tok, tmap_tok_big, tmap_w, p);
 }
 
 template <int kMode>
 __global__ void __launch_bounds__(gg::THREADS, 1)
     grouped_gemm_solo_kernel(const __grid_constant__ CUtensorMap tmap_tok,
+                             const __grid_constant__ CUtensorMap tmap_tok_big,
                              const __grid_constant__ CUtensorMap tmap_w, GemmArgs p) {
-  grouped_gemm_body<kMode, false>(tmap_tok, tmap_w, p);
+  grouped_gemm_body<kMode, false>(tmap_tok, tmap_tok_big, tmap_w, p);
 }
 
 // CTA pairs unless the experts average fewer than 8 rows each (decode), where
@@ -573,11 +593,12 @@ __global__ void __launch_bounds__(gg::THREADS, 1)
 bool gemm_use_pairs(int64_t T, int K, int E) { return T * K >= 8LL * (E > 0 ? E : 1); }
 
 int gemm_tok_box_rows() { return gg::TOK_BOX; }
+int gemm_tok_big_box_rows() { return gg::TOK_BOX_BIG; }
 int gemm_w_box_rows() { return gg::BM; }
 
 template <int kMode>
-static cudaError_t launch_mode(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p,
-                               bool pair, int num_sms, cudaStream_t stream) {
+static cudaError_t launch_mode(const TokMaps &tok, const CUtensorMap &tw, const GemmArgs &p, bool pair,
+                               int num_sms, cudaStream_t stream) {
   static int cached_units[2][2][64] = {{{0}}};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -604,21 +625,21 @@ static cudaError_t launch_mode(const CUtensorMap &ta, const CUtensorMap &tb, con
         clusters = num_sms / 2;
       units = clusters;
     }
-    kern<<<2 * units, gg::THREADS, smem, stream>>>(ta, tb, p);
+    kern<<<2 * units, gg::THREADS, smem, stream>>>(tok.small, tok.big, tw, p);
   } else {
     auto kern = grouped_gemm_solo_kernel<kMode>;
     constexpr size_t smem = gg::smem_bytes<false>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms, gg::THREADS, smem, stream>>>(ta, tb, p);
+    kern<<<num_sms, gg::THREADS, smem, stream>>>(tok.small, tok.big, tw, p);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_grouped_gemm(int mode, bool pair, const CUtensorMap &ta, const CUtensorMap &tb,
+cudaError_t launch_grouped_gemm(int mode, bool pair, const TokMaps &tok, const CUtensorMap &tw,
                                 const GemmArgs &p, int num_sms, cudaStream_t stream) {
-  if (mode == kUp) return launch_mode<kUp>(ta, tb, p, pair, num_sms, stream);
-  return launch_mode<kDown>(ta, tb, p, pair, num_sms, stream);
+  if (mode == kUp) return launch_mode<kUp>(tok, tw, p, pair, num_sms, stream);
+  return launch_mode<kDown>(tok, tw, p, pair, num_sms, stream);
 }
 
 }  // namespace srm

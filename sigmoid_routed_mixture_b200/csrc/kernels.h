@@ -34,15 +34,19 @@ struct GemmArgs {
 // Tile shape of the grouped GEMMs: the weights are the MMA's M side (256 rows
 // per CTA pair, 128 per single CTA), the tokens its N side (up to 256 per
 // tile, rounded up to 16).  CTA pairs unless the experts average fewer than 8
-// rows each.  Tensor maps: tokens [rows][K] with boxes of gemm_tok_box_rows()
-// rows, weights [rows][K] with boxes of gemm_w_box_rows() rows, 64 K-elements
-// wide, 128-byte swizzle.
+// rows each.  Tensor maps: tokens [rows][K] (TokMaps), weights [rows][K] with
+// boxes of gemm_w_box_rows() rows, 64 K-elements wide, 128-byte swizzle.
 bool gemm_use_pairs(int64_t T, int K, int E);
 int gemm_tok_box_rows();
+int gemm_tok_big_box_rows();
 int gemm_w_box_rows();
-cudaError_t launch_grouped_gemm(int mode, bool pair, const CUtensorMap &tmap_tok,
-                                const CUtensorMap &tmap_w, const GemmArgs &p, int num_sms,
-                                cudaStream_t stream);
+// the token rows as two tensor maps over the same memory: boxes of
+// gemm_tok_box_rows() rows (tail tiles) and gemm_tok_big_box_rows() rows (full tiles)
+struct TokMaps {
+  CUtensorMap small, big;
+};
+cudaError_t launch_grouped_gemm(int mode, bool pair, const TokMaps &tok, const CUtensorMap &tmap_w,
+                                const GemmArgs &p, int num_sms, cudaStream_t stream);
 
 // router: W_r split into bf16 parts [3][e_pad][H] (wsplit), fp32 partial logits
 // zp [splits][T][e_pad] (split-K only); tmap_x: x [T][H] box 64 x 128,

@@ -71,26 +71,29 @@ namespace srm {
 
 namespace gg {
 constexpr int BM = 128;        // weight rows per CTA (tensor-memory lanes)
-constexpr int BT = 256;        // tokens per tile (largest MMA N)
 constexpr int BK = 64;
 constexpr int TOK_BOX = 32;    // token rows per TMA box of a tail tile
 constexpr int TOK_BOX_BIG = 128;  // token rows per TMA box when a CTA's rows are a multiple of it
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 2 * BT;  // two accumulators
 constexpr int MAX_GROUPS = 257;
-constexpr int MAX_STAGES = 6;
+constexpr int MAX_STAGES = 8;
 constexpr int TILE_RING = 4;  // tile ids in flight between the scheduler and the roles
 
 // kPair: a CTA pair shares each tile (M = 256 weight rows, each CTA loads 128
-// of them and half of the tokens); solo: one CTA per tile (M = 128, all tokens).
+// of them and half of up to 256 tokens).  Solo (small batches, where the
+// experts hold a few rows each and the weights stream from HBM): one CTA per
+// tile, M = 128, up to 64 tokens, so that a stage is 16 KB of weights + 8 KB
+// of tokens and 8 of them keep 128 KB of weights in flight per SM.
 template <bool kPair>
 struct Cfg {
+  static constexpr int BT = kPair ? 256 : 64;           // tokens per tile (largest MMA N)
   static constexpr int W_BLOCK = kPair ? 2 * BM : BM;   // weight rows per tile (MMA M)
   static constexpr int TOK_ROWS = kPair ? BT / 2 : BT;  // token rows one CTA holds at most
-  static constexpr int STAGES = kPair ? 6 : 4;
+  static constexpr int STAGES = kPair ? 6 : 8;
   static constexpr int A_BYTES = BM * BK * 2;           // 16 KB of weights
-  static constexpr int B_BYTES = TOK_ROWS * BK * 2;     // 16 or 32 KB of token rows at most
+  static constexpr int B_BYTES = TOK_ROWS * BK * 2;     // 16 or 8 KB of token rows at most
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BT;  // two accumulators (512 or 128 columns)
   static constexpr uint32_t EPI_ARRIVALS = kPair ? 8 : 4;
 };
 
@@ -120,7 +123,7 @@ constexpr size_t smem_bytes() {
 struct TileCoord {
   int g;          // group
   int row_base;   // first token row of the tile (expert-sorted order)
-  int rows;       // valid token rows (1..256)
+  int rows;       // valid token rows (1 .. BT)
   int n;          // MMA N: rows rounded up to 16
   int w0;         // first weight row of the tile within the group
 };
@@ -154,10 +157,11 @@ __device__ __forceinline__ TileCoord decode_tile(const gg::Smem &s, int groups, 
   const int r = local - m0 * n_tiles;
   const int nt = r / cm;
   const int mt = m0 + (r - nt * cm);
+  constexpr int BT = gg::Cfg<kPair>::BT;
   TileCoord c;
   c.g = lo;
-  c.row_base = s.grp_off[lo] + mt * gg::BT;
-  c.rows = max(0, min(gg::BT, s.grp_off[lo + 1] - c.row_base));
+  c.row_base = s.grp_off[lo] + mt * BT;
+  c.rows = max(0, min(BT, s.grp_off[lo + 1] - c.row_base));
   c.n = max(16, (c.rows + 15) & ~15);
   c.w0 = nt * gg::Cfg<kPair>::W_BLOCK;
   return c;
@@ -174,6 +178,8 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
                                                   const CUtensorMap &tmap_w, const GemmArgs &p) {
   using namespace gg;
   using C = Cfg<kPair>;
+  constexpr int BT = C::BT;
+  constexpr uint32_t TMEM_COLS = C::TMEM_COLS;
   constexpr int STAGES = C::STAGES;
   constexpr int A_BYTES = C::A_BYTES;
   constexpr int B_BYTES = C::B_BYTES;

@@ -9,6 +9,7 @@ only the NVIDIA driver on the machine that loads it.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -56,14 +57,18 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     os.makedirs(BUILD_DIR, exist_ok=True)
     nvcc = _nvcc()
-    objs = []
+    jobs = []
     for src in _sources():
         obj = os.path.join(BUILD_DIR, os.path.basename(src)[:-3] + ".o")
-        cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]
-        if verbose:
+        jobs.append((src, obj, [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]))
+    if verbose:
+        for _, _, cmd in jobs:
             print(" ".join(cmd), flush=True)
-        subprocess.check_call(cmd)
-        objs.append(obj)
+    # the translation units are independent: compile them side by side
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+        for f in [ex.submit(subprocess.check_call, cmd) for _, _, cmd in jobs]:
+            f.result()
+    objs = [obj for _, obj, _ in jobs]
     tmp = LIB + ".tmp.%d" % os.getpid()
     cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs,
            "-cudart", "static"]

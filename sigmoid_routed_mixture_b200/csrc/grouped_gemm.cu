@@ -112,7 +112,7 @@ struct Smem {
   int total_mtiles;
   int tile_start[MAX_GROUPS + 1];
   int grp_off[MAX_GROUPS + 1];
-  float epi[4][32][33];  // kDown: one 32 x 32 transpose buffer per epilogue warp (padded rows)
+  float epi[4][32][33];  // one 32 x 32 transpose buffer per epilogue warp (padded rows)
 };
 template <bool kPair>
 constexpr size_t smem_bytes() {
@@ -489,34 +489,35 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
         uint32_t cv[32];
         tmem_ld32(taddr + 32 * m, cv);
         tmem_ld_wait();
-        if (kMode == kUp) {
-          // lanes 0-15 hold gate rows of features j0 .. j0+15, lanes 16-31 the
-          // matching up rows (the 32-row packing unit); after one exchange lane
-          // l has (g, u) of feature j0 + (l % 16) for tokens half*16 ..
-          // half*16+15 of the chunk, half = l / 16
-          const int half = lane >> 4;
-          const int jf = wr / 2 + (lane & 15);
-          __half *h = reinterpret_cast<__half *>(p.out);
+        // transpose the 32 weight rows x 32 tokens chunk through this warp's
+        // buffer (row stride 33: both passes conflict-free), so that lane l
+        // owns token 32m + l and reads its 32 values from its own row
+        float(&buf)[32][33] = s.epi[warp - 2];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float mine = __uint_as_float(cv[half ? k + 16 : k]);
-            const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(cv[half ? k : k + 16]), 16);
-            const float g = half ? other : mine;
-            const float u = half ? mine : other;
-            const int t = 32 * m + half * 16 + k;
-            if (t < c.rows)
-              h[static_cast<size_t>(c.row_base + t) * p.out_ld + jf] =
-                  __ushort_as_half(f16_sat(g * sigmoidf_(g) * u, sat));
+        for (int k = 0; k < 32; ++k) buf[k][lane] = __uint_as_float(cv[k]);
+        __syncwarp();
+        if (kMode == kUp) {
+          // rows 0-15 of the chunk are the gate rows of features j0 .. j0+15,
+          // rows 16-31 the matching up rows (the 32-row packing unit): lane l
+          // computes h = silu(g) * u of its token for the 16 features and
+          // writes them as two 16-byte stores (32 contiguous bytes of its h row)
+          if (32 * m + lane < c.rows) {
+            uint32_t packed[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float g0 = buf[lane][2 * j], g1 = buf[lane][2 * j + 1];
+              const float u0 = buf[lane][16 + 2 * j], u1 = buf[lane][16 + 2 * j + 1];
+              packed[j] = pack_f16x2_sat(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1, sat);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) +
+                                                   static_cast<size_t>(c.row_base + 32 * m + lane) * p.out_ld +
+                                                   wr / 2);
+            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
           }
         } else {
-          // transpose the 32 features x 32 tokens chunk through this warp's
-          // buffer (row stride 33: both passes conflict-free), so that lane l
-          // owns token 32m + l: its own destination and gate, and its 32
-          // features (64 contiguous bytes of the slot row) in four 16-byte stores
-          float(&buf)[32][33] = s.epi[warp - 2];
-#pragma unroll
-          for (int k = 0; k < 32; ++k) buf[k][lane] = __uint_as_float(cv[k]);
-          __syncwarp();
+          // lane l: its token's destination and gate, its 32 output features
+          // (64 contiguous bytes of the slot row) in four 16-byte stores
           if (my_a[m] >= 0) {
             const float gv = my_g[m];
             uint32_t packed[16];
@@ -529,8 +530,8 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
             for (int v4 = 0; v4 < 4; ++v4)
               dst[v4] = make_uint4(packed[4 * v4], packed[4 * v4 + 1], packed[4 * v4 + 2], packed[4 * v4 + 3]);
           }
-          __syncwarp();  // the buffer is read before the next chunk overwrites it
         }
+        __syncwarp();  // the buffer is read before the next chunk overwrites it
       }
       if (sat) record_error(p.err, MOE_ERR_RANGE);
       tc_fence_before();

@@ -46,7 +46,10 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;  // warp 0 TMA, warp 1 MMA + TMEM, 8 epilogue warps
-constexpr int CHUNK = 2;                      // k-blocks per tensor-core accumulation chain
+#ifndef SRM_ROUTER_CHUNK
+#define SRM_ROUTER_CHUNK 2
+#endif
+constexpr int CHUNK = SRM_ROUTER_CHUNK;       // k-blocks per tensor-core accumulation chain
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int MAX_SMEM = 232448;  // 227 KB dynamic shared memory per CTA
 }  // namespace rt

@@ -272,7 +272,6 @@ GemmArgs gemm_args(const moe_cfg_t &c, const int32_t *offsets, const int32_t *so
   p.groups = c.E + c.has_shared;
   p.tile_counter = reinterpret_cast<int *>(wsb + L.err + 128);
   p.stall = 0;
-  p.w = nullptr;
   return p;
 }
 
@@ -323,7 +322,6 @@ moe_status_t moe_expert_up(const moe_cfg_t *cfg, const moe_weights_t *weights,
   p.n_total = 2 * I;
   p.k_total = H;
   p.out_ld = I;
-  p.w = weights->w13;
   if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
   return cuda_status(srm::launch_grouped_gemm(srm::kUp, pair, tm_x, tm_w13, p, num_sms(), s));
 }
@@ -354,7 +352,6 @@ moe_status_t moe_expert_down(const moe_cfg_t *cfg, const moe_weights_t *weights,
   p.n_total = H;
   p.k_total = I;
   p.out_ld = H;
-  p.w = weights->w2;
   if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MOE_ERR_CUDA;
   return cuda_status(srm::launch_grouped_gemm(srm::kDown, pair, tm_h, tm_w2, p, num_sms(),
@@ -449,7 +446,6 @@ moe_status_t moe_dense_mlp(const moe_cfg_t *cfg, const moe_weights_t *weights, c
   p.n_total = 2 * I;
   p.k_total = H;
   p.out_ld = I;
-  p.w = weights->w13;
   if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s) != cudaSuccess ||
       srm::launch_grouped_gemm(srm::kUp, pair, tm_x, tm_w13, p, num_sms(), s) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -457,7 +453,6 @@ moe_status_t moe_dense_mlp(const moe_cfg_t *cfg, const moe_weights_t *weights, c
   p.n_total = H;
   p.k_total = I;
   p.out_ld = H;
-  p.w = weights->w2;
   if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s) != cudaSuccess ||
       srm::launch_grouped_gemm(srm::kDown, pair, tm_h, tm_w2, p, num_sms(), s) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -504,7 +499,6 @@ moe_status_t moe_ep_shared(const moe_cfg_t *cfg, const moe_weights_t *shared, co
   p.n_total = 2 * I;
   p.k_total = H;
   p.out_ld = I;
-  p.w = shared->w13;
   if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s) != cudaSuccess ||
       srm::launch_grouped_gemm(srm::kUp, pair, tm_x, tm_w13, p, num_sms(), s) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -512,7 +506,6 @@ moe_status_t moe_ep_shared(const moe_cfg_t *cfg, const moe_weights_t *shared, co
   p.n_total = H;
   p.k_total = I;
   p.out_ld = H;
-  p.w = shared->w2;
   if (cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s) != cudaSuccess)
     return MOE_ERR_CUDA;
   return cuda_status(srm::launch_grouped_gemm(srm::kDown, pair, tm_h, tm_w2, p, num_sms(), s));

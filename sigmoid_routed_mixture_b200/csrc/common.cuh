@@ -146,14 +146,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, uint64_
       : "memory");
 }
 
-// Start moving `bytes` (a multiple of 16) at a 16-byte-aligned global address
-// into L2, without waiting and without touching shared memory.
-__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
-               "r"(bytes)
-               : "memory");
-}
-
 // ----------------------------------------------------------------- tcgen05
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA

@@ -305,24 +305,6 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
             st_shared_remote(cluster_map(&s.tile_ring[ts], 1), t);
             mbar_arrive_remote(cluster_map(&s.tile_full[ts], 1));
           }
-          // The tile about one round ahead (t + units) will be taken about
-          // one tile-time from now; if it starts a new weight block, pull that
-          // block into L2 now so its first k-blocks do not wait on HBM.  Only
-          // for blocks of at most 1 MB, so that a round of them (units x 1 MB)
-          // fits in L2 (the mid-size shapes; the 3 MB GLM-5 blocks are shared
-          // by many token blocks and streamed by the ring itself).
-          const int64_t blk_bytes = static_cast<int64_t>(C::W_BLOCK) * p.k_total * 2;
-          const int tp = t + static_cast<int>(gridDim.x) / (kPair ? 2 : 1);
-          if (t >= 0 && p.w && blk_bytes <= (1 << 20) && tp < total_tiles) {
-            const TileCoord a = decode_tile<kPair>(s, groups, n_tiles, m_chunk, tp);
-            const TileCoord b = decode_tile<kPair>(s, groups, n_tiles, m_chunk, tp - 1);
-            if (a.g != b.g || a.w0 != b.w0) {
-              const uint8_t *src = static_cast<const uint8_t *>(p.w) +
-                                   (static_cast<int64_t>(a.g) * p.n_total + a.w0) * p.k_total * 2;
-              for (int64_t off = 0; off < blk_bytes; off += 65536)
-                prefetch_l2_bulk(src + off, static_cast<uint32_t>(blk_bytes - off < 65536 ? blk_bytes - off : 65536));
-            }
-          }
         }
         __syncwarp();
       }

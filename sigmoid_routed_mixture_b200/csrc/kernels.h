@@ -27,8 +27,6 @@ struct GemmArgs {
   int k_total;             // reduction length (H for kUp, I for kDown)
   int out_ld;              // elements per output row (I for kUp, H for kDown)
   int *tile_counter;       // zeroed before the launch; units take their next tile from it
-  const void *w;           // the weights the tensor map covers ([rows][k_total], 16-bit), for
-                           // L2 prefetches of small weight blocks; may be null
   int stall;               // failure-detection tests only: the producer issues no loads, so
                            // the MMA warp's bounded wait runs out (MOE_ERR_TIMEOUT)
 };

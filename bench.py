@@ -44,7 +44,7 @@ def kernels_per_step(w, num_sms=148):
     permutation (one CTA for small batches, else histogram + scan + scatter);
     token gather (invert + scatter); up GEMM; down GEMM; combine."""
     route = 1
-    permute = 1 if w.T * w.K <= 16384 else 3
+    permute = 1 if w.T * w.K <= 4096 else 3
     return route + permute + 2 + 1 + 1 + 1
 
 

@@ -594,6 +594,89 @@ def run_dsa(args, world, rank, dist, dev):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ router stage
+
+ROUTER_WORKLOADS = {"router_glm5_prefill": "glm5_prefill", "router_glm5_decode": "glm5_decode"}
+ROUTER_METRIC = "router tokens/s (GLM-5 shape: 256 experts top-8, H 6144, 1 B200)"
+
+
+def run_router(args, world, rank, dist, dev):
+    """The router alone (moe_route_packed: logits, scores, biased top-K, margin,
+    gates in one kernel) on the block's tokens, timed like the block: CUDA-graph
+    replays between device synchronisations, CUDA events.  Roofline: the split
+    logits' tensor-core work (3 x 2 T H E_pad FLOP; the algorithmic 2 T H E is
+    given too) against the bf16 peak, the bytes (x, W_r split, outputs) against
+    HBM."""
+    import torch
+
+    from sigmoid_routed_mixture_b200 import moe
+
+    w = W.WORKLOADS[ROUTER_WORKLOADS[args.workload]]
+    x, w_r, b = replica_tokens(w, rank)
+    cfg = moe.Config.of(w)
+    x_dev = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    w_r_dev, b_dev = torch.from_numpy(w_r).to(dev), torch.from_numpy(b).to(dev)
+    packed = moe.pack_router(cfg, w_r_dev)
+    ws = moe.workspace(cfg, device=dev)
+    out = moe.route_packed(cfg, x_dev, packed, b_dev, ws)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moe.route_packed(cfg, x_dev, packed, b_dev, ws, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(args.warmup):
+        graph.replay()
+    sampler = ClockSampler(torch.cuda.current_device())
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    a.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    z.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if moe.device_error(ws) != 0:
+        raise RuntimeError("device error during the timed steps")
+    t_max = max_over_ranks(a.elapsed_time(z), dist, dev)
+    ms = t_max / args.steps
+    pk = peaks()
+    e_pad = -(-w.E // 64) * 64
+    f_split = 3 * 2.0 * w.T * w.H * e_pad
+    f_alg = 2.0 * w.T * w.H * w.E
+    bytes_ = w.T * w.H * 2 + 3 * e_pad * w.H * 2 + w.E * 4 + w.T * w.K * 8 + w.T * 4
+    tpk, tpk_kind = tensor_peak(pk, t_max)
+    t_roof = max(f_split / (tpk * 1e12), bytes_ / (pk["hbm"] * 1e9))
+    if f_split / (tpk * 1e12) >= bytes_ / (pk["hbm"] * 1e9):
+        roof = {"kernel": "router_kernel", "bound": "tensor", "achieved": f_split / (ms / 1e3) / 1e12, "peak": tpk,
+                "unit": "TFLOP/s", "peak_kind": tpk_kind, "algorithmic_per_launch": f_split}
+    else:
+        roof = {"kernel": "router_kernel", "bound": "hbm", "achieved": bytes_ / (ms / 1e3) / 1e9, "peak": pk["hbm"],
+                "unit": "GB/s", "peak_kind": "copy bandwidth, " + pk["source"], "algorithmic_per_launch": bytes_}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    line = {"metric": ROUTER_METRIC, "value": w.T * world * args.steps / (t_max / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x, fp32 W_r (3-part split)",
+            "data": "synthetic (seeded)", "config": dict(workload_config(w, argparse.Namespace(gpus=world)),
+                                                         workload=args.workload),
+            "roofline": roof, "router_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof / (ms / 1e3),
+                                                  "f_split_tflop": f_split / 1e12, "f_alg_tflop": f_alg / 1e12,
+                                                  "bytes_gb": bytes_ / 1e9},
+            "launch": "cuda graph replay", "gpu_launches": args.steps, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ our arm
 
 STAGES = ["route", "permute", "gather_tokens", "expert_up", "expert_down", "combine"]
@@ -819,7 +902,7 @@ def main():
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="glm5_prefill",
-                    choices=sorted(W.WORKLOADS) + sorted(W.DSA_WORKLOADS))
+                    choices=sorted(W.WORKLOADS) + sorted(W.DSA_WORKLOADS) + sorted(ROUTER_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=0)
     ap.add_argument("--cpu-tokens", type=int, default=0)
@@ -839,6 +922,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     is_dsa = args.workload in W.DSA_WORKLOADS
+    if args.workload in ROUTER_WORKLOADS and args.impl == "reference":
+        print(json.dumps({"impl": "reference", "unavailable": "the router stage bench has no oracle arm; the "
+                          "block workloads time the oracle's router with the rest of the block"}), flush=True)
+        return
     if args.impl == "reference":
         (run_dsa_reference if is_dsa else run_reference)(args, rank)
         return
@@ -857,6 +944,11 @@ def main():
         torch.cuda.set_device(0)
     from sigmoid_routed_mixture_b200 import moe
 
+    if args.workload in ROUTER_WORKLOADS:
+        run_router(args, world, rank, dist, torch.device("cuda", torch.cuda.current_device()))
+        if dist is not None:
+            dist.destroy_process_group()
+        return
     if is_dsa:
         run_dsa(args, world, rank, dist, torch.device("cuda", torch.cuda.current_device()))
         if dist is not None:

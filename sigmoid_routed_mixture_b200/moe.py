@@ -20,7 +20,8 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libsrm_moe.so")
+# SRM_MOE_LIBRARY may name another build of the library (e.g. for an A/B of two builds)
+LIB_PATH = os.environ.get("SRM_MOE_LIBRARY") or os.path.join(_PKG, "libsrm_moe.so")
 
 # Entry points declared in include/srm_moe.h.
 SYMBOLS = (

@@ -61,12 +61,17 @@ int router_stage_bytes(int e_pad) { return rt::A_BYTES + 3 * e_pad * rt::BK * 2;
 struct RouterSmem;
 int router_stages(int e_pad, bool pair);
 
+constexpr int kMaxSplits = 16;       // more partials make the per-token reduction longer
+constexpr int kPairMinTiles = 9;     // from this many 128-token tiles on, CTA pairs
+
+// Upper bound of the split count for any SM count (sizes the partials).
 int router_splits(int T, int H) {
   const int m_tiles = (T + rt::BM - 1) / rt::BM;
   const int kblocks = H / rt::BK;
   int s = 148 / (m_tiles > 0 ? m_tiles : 1);
   const int max_s = kblocks / 2 > 0 ? kblocks / 2 : 1;
   if (s > max_s) s = max_s;
+  if (s > kMaxSplits) s = kMaxSplits;
   if (s < 1) s = 1;
   return s;
 }
@@ -247,7 +252,7 @@ __device__ __forceinline__ bool grid_barrier(int *counter, int n_ctas, int *err)
 
 // NH = e_pad / 64: each epilogue thread keeps half a row (e_pad / 2 columns).
 // kSplit: the H range is split over gridDim.y CTAs (partials + grid barrier).
-// kPair (large T, no split): clusters of two CTAs run tcgen05.mma.cta_group::2
+// kPair (enough token tiles; with or without a split): clusters of two CTAs run tcgen05.mma.cta_group::2
 // with M = 256 tokens; each CTA loads its 128 token rows and half of every
 // part's expert rows, so each byte of the split W_r crosses L2 once per 256
 // tokens instead of once per 128, and a stage is small enough for 3 of them.
@@ -256,7 +261,6 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
     router_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                   int kb_per_split, int kblocks, int stages, uint32_t tmem_cols,
                   float *__restrict__ zp, int *grid_counter, RouteOut o, int *err) {
-  static_assert(!(kSplit && kPair), "the split-K router runs on single CTAs");
   using namespace rt;
   constexpr int e_pad = NH * 64;
   constexpr int HALF = e_pad / 2;
@@ -611,10 +615,22 @@ cudaError_t launch_router_split(const float *w_r, int E, int H, uint16_t *wsplit
   return cudaGetLastError();
 }
 
+// CTA pairs (256 tokens per pair, each CTA loading half of every W_r part)
+// once there are enough token tiles: every token tile reads the whole split
+// W_r from L2, so pairs halve that traffic.  A few tiles (decode) stay single
+// CTAs, which spread W_r over many splits.
+bool router_use_pairs(int T, int H, int num_sms) {
+  (void)H;
+  (void)num_sms;
+  return (T + rt::BM - 1) / rt::BM >= kPairMinTiles;
+}
+
 int router_grid_splits(int T, int H, int num_sms) {
   const int m_tiles = (T + rt::BM - 1) / rt::BM;
+  const bool pair = router_use_pairs(T, H, num_sms);
+  const int ctas = pair ? (m_tiles + 1) / 2 * 2 : m_tiles;  // CTAs per split
   int s = router_splits(T, H);
-  const int fit = num_sms / (m_tiles > 0 ? m_tiles : 1);  // the whole grid resident at once
+  const int fit = num_sms / (ctas > 0 ? ctas : 1);  // the whole grid resident at once
   if (s > fit) s = fit;
   if (s < 1) s = 1;
   const int kblocks = H / rt::BK;
@@ -624,7 +640,6 @@ int router_grid_splits(int T, int H, int num_sms) {
 
 int router_w_box_rows(int E, bool pair) { return pair ? router_e_pad(E) / 2 : router_e_pad(E); }
 
-bool router_use_pairs(int T, int H, int num_sms) { return router_grid_splits(T, H, num_sms) == 1; }
 
 cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, const float *bias, int T,
                          int H, int E, int K, float scale, float *zp, int *grid_counter,
@@ -633,7 +648,7 @@ cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, c
   const int kblocks = H / rt::BK;
   const int splits = router_grid_splits(T, H, num_sms);
   const int kb_per = (kblocks + splits - 1) / splits;
-  const bool pair = splits == 1;  // must match router_use_pairs (the tensor map's box)
+  const bool pair = router_use_pairs(T, H, num_sms);  // the tensor map's box follows the same rule
   const int m_tiles = (T + rt::BM - 1) / rt::BM;
   dim3 grid(pair ? (m_tiles + 1) / 2 * 2 : m_tiles, splits);
   RouteOut o;
@@ -659,9 +674,15 @@ cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, c
                                                          grid_counter, o, err, stream);                    \
   }
   if (splits > 1) {
+    if (pair) {
+      SRM_ROUTER_CASES(true, true)
+    }
     SRM_ROUTER_CASES(true, false)
   }
-  SRM_ROUTER_CASES(false, true)
+  if (pair) {
+    SRM_ROUTER_CASES(false, true)
+  }
+  SRM_ROUTER_CASES(false, false)
 #undef SRM_ROUTER_CASES
 }
 

@@ -235,7 +235,7 @@ def test_malformed_offsets_are_rejected_by_the_expert_stages(T):
     MH.check_forward(case, res, np.arange(w.T))
 
 
-@pytest.mark.parametrize("T", [5, 300, 9600])  # split-K paths (5, 300) and one CTA per 128 tokens (9600)
+@pytest.mark.parametrize("T", [5, 300, 4096, 9600])  # split-K on single CTAs (5, 300), on CTA pairs (4096), no split (9600)
 def test_route_fp32_and_packed_router_agree_bit_exact(T):
     """moe_route (fp32 W_r, split into the workspace on every call) and
     moe_pack_router + moe_route_packed run the same router kernel on the same

@@ -61,7 +61,8 @@ int router_stage_bytes(int e_pad) { return rt::A_BYTES + 3 * e_pad * rt::BK * 2;
 struct RouterSmem;
 int router_stages(int e_pad, bool pair);
 
-constexpr int kMaxSplits = 16;       // more partials make the per-token reduction longer
+constexpr int kMaxSplits = 48;       // up to 48 CTAs stream W_r at decode (2 k-blocks each at H 6144)
+constexpr int kRowBatch = 16;        // token rows a CTA reduces and selects at a time after a split
 constexpr int kPairMinTiles = 9;     // from this many 128-token tiles on, CTA pairs
 
 // Upper bound of the split count for any SM count (sizes the partials).
@@ -223,6 +224,25 @@ __device__ __forceinline__ void select_token(const Src &zsrc, const float (&bias
   if (o.margin && lane == 0) o.margin[t] = K < o.E ? kth_key - next_key : INFINITY;
 }
 
+// Sorted insert into a top-LK list (keys descending).  Experts arrive in
+// ascending index order and an entry is passed only by a strictly greater key,
+// so equal keys keep ascending expert order.  A NaN key is never inserted.
+template <int LK>
+__device__ __forceinline__ void top_insert(float (&lk)[LK], int (&le)[LK], float key, int e) {
+  bool c[LK];
+#pragma unroll
+  for (int j = 0; j < LK; ++j) c[j] = key > lk[j];
+#pragma unroll
+  for (int j = LK - 1; j > 0; --j) {
+    lk[j] = c[j] ? (c[j - 1] ? lk[j - 1] : key) : lk[j];
+    le[j] = c[j] ? (c[j - 1] ? le[j - 1] : e) : le[j];
+  }
+  if (c[0]) {
+    lk[0] = key;
+    le[0] = e;
+  }
+}
+
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -248,6 +268,75 @@ __device__ __forceinline__ bool grid_barrier(int *counter, int n_ctas, int *err)
   }
   __syncthreads();
   return ok != 0;
+}
+
+// Selection for a staged tile of z rows, one thread per (row, half of the
+// experts): the thread scans experts [hf*HALF, min(E, (hf+1)*HALF)) of its row
+// in index order (s = sigmoid(z), key = s + b) into a sorted top-LK list
+// (LK > K).  The second half's lists pass through shared memory and the first
+// half's thread inserts them after its own (all their experts are higher, so
+// the order stays key descending, then expert ascending); it then holds the
+// token's K experts and the (K+1)-th key, and writes experts, gates
+// (scale * s / sum of the selected s, summed in rank order) and the margin.
+// All 32 * EPI_WARPS epilogue threads call this (it contains a named barrier);
+// `work` false skips the computation only.
+template <int LK, int HALF>
+__device__ __forceinline__ void select_staged(const float *zr, const float *bias_s, float *list_k,
+                                              int *list_e, int row, int hf, int t, bool work,
+                                              const RouteOut &o) {
+  float lk[LK];
+  int le[LK];
+#pragma unroll
+  for (int j = 0; j < LK; ++j) {
+    lk[j] = -INFINITY;
+    le[j] = 0x7fffffff;
+  }
+  const int e0 = hf * HALF;
+  const int e1 = min(o.E, e0 + HALF);
+  if (work) {
+#pragma unroll 1
+    for (int e = e0; e < e1; e += 4) {
+      const float4 z4 = *reinterpret_cast<const float4 *>(zr + e);
+      const float4 b4 = *reinterpret_cast<const float4 *>(bias_s + e);
+      const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
+      const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (e + i < e1) top_insert<LK>(lk, le, sigmoidf_(zz[i]) + bb[i], e + i);
+    }
+  }
+  if (hf == 1) {
+#pragma unroll
+    for (int j = 0; j < LK; ++j) {
+      list_k[j * rt::BM + row] = lk[j];
+      list_e[j * rt::BM + row] = le[j];
+    }
+  }
+  named_barrier(1, 32 * rt::EPI_WARPS);
+  if (hf != 0 || !work) return;
+#pragma unroll
+  for (int j = 0; j < LK; ++j) top_insert<LK>(lk, le, list_k[j * rt::BM + row], list_e[j * rt::BM + row]);
+  const int K = o.K;
+  float sk[LK];
+  float denom = 0.f, kth = 0.f, nxt = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < LK; ++k) {
+    sk[k] = 0.f;
+    if (k < K) {
+      sk[k] = le[k] < o.E ? sigmoidf_(zr[le[k]]) : 0.f;
+      denom += sk[k];
+    }
+    if (k == K - 1) kth = lk[k];
+    if (k == K) nxt = lk[k];
+  }
+#pragma unroll
+  for (int k = 0; k < LK; ++k) {
+    if (k < K) {
+      o.idx[static_cast<size_t>(t) * K + k] = le[k];
+      o.gate[static_cast<size_t>(t) * K + k] = o.scale * sk[k] / denom;
+    }
+  }
+  if (o.margin) o.margin[t] = K < o.E ? kth - nxt : INFINITY;
 }
 
 // NH = e_pad / 64: each epilogue thread keeps half a row (e_pad / 2 columns).
@@ -447,13 +536,25 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
           mbar_arrive_remote(cluster_map(&s.tempty[slot], 0));
       }
     }
+    const int epi_tid = threadIdx.x - 64;
+    const int rows = min(BM, T - m0);
     if (kSplit) {
-      if (ok && t < T) {
-        float4 *d4 = reinterpret_cast<float4 *>(zp + (static_cast<size_t>(split) * T + t) * e_pad +
-                                                hf * HALF);
+      // The partials go out through the drained ring (below): row per thread
+      // into shared memory, then whole rows per warp, so the stores coalesce.
+      if (ok) {
+        float4 *d4 = reinterpret_cast<float4 *>(zs + row * ZS + hf * HALF);
 #pragma unroll
         for (int v = 0; v < HALF / 4; ++v)
           d4[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+      }
+      named_barrier(1, 32 * EPI_WARPS);
+      if (!*abort_flag) {
+        constexpr int V = e_pad / 4;
+        float4 *dst = reinterpret_cast<float4 *>(zp + (static_cast<size_t>(split) * T + m0) * e_pad);
+        for (int i = epi_tid; i < rows * V; i += 32 * EPI_WARPS) {
+          const int r = i / V, c = i - r * V;
+          dst[i] = *reinterpret_cast<const float4 *>(zs + r * ZS + 4 * c);
+        }
       }
     } else {
       // Every MMA has completed (its tfull arrived) and so has every copy it
@@ -466,17 +567,23 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
         for (int v = 0; v < HALF / 4; ++v)
           d4[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
       }
+      // The bias and the second half's lists sit after the staged rows.
+      float *bias_s = zs + BM * ZS;
+      float *list_k = bias_s + e_pad;
+      int *list_e = reinterpret_cast<int *>(list_k + 17 * BM);
+      for (int e = epi_tid; e < e_pad; e += 32 * EPI_WARPS) bias_s[e] = e < o.E ? o.bias[e] : 0.f;
       named_barrier(1, 32 * EPI_WARPS);
-      if (!*abort_flag) {
-        float bias_r[NE];
-#pragma unroll
-        for (int j = 0; j < NE; ++j) {
-          const int e = lane + 32 * j;
-          bias_r[j] = e < o.E ? o.bias[e] : 0.f;
+      const bool work = !*abort_flag;  // guards work only: every thread takes the barriers
+      if (work && o.logits) {
+        for (int i = epi_tid; i < rows * o.E; i += 32 * EPI_WARPS) {
+          const int r = i / o.E, c = i - r * o.E;
+          o.logits[static_cast<size_t>(m0 + r) * o.E + c] = zs[r * ZS + c];
         }
-        for (int r = warp - 2; r < BM && m0 + r < T; r += EPI_WARPS)
-          select_token<NE>(static_cast<const float *>(zs + r * ZS), bias_r, m0 + r, o, lane);
       }
+      if (o.K < 9)
+        select_staged<9, HALF>(zs + row * ZS, bias_s, list_k, list_e, row, hf, t, work && t < T, o);
+      else
+        select_staged<17, HALF>(zs + row * ZS, bias_s, list_k, list_e, row, hf, t, work && t < T, o);
     }
   }
 
@@ -520,12 +627,14 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
   }
 
   if (kSplit) {
-    // Every CTA's partials are written; after the grid barrier each warp of
-    // the grid takes tokens t = w, w + W, ... (W = warps in the grid): its
-    // lanes sum the S partials of experts lane + 32j in split order, four
-    // splits at a time ((p0 + p1) + (p2 + p3), then into the running sum: a
-    // fixed order, deterministic whichever warp does it), and the warp selects
-    // from the sums held in its registers.  No barrier between tokens.
+    // Every CTA's partials are written; after the grid barrier CTA c takes the
+    // tokens t = c, c + C, c + 2C, ... (C CTAs in the grid), RB rows at a time.
+    // All its threads sum the S partials of those rows: groups of eight splits
+    // in a fixed tree ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7)) (a
+    // shorter last group in split order), then the group sums in group order
+    // (deterministic whichever CTA does it; every load of a group is
+    // independent, so a few round trips to L2 cover all S splits); the rows
+    // land in shared memory and each warp selects for one row at a time.
     const int splits = gridDim.y;
     if (!grid_barrier(grid_counter, gridDim.x * gridDim.y, err)) return;
     float bias_r[NE];
@@ -534,30 +643,68 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
       const int e = lane + 32 * j;
       bias_r[j] = e < o.E ? o.bias[e] : 0.f;
     }
-    const size_t plane = static_cast<size_t>(T) * e_pad;
-    const int warps_per_cta = blockDim.x >> 5;
-    const int n_warps = gridDim.x * gridDim.y * warps_per_cta;
-    const int gw = (blockIdx.y * gridDim.x + blockIdx.x) * warps_per_cta + warp;
-    for (int tt = gw; tt < T; tt += n_warps) {
-      const float *src = zp + static_cast<size_t>(tt) * e_pad + lane;
-      float z[NE];
+    constexpr int V = e_pad / 4;  // float4 columns of a row
+    const int n_ctas = gridDim.x * gridDim.y;
+    const int cta = blockIdx.y * gridDim.x + blockIdx.x;
+    const int n_rows = cta < T ? (T - 1 - cta) / n_ctas + 1 : 0;
+    const int groups = (splits + 7) / 8;
+    const size_t plane4 = static_cast<size_t>(T) * V;  // float4s per split
+    const float4 *zp4 = reinterpret_cast<const float4 *>(zp);
+    float4 *part = reinterpret_cast<float4 *>(zs + kRowBatch * ZS);  // [groups][kRowBatch][V]
+    const int n_warps = blockDim.x >> 5;
+    for (int r0 = 0; r0 < n_rows; r0 += kRowBatch) {
+      const int nb = min(kRowBatch, n_rows - r0);
+      for (int i = threadIdx.x; i < groups * nb * V; i += blockDim.x) {
+        const int g = i / (nb * V);
+        const int r = (i - g * nb * V) / V;
+        const int c = i - g * nb * V - r * V;
+        const int t = cta + (r0 + r) * n_ctas;
+        const float4 *q = zp4 + static_cast<size_t>(t) * V + c + static_cast<size_t>(8 * g) * plane4;
+        const int n = min(8, splits - 8 * g);
+        float4 sum;
+        if (n == 8) {
+          float4 a[8];
 #pragma unroll
-      for (int j = 0; j < NE; ++j) z[j] = 0.f;
-      int sp = 0;
-      for (; sp + 4 <= splits; sp += 4) {
-#pragma unroll
-        for (int j = 0; j < NE; ++j) {
-          const float *q = src + 32 * j + sp * plane;
-          const float a0 = __ldcg(q), a1 = __ldcg(q + plane), a2 = __ldcg(q + 2 * plane),
-                      a3 = __ldcg(q + 3 * plane);
-          z[j] += (a0 + a1) + (a2 + a3);
+          for (int k = 0; k < 8; ++k) a[k] = __ldcg(q + k * plane4);
+          sum.x = ((a[0].x + a[1].x) + (a[2].x + a[3].x)) + ((a[4].x + a[5].x) + (a[6].x + a[7].x));
+          sum.y = ((a[0].y + a[1].y) + (a[2].y + a[3].y)) + ((a[4].y + a[5].y) + (a[6].y + a[7].y));
+          sum.z = ((a[0].z + a[1].z) + (a[2].z + a[3].z)) + ((a[4].z + a[5].z) + (a[6].z + a[7].z));
+          sum.w = ((a[0].w + a[1].w) + (a[2].w + a[3].w)) + ((a[4].w + a[5].w) + (a[6].w + a[7].w));
+        } else {
+          sum = __ldcg(q);
+          for (int k = 1; k < n; ++k) {
+            const float4 v = __ldcg(q + k * plane4);
+            sum.x += v.x;
+            sum.y += v.y;
+            sum.z += v.z;
+            sum.w += v.w;
+          }
         }
+        if (groups == 1)
+          *reinterpret_cast<float4 *>(zs + r * ZS + 4 * c) = sum;
+        else
+          part[(g * kRowBatch + r) * V + c] = sum;
       }
-      for (; sp < splits; ++sp) {
-#pragma unroll
-        for (int j = 0; j < NE; ++j) z[j] += __ldcg(src + 32 * j + sp * plane);
+      __syncthreads();
+      if (groups > 1) {
+        for (int i = threadIdx.x; i < nb * V; i += blockDim.x) {
+          const int r = i / V, c = i - r * V;
+          float4 sum = part[r * V + c];
+          for (int g = 1; g < groups; ++g) {
+            const float4 v = part[(g * kRowBatch + r) * V + c];
+            sum.x += v.x;
+            sum.y += v.y;
+            sum.z += v.z;
+            sum.w += v.w;
+          }
+          *reinterpret_cast<float4 *>(zs + r * ZS + 4 * c) = sum;
+        }
+        __syncthreads();
       }
-      select_token<NE>(z, bias_r, tt, o, lane);
+      for (int r = warp; r < nb; r += n_warps)
+        select_token<NE>(static_cast<const float *>(zs + r * ZS), bias_r, cta + (r0 + r) * n_ctas, o,
+                         lane);
+      __syncthreads();
     }
   }
 }
@@ -583,6 +730,14 @@ static cudaError_t launch_router_kernel(dim3 grid, const CUtensorMap &tmap_x, co
   constexpr int e_pad = NH * 64;
   const size_t smem = router_smem_bytes(e_pad, kPair);
   const int stages = router_stages(e_pad, kPair);
+  // the selection stages z rows, the bias and 17-entry lists over the drained ring
+  const size_t staged = (static_cast<size_t>(rt::BM) * (e_pad + 4) + e_pad + 2 * 17 * rt::BM) * 4;
+  // after a split: kRowBatch staged rows and up to ceil(48 / 8) group sums of them
+  const size_t reduced = static_cast<size_t>(kRowBatch) * ((e_pad + 4) + (kMaxSplits + 7) / 8 * e_pad) * 4;
+  if (kSplit && reduced > static_cast<size_t>(stages) * (rt::A_BYTES + 3 * (kPair ? e_pad / 2 : e_pad) * rt::BK * 2))
+    return cudaErrorInvalidValue;
+  if (staged > static_cast<size_t>(stages) * (rt::A_BYTES + 3 * (kPair ? e_pad / 2 : e_pad) * rt::BK * 2))
+    return cudaErrorInvalidValue;
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(2 * e_pad)) cols <<= 1;  // two ping-pong accumulators
   auto kern = router_kernel<NH, kSplit, kPair>;

@@ -264,6 +264,47 @@ def test_route_fp32_and_packed_router_agree_bit_exact(T):
     MH.check_route(case, res, tok)
 
 
+@pytest.mark.parametrize("T,E,K", [(300, 64, 3), (9600, 64, 3), (9600, 256, 9), (9600, 256, 16)])
+def test_equal_keys_take_the_lower_expert(T, E, K):
+    """Experts 2j and 2j+1 get the same router row and bias, so their keys are
+    exactly equal; the selection must take them in expert order (the lower one
+    first, and never the higher one without the lower one).  300 tokens run the
+    split-K router, 9600 the one-pass router with its per-thread lists (K + 1 <=
+    9 and <= 17 entries).  The rest of the routing is checked against the oracle
+    where the oracle's margin is clear."""
+    w = W.WORKLOADS["glm47flash"].replace(T=T, E=E, K=K, seed=4100 + T + E + K)
+    cfg = moe.Config.of(w)
+    x, w_r, b = W.router_inputs(w)
+    w_r[1::2] = w_r[0::2]
+    b[1::2] = b[0::2]
+    x_dev = MH.to_dev_bf16(x)
+    ws = moe.workspace(cfg)
+    z = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    packed = moe.pack_router(cfg, torch.from_numpy(w_r).cuda())
+    idx, gate, margin = moe.route_packed(cfg, x_dev, packed, torch.from_numpy(b).cuda(), ws, logits=z)
+    torch.cuda.synchronize()
+    assert moe.device_error(ws) == 0
+    z, idx, gate, margin = z.cpu().numpy(), idx.cpu().numpy(), gate.cpu().numpy(), margin.cpu().numpy()
+    assert np.array_equal(z[:, 0::2].view(np.int32), z[:, 1::2].view(np.int32))
+    key = (1.0 / (1.0 + np.exp(-z.astype(np.float64)))) + b.astype(np.float64)
+    for t in range(T):
+        sel = idx[t].tolist()
+        assert len(set(sel)) == K
+        for e in sel:
+            if e % 2 == 1:
+                assert e - 1 in sel, "token %d took expert %d without its equal %d" % (t, e, e - 1)
+        for k in range(K - 1):
+            a, c = sel[k], sel[k + 1]
+            if a // 2 == c // 2:
+                assert a < c, "token %d: equal keys out of expert order %s" % (t, sel)
+            else:
+                assert key[t, a] >= key[t, c] - 1e-6
+    case = MH.Case(w, x=x, w_r=w_r, b=b, weights={})
+    res = dict(idx=idx, gate=gate, margin=margin, logits=z)
+    tok = np.arange(T) if T <= 512 else np.random.default_rng(T).choice(T, 384, replace=False)
+    MH.check_route(case, res, tok)
+
+
 def test_pack_reports_w2_values_fp16_cannot_hold():
     """moe_pack_weights stores W2 as fp16.  bf16 weights beyond +-65504 saturate
     and ones finer than fp16's 2^-24 spacing are rounded; the call counts them.

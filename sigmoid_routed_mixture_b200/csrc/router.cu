@@ -61,8 +61,9 @@ int router_stage_bytes(int e_pad) { return rt::A_BYTES + 3 * e_pad * rt::BK * 2;
 struct RouterSmem;
 int router_stages(int e_pad, bool pair);
 
-constexpr int kMaxSplits = 48;       // up to 48 CTAs stream W_r at decode (2 k-blocks each at H 6144)
-constexpr int kRowBatch = 16;        // token rows a CTA reduces and selects at a time after a split
+constexpr int kMaxSplits = 96;       // up to 96 CTAs stream W_r at decode (one k-block each at H 6144)
+constexpr int kRowBatch = 8;         // token rows a CTA reduces and selects at a time after a split
+constexpr int kRankRows = 1;         // a batch of this many rows takes the CTA-wide rank selection
 constexpr int kPairMinTiles = 9;     // from this many 128-token tiles on, CTA pairs
 
 // Upper bound of the split count for any SM count (sizes the partials).
@@ -70,7 +71,7 @@ int router_splits(int T, int H) {
   const int m_tiles = (T + rt::BM - 1) / rt::BM;
   const int kblocks = H / rt::BK;
   int s = 148 / (m_tiles > 0 ? m_tiles : 1);
-  const int max_s = kblocks / 2 > 0 ? kblocks / 2 : 1;
+  const int max_s = kblocks > 0 ? kblocks : 1;
   if (s > max_s) s = max_s;
   if (s > kMaxSplits) s = kMaxSplits;
   if (s < 1) s = 1;
@@ -337,6 +338,115 @@ __device__ __forceinline__ void select_staged(const float *zr, const float *bias
     }
   }
   if (o.margin) o.margin[t] = K < o.E ? kth - nxt : INFINITY;
+}
+
+// Selection for up to kRankRows tokens by the whole CTA (a decode-sized batch
+// after a split, where one warp per token would leave the latency of its
+// rounds exposed).  Thread e < E_PAD owns expert e of every row: key =
+// sigmoid(z) + b.  "a beats b" is the selection order: a larger key, or an
+// equal key and a lower expert.  (1) Each thread counts the experts of its own
+// warp that beat it; the (at most K + 1) it leaves beaten by at most K of them
+// are the warp's candidates, kept in LKC slots (the rest padding that beats
+// nothing).  (2) A candidate's count of the beating candidates of all warps is
+// its rank in the whole row whenever that rank is at most K: an expert that
+// beats it either is a candidate or is beaten by K + 1 candidates of its warp
+// that also beat it, which puts the rank above K anyway.  Ranks 0..K-1 are the
+// K slots in order, rank K gives the margin.  NaN and -inf keys are never
+// selected, as in the other selection paths.  All threads of the CTA call this
+// (it has __syncthreads); rows r < nb sit at zs + r * zstride.
+template <int E_PAD, int LKC>
+__device__ __forceinline__ void select_rank_rows(const float *zs, int zstride, int nb, float my_bias,
+                                                 float *scratch, int t0, int t_step, const RouteOut &o) {
+  constexpr int NWARP = E_PAD / 32;
+  constexpr int R = kRankRows;
+  float *key_s = scratch;                                          // [R][E_PAD]
+  float *cand_k = key_s + R * E_PAD;                               // [R][NWARP][LKC]
+  int *cand_e = reinterpret_cast<int *>(cand_k + R * NWARP * LKC);  // [R][NWARP][LKC]
+  float *sel_k = reinterpret_cast<float *>(cand_e + R * NWARP * LKC);  // [R][17]
+  float *sel_s = sel_k + R * 17;                                   // [R][17]
+  int *sel_e = reinterpret_cast<int *>(sel_s + R * 17);            // [R][17]
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int K = o.K;
+  const bool mine = tid < o.E;
+  float key[R], sv[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    key[r] = -INFINITY;
+    sv[r] = 0.f;
+    if (r < nb && tid < E_PAD) {
+      if (mine) {
+        const float z = zs[r * zstride + tid];
+        if (o.logits) o.logits[static_cast<size_t>(t0 + r * t_step) * o.E + tid] = z;
+        sv[r] = sigmoidf_(z);
+        key[r] = sv[r] + my_bias;
+      }
+      key_s[r * E_PAD + tid] = key[r];
+    }
+  }
+  if (tid < R * 17) {
+    sel_k[tid] = 0.f;
+    sel_s[tid] = 0.f;
+    sel_e[tid] = 0x7fffffff;
+  }
+  __syncthreads();
+  bool cand[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    cand[r] = false;
+    if (r < nb && w < NWARP) {
+      const float4 *wk = reinterpret_cast<const float4 *>(key_s + r * E_PAD + 32 * w);
+      int beaten = 0;
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 k4 = wk[j4];
+        const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) beaten += (4 * j4 + i < lane) ? (kk[i] >= key[r]) : (kk[i] > key[r]);
+      }
+      cand[r] = mine && key[r] > -INFINITY && beaten <= K;  // NaN compares false
+      const unsigned m = __ballot_sync(0xffffffffu, cand[r]);
+      const int n = __popc(m);
+      if (cand[r]) {  // candidates fill slots 0..n-1
+        const int slot = __popc(m & ((1u << lane) - 1u));
+        cand_k[(r * NWARP + w) * LKC + slot] = key[r];
+        cand_e[(r * NWARP + w) * LKC + slot] = tid;
+      }
+      if (lane >= n && lane < LKC) {  // lane l pads slot l
+        cand_k[(r * NWARP + w) * LKC + lane] = -INFINITY;
+        cand_e[(r * NWARP + w) * LKC + lane] = 0x7fffffff;
+      }
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (cand[r]) {
+      int rank = 0;
+#pragma unroll
+      for (int i = 0; i < NWARP * LKC; ++i) {
+        const float kc = cand_k[r * NWARP * LKC + i];
+        const int ec = cand_e[r * NWARP * LKC + i];
+        rank += (kc > key[r]) || (kc == key[r] && ec < tid);
+      }
+      if (rank <= K) {
+        sel_k[r * 17 + rank] = key[r];
+        if (rank < K) {
+          sel_s[r * 17 + rank] = sv[r];
+          sel_e[r * 17 + rank] = tid;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < nb * K) {
+    const int r = tid / K, k = tid - r * K;
+    const int t = t0 + r * t_step;
+    float denom = 0.f;
+    for (int i = 0; i < K; ++i) denom += sel_s[r * 17 + i];
+    o.idx[static_cast<size_t>(t) * K + k] = sel_e[r * 17 + k];
+    o.gate[static_cast<size_t>(t) * K + k] = o.scale * sel_s[r * 17 + k] / denom;
+    if (k == 0 && o.margin) o.margin[t] = K < o.E ? sel_k[r * 17 + K - 1] - sel_k[r * 17 + K] : INFINITY;
+  }
 }
 
 // NH = e_pad / 64: each epilogue thread keeps half a row (e_pad / 2 columns).
@@ -636,6 +746,8 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
     // independent, so a few round trips to L2 cover all S splits); the rows
     // land in shared memory and each warp selects for one row at a time.
     const int splits = gridDim.y;
+    // this thread's expert's bias for the CTA-wide selection, fetched while the grid meets
+    const float my_bias = static_cast<int>(threadIdx.x) < o.E ? o.bias[threadIdx.x] : 0.f;
     if (!grid_barrier(grid_counter, gridDim.x * gridDim.y, err)) return;
     float bias_r[NE];
 #pragma unroll
@@ -701,9 +813,18 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
         }
         __syncthreads();
       }
-      for (int r = warp; r < nb; r += n_warps)
-        select_token<NE>(static_cast<const float *>(zs + r * ZS), bias_r, cta + (r0 + r) * n_ctas, o,
-                         lane);
+      if (nb <= kRankRows) {  // few rows: the whole CTA ranks their experts together
+        if (o.K < 9)
+          select_rank_rows<e_pad, 9>(zs, ZS, nb, my_bias, reinterpret_cast<float *>(part), cta + r0 * n_ctas,
+                                     n_ctas, o);
+        else
+          select_rank_rows<e_pad, 17>(zs, ZS, nb, my_bias, reinterpret_cast<float *>(part), cta + r0 * n_ctas,
+                                      n_ctas, o);
+      } else {
+        for (int r = warp; r < nb; r += n_warps)
+          select_token<NE>(static_cast<const float *>(zs + r * ZS), bias_r, cta + (r0 + r) * n_ctas, o,
+                           lane);
+      }
       __syncthreads();
     }
   }
@@ -732,7 +853,7 @@ static cudaError_t launch_router_kernel(dim3 grid, const CUtensorMap &tmap_x, co
   const int stages = router_stages(e_pad, kPair);
   // the selection stages z rows, the bias and 17-entry lists over the drained ring
   const size_t staged = (static_cast<size_t>(rt::BM) * (e_pad + 4) + e_pad + 2 * 17 * rt::BM) * 4;
-  // after a split: kRowBatch staged rows and up to ceil(48 / 8) group sums of them
+  // after a split: kRowBatch staged rows and up to ceil(kMaxSplits / 8) group sums of them
   const size_t reduced = static_cast<size_t>(kRowBatch) * ((e_pad + 4) + (kMaxSplits + 7) / 8 * e_pad) * 4;
   if (kSplit && reduced > static_cast<size_t>(stages) * (rt::A_BYTES + 3 * (kPair ? e_pad / 2 : e_pad) * rt::BK * 2))
     return cudaErrorInvalidValue;

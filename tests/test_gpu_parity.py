@@ -264,13 +264,16 @@ def test_route_fp32_and_packed_router_agree_bit_exact(T):
     MH.check_route(case, res, tok)
 
 
-@pytest.mark.parametrize("T,E,K", [(300, 64, 3), (9600, 64, 3), (9600, 256, 9), (9600, 256, 16)])
+@pytest.mark.parametrize("T,E,K", [(300, 64, 3), (9600, 64, 3), (9600, 256, 9), (9600, 256, 16),
+                                   (64, 256, 8), (64, 256, 16), (40, 64, 3)])
 def test_equal_keys_take_the_lower_expert(T, E, K):
     """Experts 2j and 2j+1 get the same router row and bias, so their keys are
     exactly equal; the selection must take them in expert order (the lower one
     first, and never the higher one without the lower one).  300 tokens run the
-    split-K router, 9600 the one-pass router with its per-thread lists (K + 1 <=
-    9 and <= 17 entries).  The rest of the routing is checked against the oracle
+    split-K router with one warp per token, 64 and 40 tokens the split-K router
+    whose CTAs rank each token's experts together (a decode batch: at most four
+    tokens per CTA), 9600 the one-pass router with its per-thread lists (K + 1
+    <= 9 and <= 17 entries).  The rest of the routing is checked against the oracle
     where the oracle's margin is clear."""
     w = W.WORKLOADS["glm47flash"].replace(T=T, E=E, K=K, seed=4100 + T + E + K)
     cfg = moe.Config.of(w)

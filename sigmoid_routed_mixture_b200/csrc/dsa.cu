@@ -496,16 +496,44 @@ __device__ __forceinline__ int warp_exclusive_scan(int *cnt, int n) {
   return __shfl_sync(0xffffffffu, incl, 31);
 }
 
+#ifndef SRM_TOPK_FIRST_BITS
+#define SRM_TOPK_FIRST_BITS 8
+#endif
+#ifndef SRM_TOPK_MIN_BLOCKS
+#define SRM_TOPK_MIN_BLOCKS 6
+#endif
+
+// Radix passes of the top-k select: the first takes kTopkFirstBits of the
+// 32-bit key, the others split the rest evenly (8: four passes of 8 bits; 11:
+// passes of 11, 11 and 10 bits).  Measured at 4 x 4096 rows of 4096 keys: 8 bits
+// 0.153 ms, 11 bits 0.355 ms (one warp walks 2048 bins per pass while the
+// others wait), so 8 is the default.
+//
+// The 256-thread form (rows of up to 4096 keys) is compiled for
+// kTopkMinBlocks256 resident CTAs per SM: at 6 (40 registers, a few spilled)
+// it took 0.121 ms against 0.153 ms at 3 (79 registers, no spill) and 0.128 ms
+// at 8; the rows are short, so more CTAs in flight hide each one's load latency.
+constexpr int kTopkFirstBits = SRM_TOPK_FIRST_BITS;
+constexpr int kTopkPasses = kTopkFirstBits == 8 ? 4 : 3;
+__host__ __device__ constexpr int topk_pass_bits(int pass) {
+  return kTopkFirstBits == 8 ? 8 : (pass < 2 ? 11 : 10);
+}
+__host__ __device__ constexpr int topk_pass_shift(int pass) {
+  return kTopkFirstBits == 8 ? 24 - 8 * pass : (pass == 0 ? 21 : (pass == 1 ? 10 : 0));
+}
+static_assert(kTopkFirstBits == 8 || kTopkFirstBits == 11, "first radix pass of 8 or 11 bits");
+constexpr int kTopkMinBlocks256 = SRM_TOPK_MIN_BLOCKS;
+
 // One CTA per query row.  Thread i holds keys j*NT + i (j < VPT) of the
 // visible part of the row in registers (coalesced loads).  Keys are ordered by
 // index as (j, warp, lane), so ranks in index order come from per-(j, warp)
 // counts: ballots, one table, one warp scan.
 template <int NT, int VPT>
-__global__ void __launch_bounds__(NT)
+__global__ void __launch_bounds__(NT, NT == 256 ? kTopkMinBlocks256 : 1)
     dsa_topk_kernel(const float *__restrict__ scores, int T, int S, int n_sel,
                     int32_t *__restrict__ sel) {
   constexpr int NW = NT / 32;
-  __shared__ int hist[256];
+  __shared__ int hist[1 << (kTopkFirstBits > 8 ? kTopkFirstBits : 8)];
   __shared__ int cnt[VPT * NW];
   __shared__ int pick[3];  // digit, keys above it, keys in it
   const int64_t row = blockIdx.x;
@@ -524,26 +552,27 @@ __global__ void __launch_bounds__(NT)
     const int idx = j * NT + tid;
     v[j] = idx < n_vis ? order_key(__ldg(src + idx)) : 0u;
   }
-  // radix select of the n_sel-th largest key, 8 bits at a time
+  // radix select of the n_sel-th largest key, most significant digit first
   uint32_t prefix = 0, pmask = 0;
   int k_rem = n_sel, n_eq = 0;
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += NT) hist[i] = 0;
+  for (int pass = 0; pass < kTopkPasses; ++pass) {
+    const int shift = topk_pass_shift(pass);
+    const int nbins = 1 << topk_pass_bits(pass);
+    const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
+    for (int i = tid; i < nbins; i += NT) hist[i] = 0;
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int idx = j * NT + tid;
-      if (idx < n_vis && (v[j] & pmask) == prefix) atomicAdd(&hist[(v[j] >> shift) & 255u], 1);
+      if (idx < n_vis && (v[j] & pmask) == prefix) atomicAdd(&hist[(v[j] >> shift) & dmask], 1);
     }
     __syncthreads();
-    if (tid < 32) {  // digits 255 .. 0, eight per lane: find the one holding the k_rem-th key
-      int c[8], sum = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        c[i] = hist[255 - (tid * 8 + i)];
-        sum += c[i];
-      }
+    if (tid < 32) {  // digits nbins-1 .. 0, nbins/32 per lane: find the one holding the k_rem-th key
+      const int bpl = nbins >> 5;
+      const int top = nbins - 1 - tid * bpl;  // this lane's digits: top, top-1, ..., top-bpl+1
+      int sum = 0;
+      for (int i = 0; i < bpl; ++i) sum += hist[top - i];
       int incl = sum;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
@@ -551,14 +580,17 @@ __global__ void __launch_bounds__(NT)
         if (tid >= d) incl += x;
       }
       int above = incl - sum;  // keys in higher digits than this lane's first
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (above < k_rem && k_rem <= above + c[i]) {
-          pick[0] = 255 - (tid * 8 + i);
-          pick[1] = above;
-          pick[2] = c[i];
+      if (above < k_rem && k_rem <= incl) {  // exactly one lane
+        for (int i = 0; i < bpl; ++i) {
+          const int c = hist[top - i];
+          if (k_rem <= above + c) {
+            pick[0] = top - i;
+            pick[1] = above;
+            pick[2] = c;
+            break;
+          }
+          above += c;
         }
-        above += c[i];
       }
     }
     __syncthreads();
@@ -566,7 +598,7 @@ __global__ void __launch_bounds__(NT)
     k_rem -= pick[1];
     n_eq = pick[2];
     prefix |= static_cast<uint32_t>(digit) << shift;
-    pmask |= 255u << shift;
+    pmask |= dmask << shift;
     __syncthreads();
     // every key of the chosen bin is taken: the keys to keep are exactly those
     // whose bits so far are >= prefix, and no lower digit is needed (the same

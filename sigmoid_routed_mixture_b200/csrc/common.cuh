@@ -43,6 +43,16 @@ __device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi, bool &sat
 
 __device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + expf(-v)); }
 
+// silu(g) = g * sigmoid(g) from the hardware approximations (ex2 through
+// __expf, rcp.approx): relative error near 2^-21, far below the fp16 rounding
+// (2^-11) of the intermediate it feeds.  For g < -88 the exponential is +inf
+// and the reciprocal 0, so the result is a signed zero.
+__device__ __forceinline__ float silu_approx(float g) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + __expf(-g)));
+  return g * r;
+}
+
 // ----------------------------------------------------------------- errors
 
 __device__ __forceinline__ void record_error(int *err, int code) {

@@ -74,7 +74,11 @@ constexpr int BM = 128;        // weight rows per CTA (tensor-memory lanes)
 constexpr int BK = 64;
 constexpr int TOK_BOX = 32;    // token rows per TMA box of a tail tile
 constexpr int TOK_BOX_BIG = 128;  // token rows per TMA box when a CTA's rows are a multiple of it
-constexpr int THREADS = 192;
+#ifndef SRM_GEMM_EPI_WARPS
+#define SRM_GEMM_EPI_WARPS 4
+#endif
+constexpr int EPI_WARPS = SRM_GEMM_EPI_WARPS;  // 4, or 8 (two per tensor-memory lane quarter)
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int MAX_GROUPS = 257;
 constexpr int MAX_STAGES = 8;
 constexpr int TILE_RING = 4;  // tile ids in flight between the scheduler and the roles
@@ -89,12 +93,12 @@ struct Cfg {
   static constexpr int BT = kPair ? 256 : 64;           // tokens per tile (largest MMA N)
   static constexpr int W_BLOCK = kPair ? 2 * BM : BM;   // weight rows per tile (MMA M)
   static constexpr int TOK_ROWS = kPair ? BT / 2 : BT;  // token rows one CTA holds at most
-  static constexpr int STAGES = kPair ? 6 : 8;
+  static constexpr int STAGES = kPair ? (EPI_WARPS == 8 ? 5 : 6) : (EPI_WARPS == 8 ? 7 : 8);
   static constexpr int A_BYTES = BM * BK * 2;           // 16 KB of weights
   static constexpr int B_BYTES = TOK_ROWS * BK * 2;     // 16 or 8 KB of token rows at most
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BT;  // two accumulators (512 or 128 columns)
-  static constexpr uint32_t EPI_ARRIVALS = kPair ? 8 : 4;
+  static constexpr uint32_t EPI_ARRIVALS = (kPair ? 2 : 1) * EPI_WARPS;
 };
 
 struct Smem {
@@ -112,12 +116,14 @@ struct Smem {
   int total_mtiles;
   int tile_start[MAX_GROUPS + 1];
   int grp_off[MAX_GROUPS + 1];
-  float epi[4][32][33];  // one 32 x 32 transpose buffer per epilogue warp (padded rows)
+  float epi[EPI_WARPS][32][33];  // one 32 x 32 transpose buffer per epilogue warp (padded rows)
 };
 template <bool kPair>
 constexpr size_t smem_bytes() {
   return 1024 /*alignment slack*/ + Cfg<kPair>::STAGES * Cfg<kPair>::STAGE_BYTES + sizeof(Smem);
 }
+static_assert(smem_bytes<true>() <= 232448 && smem_bytes<false>() <= 232448,
+              "grouped GEMM shared memory above 227 KB");
 }  // namespace gg
 
 struct TileCoord {
@@ -489,6 +495,7 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
 #pragma unroll
       for (int m = 0; m < CHUNKS; ++m) {
         if (32 * m >= c.n) break;  // uniform across the warp
+        if (EPI_WARPS == 8 && (m & 1) != ((warp - 2) >> 2)) continue;  // the other warp of this quarter
         uint32_t cv[32];
         tmem_ld32(taddr + 32 * m, cv);
         tmem_ld_wait();
@@ -510,7 +517,7 @@ __device__ __forceinline__ void grouped_gemm_body(const CUtensorMap &tmap_tok, c
             for (int j = 0; j < 8; ++j) {
               const float g0 = buf[lane][2 * j], g1 = buf[lane][2 * j + 1];
               const float u0 = buf[lane][16 + 2 * j], u1 = buf[lane][16 + 2 * j + 1];
-              packed[j] = pack_f16x2_sat(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1, sat);
+              packed[j] = pack_f16x2_sat(silu_approx(g0) * u0, silu_approx(g1) * u1, sat);
             }
             uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) +
                                                    static_cast<size_t>(c.row_base + 32 * m + lane) * p.out_ld +

@@ -766,36 +766,59 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
     const int n_warps = blockDim.x >> 5;
     for (int r0 = 0; r0 < n_rows; r0 += kRowBatch) {
       const int nb = min(kRowBatch, n_rows - r0);
-      for (int i = threadIdx.x; i < groups * nb * V; i += blockDim.x) {
-        const int g = i / (nb * V);
-        const int r = (i - g * nb * V) / V;
-        const int c = i - g * nb * V - r * V;
-        const int t = cta + (r0 + r) * n_ctas;
-        const float4 *q = zp4 + static_cast<size_t>(t) * V + c + static_cast<size_t>(8 * g) * plane4;
-        const int n = min(8, splits - 8 * g);
-        float4 sum;
-        if (n == 8) {
-          float4 a[8];
+      // Up to three items per thread, all their loads issued before any sum, so
+      // one round trip to L2 covers the thread's share of the splits.
+      const int n_items = groups * nb * V;
+      constexpr int U = 3;
+      for (int i0 = threadIdx.x; i0 < n_items; i0 += U * blockDim.x) {
+        float4 a[U][8];
+        int n[U];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) a[k] = __ldcg(q + k * plane4);
-          sum.x = ((a[0].x + a[1].x) + (a[2].x + a[3].x)) + ((a[4].x + a[5].x) + (a[6].x + a[7].x));
-          sum.y = ((a[0].y + a[1].y) + (a[2].y + a[3].y)) + ((a[4].y + a[5].y) + (a[6].y + a[7].y));
-          sum.z = ((a[0].z + a[1].z) + (a[2].z + a[3].z)) + ((a[4].z + a[5].z) + (a[6].z + a[7].z));
-          sum.w = ((a[0].w + a[1].w) + (a[2].w + a[3].w)) + ((a[4].w + a[5].w) + (a[6].w + a[7].w));
-        } else {
-          sum = __ldcg(q);
-          for (int k = 1; k < n; ++k) {
-            const float4 v = __ldcg(q + k * plane4);
-            sum.x += v.x;
-            sum.y += v.y;
-            sum.z += v.z;
-            sum.w += v.w;
+        for (int u = 0; u < U; ++u) {
+          const int i = i0 + u * blockDim.x;
+          n[u] = 0;
+          if (i < n_items) {
+            const int g = i / (nb * V);
+            const int r = (i - g * nb * V) / V;
+            const int c = i - g * nb * V - r * V;
+            const int t = cta + (r0 + r) * n_ctas;
+            const float4 *q = zp4 + static_cast<size_t>(t) * V + c + static_cast<size_t>(8 * g) * plane4;
+            n[u] = min(8, splits - 8 * g);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              if (k < n[u]) a[u][k] = __ldcg(q + k * plane4);
           }
         }
-        if (groups == 1)
-          *reinterpret_cast<float4 *>(zs + r * ZS + 4 * c) = sum;
-        else
-          part[(g * kRowBatch + r) * V + c] = sum;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int i = i0 + u * blockDim.x;
+          if (i >= n_items) continue;
+          const int g = i / (nb * V);
+          const int r = (i - g * nb * V) / V;
+          const int c = i - g * nb * V - r * V;
+          float4 sum;
+          if (n[u] == 8) {
+            sum.x = ((a[u][0].x + a[u][1].x) + (a[u][2].x + a[u][3].x)) + ((a[u][4].x + a[u][5].x) + (a[u][6].x + a[u][7].x));
+            sum.y = ((a[u][0].y + a[u][1].y) + (a[u][2].y + a[u][3].y)) + ((a[u][4].y + a[u][5].y) + (a[u][6].y + a[u][7].y));
+            sum.z = ((a[u][0].z + a[u][1].z) + (a[u][2].z + a[u][3].z)) + ((a[u][4].z + a[u][5].z) + (a[u][6].z + a[u][7].z));
+            sum.w = ((a[u][0].w + a[u][1].w) + (a[u][2].w + a[u][3].w)) + ((a[u][4].w + a[u][5].w) + (a[u][6].w + a[u][7].w));
+          } else {
+            sum = a[u][0];
+#pragma unroll
+            for (int k = 1; k < 8; ++k) {
+              if (k < n[u]) {
+                sum.x += a[u][k].x;
+                sum.y += a[u][k].y;
+                sum.z += a[u][k].z;
+                sum.w += a[u][k].w;
+              }
+            }
+          }
+          if (groups == 1)
+            *reinterpret_cast<float4 *>(zs + r * ZS + 4 * c) = sum;
+          else
+            part[(g * kRowBatch + r) * V + c] = sum;
+        }
       }
       __syncthreads();
       if (groups > 1) {

@@ -264,18 +264,19 @@ def test_route_fp32_and_packed_router_agree_bit_exact(T):
     MH.check_route(case, res, tok)
 
 
-@pytest.mark.parametrize("T,E,K", [(300, 64, 3), (9600, 64, 3), (9600, 256, 9), (9600, 256, 16),
-                                   (64, 256, 8), (64, 256, 16), (40, 64, 3)])
-def test_equal_keys_take_the_lower_expert(T, E, K):
+@pytest.mark.parametrize("T,E,K,H", [(300, 64, 3, 2048), (9600, 64, 3, 2048), (9600, 256, 9, 2048),
+                                     (9600, 256, 16, 2048), (64, 256, 8, 2048), (64, 256, 16, 2048),
+                                     (40, 64, 3, 2048), (64, 256, 8, 6144), (64, 256, 16, 6144)])
+def test_equal_keys_take_the_lower_expert(T, E, K, H):
     """Experts 2j and 2j+1 get the same router row and bias, so their keys are
     exactly equal; the selection must take them in expert order (the lower one
-    first, and never the higher one without the lower one).  300 tokens run the
-    split-K router with one warp per token, 64 and 40 tokens the split-K router
-    whose CTAs rank each token's experts together (a decode batch: at most four
-    tokens per CTA), 9600 the one-pass router with its per-thread lists (K + 1
-    <= 9 and <= 17 entries).  The rest of the routing is checked against the oracle
+    first, and never the higher one without the lower one).  Split-K router:
+    one warp per token where a CTA holds several tokens (300 tokens; 64 at
+    H 2048, 32 splits), the CTA-wide ranking where it holds one (64 tokens at
+    H 6144, 96 splits; 40 tokens: both kinds of CTA).  9600 tokens: the
+    one-pass router with its per-thread lists (K + 1 <= 9 and <= 17 entries).  The rest of the routing is checked against the oracle
     where the oracle's margin is clear."""
-    w = W.WORKLOADS["glm47flash"].replace(T=T, E=E, K=K, seed=4100 + T + E + K)
+    w = W.WORKLOADS["glm47flash"].replace(T=T, E=E, K=K, H=H, seed=4100 + T + E + K + H)
     cfg = moe.Config.of(w)
     x, w_r, b = W.router_inputs(w)
     w_r[1::2] = w_r[0::2]

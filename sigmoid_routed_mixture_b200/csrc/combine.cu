@@ -17,6 +17,16 @@
 namespace srm {
 
 // 8 fp16 values (16 bytes) added to the fp32 sums
+__device__ __forceinline__ void add8v(float (&acc)[8], const uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[k]));
+    acc[2 * k] += f.x;
+    acc[2 * k + 1] += f.y;
+  }
+}
+
 __device__ __forceinline__ void add8(float (&acc)[8], const uint16_t *src) {
   const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(src));
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -28,6 +38,9 @@ __device__ __forceinline__ void add8(float (&acc)[8], const uint16_t *src) {
   }
 }
 
+// KK > 0: the kernel for K = KK, every slot row's load issued before the sums
+// (more loads in flight per thread); KK = 0: any K.  Same summation order.
+template <int KK>
 __global__ void __launch_bounds__(256)
     combine_kernel(const uint16_t *__restrict__ Y, const uint16_t *__restrict__ residual,
                    uint16_t *__restrict__ y, int T, int H, int K, int has_shared) {
@@ -39,8 +52,18 @@ __global__ void __launch_bounds__(256)
     const int64_t t = i / vecs;
     const int64_t col = (i - t * vecs) * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k < K; ++k) add8(acc, Y + (t * K + k) * H + col);
-    if (has_shared) add8(acc, Y + (tk + t) * H + col);
+    if (KK > 0) {
+      uint4 v[KK + 1];
+#pragma unroll
+      for (int k = 0; k < KK; ++k) v[k] = __ldcs(reinterpret_cast<const uint4 *>(Y + (t * KK + k) * H + col));
+      if (has_shared) v[KK] = __ldcs(reinterpret_cast<const uint4 *>(Y + (tk + t) * H + col));
+#pragma unroll
+      for (int k = 0; k < KK; ++k) add8v(acc, v[k]);
+      if (has_shared) add8v(acc, v[KK]);
+    } else {
+      for (int k = 0; k < K; ++k) add8(acc, Y + (t * K + k) * H + col);
+      if (has_shared) add8(acc, Y + (tk + t) * H + col);
+    }
     if (residual) {  // x_{n+1} = x'_n + Delta_ffn: the block output added to the residual stream
       const uint4 r = *reinterpret_cast<const uint4 *>(residual + t * H + col);
       const uint32_t w[4] = {r.x, r.y, r.z, r.w};
@@ -65,7 +88,12 @@ cudaError_t launch_combine(const uint16_t *Y, const uint16_t *residual, uint16_t
   int64_t blocks = (total + 255) / 256;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   if (blocks > cap) blocks = cap;
-  combine_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(Y, residual, y, T, H, K, has_shared);
+  if (K == 8)
+    combine_kernel<8><<<static_cast<int>(blocks), 256, 0, stream>>>(Y, residual, y, T, H, K, has_shared);
+  else if (K == 4)
+    combine_kernel<4><<<static_cast<int>(blocks), 256, 0, stream>>>(Y, residual, y, T, H, K, has_shared);
+  else
+    combine_kernel<0><<<static_cast<int>(blocks), 256, 0, stream>>>(Y, residual, y, T, H, K, has_shared);
   return cudaGetLastError();
 }
 

@@ -22,15 +22,18 @@
 //      chains promoted to fp32 registers (see below), then the selection in
 //      the same kernel:
 //        - one CTA per 128 tokens (no split of H): the epilogue warps stage
-//          their fp32 z rows in shared memory (the drained operand ring) and
-//          each warp selects for its tokens: s, keys, K rounds of a warp
-//          arg-max (key descending, index ascending), one more round for the
-//          margin, gates.  z never reaches global memory unless asked for.
+//          their fp32 z rows in shared memory (the drained operand ring); one
+//          thread per (token, half of the experts) builds a sorted top-(K+1)
+//          list of (key, expert) in registers, the halves merge, and the
+//          first half's thread writes experts, gates and margin.  z never
+//          reaches global memory unless asked for.
 //        - few 128-token tiles (decode): the H range is split over S CTAs;
-//          each writes fp32 partial logits, all CTAs of the grid (at most one
-//          per SM, so all resident together) meet at a bounded grid barrier,
-//          then every CTA takes some tokens, sums the S partials in a fixed
-//          order (deterministic) and selects.
+//          each writes fp32 partial logits (whole rows, through shared
+//          memory), all CTAs of the grid (at most one per SM, so all resident
+//          together) meet at a bounded grid barrier, then every CTA takes
+//          some tokens, sums the S partials in a fixed order (deterministic)
+//          and selects: a CTA-wide ranking for a single token, otherwise K + 1
+//          rounds of a warp arg-max (key descending, index ascending) per token.
 #include <cuda.h>
 #include <math.h>
 

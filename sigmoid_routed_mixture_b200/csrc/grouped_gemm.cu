@@ -16,15 +16,18 @@
 // count, can be any multiple of 16 up to 256: a group whose row count is not a
 // multiple of 256 pads its last tile to 16 rows, not to 256 (with tokens on
 // the M side, 16.8% of the rows of the 16384-token GLM-5 block were padding).
+// (Measured on B200: a k-block of a pair tile takes about as long at 16 tokens
+// as at 256, so such a tail still costs about a full tile's time.)
 //
 //   kUp   : for every group g (routed experts 0..E-1, shared expert E), the
 //           packed W13_g rows against its token rows (xs: token rows in
 //           expert-sorted order, gather.cu).  W13 is packed in units of 32
-//           rows, 16 gate rows then the 16 matching up rows, so TMEM lanes
-//           l and l + 16 of a warp hold gate and up of one feature: one
-//           shuffle pairs them, epilogue h = silu(g) * u -> fp16 h[row][I]
-//           (three more mantissa bits than bf16 at the same tensor-core rate;
-//           |h| saturates at 65504, flagged MOE_ERR_RANGE).
+//           rows, 16 gate rows then the 16 matching up rows, so a warp's 32
+//           TMEM lanes hold gate and up of 16 features; each 32-token chunk
+//           is transposed through shared memory so that a lane holds one
+//           token's 16 gate and 16 up values: h = silu(g) * u -> fp16
+//           h[row][I] (three more mantissa bits than bf16 at the same
+//           tensor-core rate; |h| saturates at 65504, flagged MOE_ERR_RANGE).
 //   kDown : W2_g rows (output features, fp16; an exact conversion of bf16
 //           weights in fp16's normal range) against the token rows of h
 //           (fp16); epilogue multiplies by the routing gate (1 for the shared
@@ -33,19 +36,20 @@
 //
 // Tiling: a work tile is (group, weight block of 256 rows, token block of up
 // to 256 rows).  On a CTA pair each CTA loads 128 of the weight rows and half
-// of the tile's token rows (N/2, in TMA boxes of 32 rows), the leader issues
+// of the tile's token rows (N/2: one 128-row TMA box for a full tile, boxes of
+// 32 rows for a group's last, partial one), the leader issues
 // tcgen05.mma.cta_group::2 with M = 256 and N = the tile's token count
 // rounded up to 16, and each CTA receives its 128 weight rows x N tokens in
 // its own tensor memory.  K loop in steps of 64 (one 128-byte swizzle atom), a
-// 6-stage TMA ring per CTA (4 for single CTAs), two accumulators of 256
+// 6-stage TMA ring per CTA (8 for single CTAs), two accumulators of 256
 // columns so the epilogue of one tile overlaps the main loop of the next.
 // Warp roles (6 warps per CTA):
 //   warp 0: TMA producer (one lane issues the CTA's weight and token loads)
 //   warp 1: tensor-memory allocation; in the leader also single-thread MMA issue
 //   warps 2-5: epilogue (tensor memory -> registers -> global)
 // Work tiles are ordered (group, weight block, token block), token block
-// fastest; a unit (CTA pair or single CTA) takes its next tile from a global
-// atomic counter when it is ready for one, so the tiles that share a weight
+// fastest; a unit (CTA pair or single CTA) takes its tiles from a global
+// atomic counter (the leader keeps two ids published ahead), so the tiles that share a weight
 // block start together and read it from DRAM once; the per-group token-block
 // counts come from the group offsets on the device, so the host never
 // synchronises.

@@ -349,8 +349,9 @@ __device__ __forceinline__ void select_staged(const float *zr, const float *bias
 // sigmoid(z) + b.  "a beats b" is the selection order: a larger key, or an
 // equal key and a lower expert.  (1) Each thread counts the experts of its own
 // warp that beat it; the (at most K + 1) it leaves beaten by at most K of them
-// are the warp's candidates, kept in LKC slots (the rest padding that beats
-// nothing).  (2) A candidate's count of the beating candidates of all warps is
+// are the warp's candidates, kept in LKS slots (LKC rounded up to a multiple
+// of four, for 16-byte loads; the rest padding that beats nothing).  (2) A
+// candidate's count of the beating candidates of all warps is
 // its rank in the whole row whenever that rank is at most K: an expert that
 // beats it either is a candidate or is beaten by K + 1 candidates of its warp
 // that also beat it, which puts the rank above K anyway.  Ranks 0..K-1 are the
@@ -362,10 +363,11 @@ __device__ __forceinline__ void select_rank_rows(const float *zs, int zstride, i
                                                  float *scratch, int t0, int t_step, const RouteOut &o) {
   constexpr int NWARP = E_PAD / 32;
   constexpr int R = kRankRows;
+  constexpr int LKS = (LKC + 3) / 4 * 4;                           // slots per warp (16-byte rows)
   float *key_s = scratch;                                          // [R][E_PAD]
-  float *cand_k = key_s + R * E_PAD;                               // [R][NWARP][LKC]
-  int *cand_e = reinterpret_cast<int *>(cand_k + R * NWARP * LKC);  // [R][NWARP][LKC]
-  float *sel_k = reinterpret_cast<float *>(cand_e + R * NWARP * LKC);  // [R][17]
+  float *cand_k = key_s + R * E_PAD;                               // [R][NWARP][LKS]
+  int *cand_e = reinterpret_cast<int *>(cand_k + R * NWARP * LKS);  // [R][NWARP][LKS]
+  float *sel_k = reinterpret_cast<float *>(cand_e + R * NWARP * LKS);  // [R][17]
   float *sel_s = sel_k + R * 17;                                   // [R][17]
   int *sel_e = reinterpret_cast<int *>(sel_s + R * 17);            // [R][17]
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -411,12 +413,12 @@ __device__ __forceinline__ void select_rank_rows(const float *zs, int zstride, i
       const int n = __popc(m);
       if (cand[r]) {  // candidates fill slots 0..n-1
         const int slot = __popc(m & ((1u << lane) - 1u));
-        cand_k[(r * NWARP + w) * LKC + slot] = key[r];
-        cand_e[(r * NWARP + w) * LKC + slot] = tid;
+        cand_k[(r * NWARP + w) * LKS + slot] = key[r];
+        cand_e[(r * NWARP + w) * LKS + slot] = tid;
       }
-      if (lane >= n && lane < LKC) {  // lane l pads slot l
-        cand_k[(r * NWARP + w) * LKC + lane] = -INFINITY;
-        cand_e[(r * NWARP + w) * LKC + lane] = 0x7fffffff;
+      if (lane >= n && lane < LKS) {  // lane l pads slot l
+        cand_k[(r * NWARP + w) * LKS + lane] = -INFINITY;
+        cand_e[(r * NWARP + w) * LKS + lane] = 0x7fffffff;
       }
     }
   }
@@ -425,11 +427,16 @@ __device__ __forceinline__ void select_rank_rows(const float *zs, int zstride, i
   for (int r = 0; r < R; ++r) {
     if (cand[r]) {
       int rank = 0;
+      const float4 *ck = reinterpret_cast<const float4 *>(cand_k + r * NWARP * LKS);
+      const int4 *ce = reinterpret_cast<const int4 *>(cand_e + r * NWARP * LKS);
 #pragma unroll
-      for (int i = 0; i < NWARP * LKC; ++i) {
-        const float kc = cand_k[r * NWARP * LKC + i];
-        const int ec = cand_e[r * NWARP * LKC + i];
-        rank += (kc > key[r]) || (kc == key[r] && ec < tid);
+      for (int i = 0; i < NWARP * LKS / 4; ++i) {
+        const float4 kc = ck[i];
+        const int4 ec = ce[i];
+        rank += (kc.x > key[r]) || (kc.x == key[r] && ec.x < tid);
+        rank += (kc.y > key[r]) || (kc.y == key[r] && ec.y < tid);
+        rank += (kc.z > key[r]) || (kc.z == key[r] && ec.z < tid);
+        rank += (kc.w > key[r]) || (kc.w == key[r] && ec.w < tid);
       }
       if (rank <= K) {
         sel_k[r * 17 + rank] = key[r];

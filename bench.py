@@ -190,7 +190,8 @@ def kernel_source_hash(kernel):
 
 def measured_traffic(workload, kernel):
     """DRAM bytes per launch from a committed ncu capture (the `traffic` lines of
-    profiles/*.md), or None when the kernel's sources changed since it was taken."""
+    the profile summaries), or None when the kernel's sources changed since it
+    was taken."""
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
         return None

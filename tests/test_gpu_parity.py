@@ -144,6 +144,25 @@ def test_glm5_full_size_sampled(name):
     free()
 
 
+def test_glm5_largest_batch_sampled():
+    """65536 GLM-5 tokens (four times the benchmark's batch, about 38 GB on the
+    device): 512 router tiles in several waves, 524288 assignments in the
+    permutation, a shared-expert group of 256 token blocks walked in chunks, and
+    the index arithmetic of every stage at its largest.  Router on a 1024-token
+    subset, permutation on all tokens, output on a seeded sample."""
+    w = W.WORKLOADS["glm5_prefill"].replace(T=65536, seed=4500)
+    case = MH.Case(w)
+    res = case.run()
+    assert res["err"] == 0
+    sub = np.sort(np.random.default_rng(2).choice(w.T, size=1024, replace=False))
+    near = MH.check_route(case, res, sub)
+    assert near < 0.05 * len(sub)
+    MH.check_permute(case, res)
+    MH.check_forward(case, res, MH.sample_tokens(res, w.T, 6))
+    del case, res
+    free()
+
+
 def test_ablation_uses_gates_as_given():
     """Zeroing the gates of every slot that chose expert 3 (and only those)
     changes the output exactly by those slots; zero gates leave the shared

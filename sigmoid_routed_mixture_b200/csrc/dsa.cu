@@ -525,17 +525,24 @@ static_assert(kTopkFirstBits == 8 || kTopkFirstBits == 11, "first radix pass of 
 constexpr int kTopkMinBlocks256 = SRM_TOPK_MIN_BLOCKS;
 
 // One CTA per query row.  Thread i holds keys j*NT + i (j < VPT) of the
-// visible part of the row in registers (coalesced loads).  Keys are ordered by
-// index as (j, warp, lane), so ranks in index order come from per-(j, warp)
-// counts: ballots, one table, one warp scan.
+// visible part of the row in registers (coalesced loads); the slots past the
+// visible keys hold key 0, below the key of every float but the one NaN whose
+// bits are all set (order_key(-inf) is 0x007fffff), so the radix passes and
+// the compaction need no bounds test: the hidden slots are taken out of bin 0
+// of any pass whose prefix is 0, rank after every visible key of equal value
+// (their indices are larger) and, if taken at all, only past position n_sel.
+// Keys are ordered by index as (j, warp, lane), so ranks in index order come
+// from per-(j, warp) counts: ballots, one table, one warp scan.
 template <int NT, int VPT>
 __global__ void __launch_bounds__(NT, NT == 256 ? kTopkMinBlocks256 : 1)
     dsa_topk_kernel(const float *__restrict__ scores, int T, int S, int n_sel,
                     int32_t *__restrict__ sel) {
   constexpr int NW = NT / 32;
-  __shared__ int hist[1 << (kTopkFirstBits > 8 ? kTopkFirstBits : 8)];
+  constexpr int HB = 1 << (kTopkFirstBits > 8 ? kTopkFirstBits : 8);
+  // two histograms: a pass counts into one while it clears the other for the next
+  __shared__ int hist[2][HB];
   __shared__ int cnt[VPT * NW];
-  __shared__ int pick[3];  // digit, keys above it, keys in it
+  __shared__ int pick[2][3];  // per pass parity: digit, keys above it, keys in it
   const int64_t row = blockIdx.x;
   const int t = static_cast<int>(row % T);
   const int n_vis = S - T + t + 1;  // keys this query sees
@@ -552,27 +559,35 @@ __global__ void __launch_bounds__(NT, NT == 256 ? kTopkMinBlocks256 : 1)
     const int idx = j * NT + tid;
     v[j] = idx < n_vis ? order_key(__ldg(src + idx)) : 0u;
   }
+  const int n_hid = VPT * NT - n_vis;
+  for (int i = tid; i < 2 * HB; i += NT) (&hist[0][0])[i] = 0;
+  __syncthreads();
   // radix select of the n_sel-th largest key, most significant digit first
   uint32_t prefix = 0, pmask = 0;
   int k_rem = n_sel, n_eq = 0;
 #pragma unroll 1
   for (int pass = 0; pass < kTopkPasses; ++pass) {
+    int *h = hist[pass & 1];
     const int shift = topk_pass_shift(pass);
     const int nbins = 1 << topk_pass_bits(pass);
     const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
-    for (int i = tid; i < nbins; i += NT) hist[i] = 0;
-    __syncthreads();
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      const int idx = j * NT + tid;
-      if (idx < n_vis && (v[j] & pmask) == prefix) atomicAdd(&hist[(v[j] >> shift) & dmask], 1);
+    for (int j = 0; j < VPT; ++j)
+      if ((v[j] & pmask) == prefix) atomicAdd(&h[(v[j] >> shift) & dmask], 1);
+    // the next pass's histogram: its last reader was the previous pass's
+    // search, which ended before that pass's second barrier
+    if (pass + 1 < kTopkPasses) {
+      int *hn = hist[(pass + 1) & 1];
+      for (int i = tid; i < (1 << topk_pass_bits(pass + 1)); i += NT) hn[i] = 0;
     }
     __syncthreads();
     if (tid < 32) {  // digits nbins-1 .. 0, nbins/32 per lane: find the one holding the k_rem-th key
       const int bpl = nbins >> 5;
       const int top = nbins - 1 - tid * bpl;  // this lane's digits: top, top-1, ..., top-bpl+1
+      const int hid0 = prefix == 0u ? n_hid : 0;  // hidden slots counted in bin 0
       int sum = 0;
-      for (int i = 0; i < bpl; ++i) sum += hist[top - i];
+      for (int i = 0; i < bpl; ++i) sum += h[top - i];
+      if (top - bpl + 1 == 0) sum -= hid0;
       int incl = sum;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
@@ -582,11 +597,11 @@ __global__ void __launch_bounds__(NT, NT == 256 ? kTopkMinBlocks256 : 1)
       int above = incl - sum;  // keys in higher digits than this lane's first
       if (above < k_rem && k_rem <= incl) {  // exactly one lane
         for (int i = 0; i < bpl; ++i) {
-          const int c = hist[top - i];
+          const int c = h[top - i] - (top - i == 0 ? hid0 : 0);
           if (k_rem <= above + c) {
-            pick[0] = top - i;
-            pick[1] = above;
-            pick[2] = c;
+            pick[pass & 1][0] = top - i;
+            pick[pass & 1][1] = above;
+            pick[pass & 1][2] = c;
             break;
           }
           above += c;
@@ -594,12 +609,11 @@ __global__ void __launch_bounds__(NT, NT == 256 ? kTopkMinBlocks256 : 1)
       }
     }
     __syncthreads();
-    const int digit = pick[0];
-    k_rem -= pick[1];
-    n_eq = pick[2];
+    const int digit = pick[pass & 1][0];
+    k_rem -= pick[pass & 1][1];
+    n_eq = pick[pass & 1][2];
     prefix |= static_cast<uint32_t>(digit) << shift;
     pmask |= dmask << shift;
-    __syncthreads();
     // every key of the chosen bin is taken: the keys to keep are exactly those
     // whose bits so far are >= prefix, and no lower digit is needed (the same
     // value for the whole CTA, so the exit is uniform)
@@ -611,40 +625,35 @@ __global__ void __launch_bounds__(NT, NT == 256 ? kTopkMinBlocks256 : 1)
   const unsigned lt = (1u << lane) - 1u;
   uint64_t eq_take = ~uint64_t(0);  // bit j: this thread's key j, if equal, is taken
   if (n_eq > k_rem) {  // ties across the threshold: rank the equal keys by index
+    unsigned me[VPT];
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && (v[j] & pmask) == prefix);
-      if (lane == 0) cnt[j * NW + warp] = __popc(m);
+      me[j] = __ballot_sync(0xffffffffu, (v[j] & pmask) == prefix);
+      if (lane == 0) cnt[j * NW + warp] = __popc(me[j]);
     }
     __syncthreads();
     if (warp == 0) warp_exclusive_scan(cnt, VPT * NW);
     __syncthreads();
     eq_take = 0;
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      const unsigned m = __ballot_sync(0xffffffffu, j * NT + tid < n_vis && (v[j] & pmask) == prefix);
-      if (cnt[j * NW + warp] + __popc(m & lt) < k_rem) eq_take |= uint64_t(1) << j;
-    }
+    for (int j = 0; j < VPT; ++j)
+      if (cnt[j * NW + warp] + __popc(me[j] & lt) < k_rem) eq_take |= uint64_t(1) << j;
     __syncthreads();
   }
-  uint64_t take_bits = 0;
+  unsigned mk[VPT];  // per j: the warp's lanes whose key j is taken
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const uint32_t vm = v[j] & pmask;
-    const bool take = j * NT + tid < n_vis && (vm > prefix || (vm == prefix && ((eq_take >> j) & 1u)));
-    const unsigned m = __ballot_sync(0xffffffffu, take);
-    if (take) take_bits |= uint64_t(1) << j;
-    if (lane == 0) cnt[j * NW + warp] = __popc(m);
+    mk[j] = __ballot_sync(0xffffffffu, vm > prefix || (vm == prefix && ((eq_take >> j) & 1u)));
+    if (lane == 0) cnt[j * NW + warp] = __popc(mk[j]);
   }
   __syncthreads();
   if (warp == 0) warp_exclusive_scan(cnt, VPT * NW);
   __syncthreads();
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
-    const bool take = (take_bits >> j) & 1u;
-    const unsigned m = __ballot_sync(0xffffffffu, take);
-    const int pos = cnt[j * NW + warp] + __popc(m & lt);
-    if (take && pos < n_sel) out[pos] = j * NT + tid;
+    const int pos = cnt[j * NW + warp] + __popc(mk[j] & lt);
+    if (((mk[j] >> lane) & 1u) && pos < n_sel) out[pos] = j * NT + tid;
   }
 }
 

@@ -193,6 +193,33 @@ def test_topk_alone_on_given_scores_is_exact():
             assert np.array_equal(got[b, t], want), (b, t)
 
 
+@pytest.mark.parametrize("S,T", [(4000, 4), (5000, 3), (20000, 2)])
+def test_topk_threshold_among_the_lowest_keys(S, T):
+    """Rows whose topk-th score is -inf or the most negative finite float, so the
+    radix passes' leading digits are 0 (the bin the padding past the visible keys
+    also falls in): visible -inf scores before hidden keys, ties by index, on each
+    register layout of the top-k."""
+    rng = np.random.default_rng(S)
+    sc = np.full((1, T, S), -np.inf, dtype=np.float32)
+    lowest = np.float32(-3.4e38)
+    for t in range(T):
+        n_vis = S - T + t + 1
+        n_fin = [1000, 1500, 700, 2047][t % 4]
+        pick = rng.permutation(n_vis)
+        sc[0, t, pick[:n_fin]] = rng.standard_normal(n_fin).astype(np.float32)
+        if t % 2 == 1:  # a run of the most negative finite value straddling the threshold
+            sc[0, t, pick[n_fin:n_fin + 900]] = lowest
+    cfg = dsa.Config(1, T, S, topk=2048)
+    ws = dsa.workspace(cfg)
+    got = dsa.topk(cfg, torch.from_numpy(sc).cuda(), ws).cpu().numpy()
+    for t in range(T):
+        pos = S - T + t
+        row = np.full(S, -np.inf)
+        row[:pos + 1] = sc[0, t, :pos + 1]
+        want, _, _ = O.dsa_select(row, 2048)
+        assert np.array_equal(got[0, t], want), (S, t)
+
+
 def test_large_cache_topk_variants():
     """Key counts for each register layout of the top-k (<= 4096, <= 16384, <= 32768)."""
     rng = np.random.default_rng(6)

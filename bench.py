@@ -597,8 +597,13 @@ def run_dsa(args, world, rank, dist, dev):
 
 # ------------------------------------------------------------------ router stage
 
-ROUTER_WORKLOADS = {"router_glm5_prefill": "glm5_prefill", "router_glm5_decode": "glm5_decode"}
-ROUTER_METRIC = "router tokens/s (GLM-5 shape: 256 experts top-8, H 6144, 1 B200)"
+ROUTER_WORKLOADS = {"router_glm5_prefill": "glm5_prefill", "router_glm5_decode": "glm5_decode",
+                    "router_glm47flash": "glm47flash"}
+
+
+def router_metric(w):
+    shape = "GLM-5 shape" if w.name.startswith("glm5") else "GLM-4.7-Flash shape"
+    return "router tokens/s (%s: %d experts top-%d, H %d, 1 B200)" % (shape, w.E, w.K, w.H)
 
 
 def run_router(args, world, rank, dist, dev):
@@ -665,7 +670,7 @@ def run_router(args, world, rank, dist, dev):
                 "unit": "GB/s", "peak_kind": "copy bandwidth, " + pk["source"], "algorithmic_per_launch": bytes_}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = None
-    line = {"metric": ROUTER_METRIC, "value": w.T * world * args.steps / (t_max / 1e3), "unit": UNIT,
+    line = {"metric": router_metric(w), "value": w.T * world * args.steps / (t_max / 1e3), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x, fp32 W_r (3-part split)",
             "data": "synthetic (seeded)", "config": dict(workload_config(w, argparse.Namespace(gpus=world)),

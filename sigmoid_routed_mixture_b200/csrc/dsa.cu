@@ -500,28 +500,31 @@ __device__ __forceinline__ int warp_exclusive_scan(int *cnt, int n) {
 #define SRM_TOPK_FIRST_BITS 8
 #endif
 #ifndef SRM_TOPK_MIN_BLOCKS
-#define SRM_TOPK_MIN_BLOCKS 6
+#define SRM_TOPK_MIN_BLOCKS 8
 #endif
 
-// Radix passes of the top-k select: the first takes kTopkFirstBits of the
-// 32-bit key, the others split the rest evenly (8: four passes of 8 bits; 11:
-// passes of 11, 11 and 10 bits).  Measured at 4 x 4096 rows of 4096 keys: 8 bits
-// 0.153 ms, 11 bits 0.355 ms (one warp walks 2048 bins per pass while the
-// others wait), so 8 is the default.
+// Radix passes of the top-k select: the first takes FB bits of the 32-bit key,
+// the others split the rest evenly (8: four passes of 8 bits, the digit found
+// by one warp; 11: passes of 11, 11 and 10 bits, the digit found by a scan over
+// the whole CTA).  Measured on one B200, rows of up to 4096 keys (4 x 4096
+// queries): 0.091 ms with 8 bits, 0.104 ms with 11 (the CTA-wide search costs
+// more than the pass it saves; with the 2048 bins walked by one warp it was
+// 0.355 ms); rows of 32768 keys (64 decode queries): 24.6 us either way.  So 8
+// is the default and SRM_TOPK_FIRST_BITS=11 a compile-time alternative.
 //
 // The 256-thread form (rows of up to 4096 keys) is compiled for
-// kTopkMinBlocks256 resident CTAs per SM: at 6 (40 registers, a few spilled)
-// it took 0.121 ms against 0.153 ms at 3 (79 registers, no spill) and 0.128 ms
-// at 8; the rows are short, so more CTAs in flight hide each one's load latency.
-constexpr int kTopkFirstBits = SRM_TOPK_FIRST_BITS;
-constexpr int kTopkPasses = kTopkFirstBits == 8 ? 4 : 3;
-__host__ __device__ constexpr int topk_pass_bits(int pass) {
-  return kTopkFirstBits == 8 ? 8 : (pass < 2 ? 11 : 10);
+// kTopkMinBlocks256 resident CTAs per SM: 5 / 6 / 8 of them took 0.097 /
+// 0.091 / 0.089 ms (at 8: 32 registers, some spilled; before the passes were
+// unrolled, 3 / 6 / 8 took 0.153 / 0.121 / 0.128 ms); the rows are short, so
+// more CTAs in flight hide each one's load latency.
+__host__ __device__ constexpr int topk_passes(int fb) { return fb == 8 ? 4 : 3; }
+__host__ __device__ constexpr int topk_pass_bits(int fb, int pass) {
+  return fb == 8 ? 8 : (pass < 2 ? 11 : 10);
 }
-__host__ __device__ constexpr int topk_pass_shift(int pass) {
-  return kTopkFirstBits == 8 ? 24 - 8 * pass : (pass == 0 ? 21 : (pass == 1 ? 10 : 0));
+__host__ __device__ constexpr int topk_pass_shift(int fb, int pass) {
+  return fb == 8 ? 24 - 8 * pass : (pass == 0 ? 21 : (pass == 1 ? 10 : 0));
 }
-static_assert(kTopkFirstBits == 8 || kTopkFirstBits == 11, "first radix pass of 8 or 11 bits");
+static_assert(SRM_TOPK_FIRST_BITS == 8 || SRM_TOPK_FIRST_BITS == 11, "first radix pass of 8 or 11 bits");
 constexpr int kTopkMinBlocks256 = SRM_TOPK_MIN_BLOCKS;
 
 // One CTA per query row.  Thread i holds keys j*NT + i (j < VPT) of the
@@ -533,23 +536,30 @@ constexpr int kTopkMinBlocks256 = SRM_TOPK_MIN_BLOCKS;
 // (their indices are larger) and, if taken at all, only past position n_sel.
 // Keys are ordered by index as (j, warp, lane), so ranks in index order come
 // from per-(j, warp) counts: ballots, one table, one warp scan.
-template <int NT, int VPT>
+template <int NT, int VPT, int FB>
 __global__ void __launch_bounds__(NT, NT == 256 ? kTopkMinBlocks256 : 1)
     dsa_topk_kernel(const float *__restrict__ scores, int T, int S, int n_sel,
                     int32_t *__restrict__ sel) {
   constexpr int NW = NT / 32;
-  constexpr int HB = 1 << (kTopkFirstBits > 8 ? kTopkFirstBits : 8);
+  constexpr int HB = 1 << FB;
+  constexpr int kPasses = topk_passes(FB);
   // two histograms: a pass counts into one while it clears the other for the next
   __shared__ int hist[2][HB];
   __shared__ int cnt[VPT * NW];
   __shared__ int pick[2][3];  // per pass parity: digit, keys above it, keys in it
+  __shared__ int wtot[NW];    // per warp: keys in its digits (CTA-wide search)
   const int64_t row = blockIdx.x;
   const int t = static_cast<int>(row % T);
   const int n_vis = S - T + t + 1;  // keys this query sees
   int32_t *out = sel + row * n_sel;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (n_vis <= n_sel) {  // every visible key, then the lowest-index hidden ones
-    for (int j = tid; j < n_sel; j += NT) out[j] = j;
+    if ((n_sel & 3) == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
+      int4 *out4 = reinterpret_cast<int4 *>(out);
+      for (int j = tid; j < n_sel / 4; j += NT) out4[j] = make_int4(4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3);
+    } else {
+      for (int j = tid; j < n_sel; j += NT) out[j] = j;
+    }
     return;
   }
   const float *src = scores + row * S;
@@ -565,46 +575,86 @@ __global__ void __launch_bounds__(NT, NT == 256 ? kTopkMinBlocks256 : 1)
   // radix select of the n_sel-th largest key, most significant digit first
   uint32_t prefix = 0, pmask = 0;
   int k_rem = n_sel, n_eq = 0;
-#pragma unroll 1
-  for (int pass = 0; pass < kTopkPasses; ++pass) {
+  // unrolled: each pass's shift and bin count are constants, and the first
+  // pass's prefix test (against prefix 0 under mask 0) folds away (4 x 4096 rows,
+  // six CTAs per SM: 0.103 ms with the passes in a loop, 0.091 ms unrolled)
+#pragma unroll
+  for (int pass = 0; pass < kPasses; ++pass) {
     int *h = hist[pass & 1];
-    const int shift = topk_pass_shift(pass);
-    const int nbins = 1 << topk_pass_bits(pass);
+    const int shift = topk_pass_shift(FB, pass);
+    const int nbins = 1 << topk_pass_bits(FB, pass);
     const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
 #pragma unroll
     for (int j = 0; j < VPT; ++j)
       if ((v[j] & pmask) == prefix) atomicAdd(&h[(v[j] >> shift) & dmask], 1);
     // the next pass's histogram: its last reader was the previous pass's
     // search, which ended before that pass's second barrier
-    if (pass + 1 < kTopkPasses) {
+    if (pass + 1 < kPasses) {
       int *hn = hist[(pass + 1) & 1];
-      for (int i = tid; i < (1 << topk_pass_bits(pass + 1)); i += NT) hn[i] = 0;
+      for (int i = tid; i < (1 << topk_pass_bits(FB, pass + 1)); i += NT) hn[i] = 0;
     }
     __syncthreads();
-    if (tid < 32) {  // digits nbins-1 .. 0, nbins/32 per lane: find the one holding the k_rem-th key
-      const int bpl = nbins >> 5;
-      const int top = nbins - 1 - tid * bpl;  // this lane's digits: top, top-1, ..., top-bpl+1
-      const int hid0 = prefix == 0u ? n_hid : 0;  // hidden slots counted in bin 0
+    const int hid0 = prefix == 0u ? n_hid : 0;  // hidden slots counted in bin 0
+    if constexpr (FB == 8) {
+      if (tid < 32) {  // digits nbins-1 .. 0, nbins/32 per lane: find the one holding the k_rem-th key
+        const int bpl = nbins >> 5;
+        const int top = nbins - 1 - tid * bpl;  // this lane's digits: top, top-1, ..., top-bpl+1
+        int sum = 0;
+        for (int i = 0; i < bpl; ++i) sum += h[top - i];
+        if (top - bpl + 1 == 0) sum -= hid0;
+        int incl = sum;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const int x = __shfl_up_sync(0xffffffffu, incl, d);
+          if (tid >= d) incl += x;
+        }
+        int above = incl - sum;  // keys in higher digits than this lane's first
+        if (above < k_rem && k_rem <= incl) {  // exactly one lane
+          for (int i = 0; i < bpl; ++i) {
+            const int c = h[top - i] - (top - i == 0 ? hid0 : 0);
+            if (k_rem <= above + c) {
+              pick[pass & 1][0] = top - i;
+              pick[pass & 1][1] = above;
+              pick[pass & 1][2] = c;
+              break;
+            }
+            above += c;
+          }
+        }
+      }
+    } else {  // every thread takes nbins/NT digits, highest first by thread; a CTA-wide scan
+      constexpr int kMaxBpt = (1 << FB) / NT;
+      const int bpt = nbins / NT;
+      const int top = nbins - 1 - tid * bpt;  // this thread's digits: top, ..., top-bpt+1
+      int c[kMaxBpt];
       int sum = 0;
-      for (int i = 0; i < bpl; ++i) sum += h[top - i];
-      if (top - bpl + 1 == 0) sum -= hid0;
+#pragma unroll
+      for (int i = 0; i < kMaxBpt; ++i) {
+        c[i] = i < bpt ? h[top - i] : 0;
+        sum += c[i];
+      }
+      if (top - bpt + 1 == 0) sum -= hid0;
       int incl = sum;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
         const int x = __shfl_up_sync(0xffffffffu, incl, d);
-        if (tid >= d) incl += x;
+        if (lane >= d) incl += x;
       }
-      int above = incl - sum;  // keys in higher digits than this lane's first
-      if (above < k_rem && k_rem <= incl) {  // exactly one lane
-        for (int i = 0; i < bpl; ++i) {
-          const int c = h[top - i] - (top - i == 0 ? hid0 : 0);
-          if (k_rem <= above + c) {
+      if (lane == 31) wtot[warp] = incl;
+      __syncthreads();
+      int above = incl - sum;  // keys in higher digits than this thread's first
+      for (int w = 0; w < warp; ++w) above += wtot[w];
+      if (above < k_rem && k_rem <= above + sum) {  // exactly one thread
+#pragma unroll
+        for (int i = 0; i < kMaxBpt; ++i) {
+          const int ci = c[i] - (top - i == 0 ? hid0 : 0);
+          if (i < bpt && k_rem <= above + ci) {
             pick[pass & 1][0] = top - i;
             pick[pass & 1][1] = above;
-            pick[pass & 1][2] = c;
+            pick[pass & 1][2] = ci;
             break;
           }
-          above += c;
+          above += ci;
         }
       }
     }
@@ -710,11 +760,11 @@ cudaError_t launch_dsa_topk(const float *scores, int64_t B, int T, int S, int to
   if (rows > 0x7fffffff) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(rows));
   if (S <= 256 * 16)
-    dsa_topk_kernel<256, 16><<<grid, 256, 0, stream>>>(scores, T, S, n_sel, sel);
+    dsa_topk_kernel<256, 16, SRM_TOPK_FIRST_BITS><<<grid, 256, 0, stream>>>(scores, T, S, n_sel, sel);
   else if (S <= 1024 * 16)
-    dsa_topk_kernel<1024, 16><<<grid, 1024, 0, stream>>>(scores, T, S, n_sel, sel);
+    dsa_topk_kernel<1024, 16, SRM_TOPK_FIRST_BITS><<<grid, 1024, 0, stream>>>(scores, T, S, n_sel, sel);
   else if (S <= 512 * 64)
-    dsa_topk_kernel<512, 64><<<grid, 512, 0, stream>>>(scores, T, S, n_sel, sel);
+    dsa_topk_kernel<512, 64, SRM_TOPK_FIRST_BITS><<<grid, 512, 0, stream>>>(scores, T, S, n_sel, sel);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

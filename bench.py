@@ -41,10 +41,12 @@ KERNELS_PER_DENSE_STEP = 4  # identity rows 1 + up 1 + down 1 + combine 1
 def kernels_per_step(w, num_sms=148):
     """Kernel launches of one routed step: the router (one kernel: logits,
     selection and gates, with the router weights split once at pack time);
-    permutation (one CTA for small batches, else histogram + scan + scatter);
-    token gather (invert + scatter); up GEMM; down GEMM; combine."""
+    permutation (one CTA for small batches, one launch over at most one
+    1024-assignment chunk per SM, else histogram + scan + scatter); token gather
+    (invert + scatter); up GEMM; down GEMM; combine."""
     route = 1
-    permute = 1 if w.T * w.K <= 4096 else 3
+    n = w.T * w.K
+    permute = 1 if n <= 4096 or -(-n // 1024) <= num_sms else 3
     return route + permute + 2 + 1 + 1 + 1
 
 

@@ -242,7 +242,8 @@ moe_status_t moe_permute(const moe_cfg_t *cfg, const int32_t *topk_idx, int32_t 
   }
   return cuda_status(srm::launch_permute(
       topk_idx, static_cast<int>(cfg->T), cfg->E, cfg->K, cfg->has_shared, counts, offsets, sorted,
-      reinterpret_cast<int32_t *>(wsb + L.scratch), reinterpret_cast<int *>(wsb + L.err), s));
+      reinterpret_cast<int32_t *>(wsb + L.scratch), reinterpret_cast<int *>(wsb + L.err), s,
+      reinterpret_cast<int *>(wsb + L.err + 96), num_sms()));
 }
 
 namespace {

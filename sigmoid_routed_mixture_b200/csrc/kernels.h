@@ -65,11 +65,12 @@ cudaError_t launch_route(const CUtensorMap &tmap_x, const CUtensorMap &tmap_w, c
                          int32_t *idx, float *gate, float *margin, float *logits, int *err,
                          int num_sms, cudaStream_t stream);
 
-// chunk scratch: int32 [E * nchunks]
+// chunk scratch: int32 [E * nchunks]; with a grid counter (one int, zeroed
+// here) and at most num_sms chunks, one fused launch instead of three
 int permute_num_chunks(int64_t n_assign);
 cudaError_t launch_permute(const int32_t *idx, int T, int E, int K, int has_shared, int32_t *counts,
                            int32_t *offsets, int32_t *sorted, int32_t *chunk_scratch, int *err,
-                           cudaStream_t stream);
+                           cudaStream_t stream, int *grid_counter = nullptr, int num_sms = 0);
 
 // token rows in expert-sorted order: xs[p] = x[token of sorted[p]]; pos is
 // int32 scratch [rows] (row id -> sorted position)

@@ -11,7 +11,9 @@
 //              (routed row id t*K + slot; shared row id T*K + t).
 // No step depends on the order in which atomics land: the per-chunk
 // histograms only count, and the scatter ranks entries with warp matches and
-// per-warp counts in a fixed order.
+// per-warp counts in a fixed order.  Three forms: one CTA for small batches;
+// one launch with a grid barrier while the 1024-assignment chunks fit one CTA
+// per SM; histogram, scan and scatter kernels beyond that.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -252,9 +254,124 @@ __global__ void __launch_bounds__(pm::SMALL_THREADS)
     for (int t = tid; t < T; t += pm::SMALL_THREADS) sorted[routed + t] = n + t;
 }
 
+// Chunked batches whose chunks fit one CTA per SM: the same histogram ->
+// scan -> stable scatter in ONE launch (three launches and a one-CTA scan
+// otherwise).  Warp w of CTA c owns the contiguous assignments
+// [c*CHUNK + w*CHUNK/WARPS, +CHUNK/WARPS) in registers:
+//   1) each warp counts its entries per expert (warp matches, one writer per
+//      expert per step); per expert, an exclusive scan over the warps, and the
+//      chunk's count published to scratch[c * E + e];
+//   2) a grid barrier (one arrival per CTA on a counter zeroed before the
+//      launch, a bounded wait);
+//   3) every CTA reads all chunks' counts: per expert the total and the counts
+//      of the chunks before its own; the exclusive scan of the totals over the
+//      experts gives the group offsets (the same numbers in every CTA; CTA 0
+//      writes counts and offsets);
+//   4) each warp writes every entry to its expert's running position: entries
+//      ascending (chunk, warp, step, lane) keep ascending positions.
+namespace pm {
+constexpr int FUSED_STEPS = CHUNK / THREADS;  // 32-entry steps per warp
+static_assert(THREADS == MAX_E, "one thread per expert in the offset scan");
+}  // namespace pm
+
+__global__ void __launch_bounds__(pm::THREADS)
+    permute_fused_kernel(const int32_t *__restrict__ idx, int n, int E, int T, int has_shared,
+                         int32_t *__restrict__ scratch, int *grid_counter, int32_t *__restrict__ counts,
+                         int32_t *__restrict__ offsets, int32_t *__restrict__ sorted, int *err) {
+  __shared__ int whist[pm::WARPS][pm::MAX_E];  // counts, then each warp's running positions
+  __shared__ int base[pm::MAX_E];               // first position of this chunk's entries per expert
+  __shared__ int wsum[pm::WARPS];
+  __shared__ int routed_total;
+  const int c = blockIdx.x, nchunks = gridDim.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int k = tid; k < pm::WARPS * pm::MAX_E; k += pm::THREADS) (&whist[0][0])[k] = 0;
+  const int seg0 = c * pm::CHUNK + warp * (pm::CHUNK / pm::WARPS);
+  int e_reg[pm::FUSED_STEPS];
+#pragma unroll
+  for (int j = 0; j < pm::FUSED_STEPS; ++j) {
+    const int i = seg0 + j * 32 + lane;
+    int e = -1;
+    if (i < n) {
+      e = idx[i];
+      if (e < 0 || e >= E) {
+        record_error(err, MOE_ERR_BAD_INDEX);
+        e = -1;
+      }
+    }
+    e_reg[j] = e;
+  }
+  __syncthreads();
+  const unsigned lt_mask = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < pm::FUSED_STEPS; ++j) {
+    const int e = e_reg[j];
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && __popc(same & lt_mask) == 0) whist[warp][e] += __popc(same);
+    __syncwarp();
+  }
+  __syncthreads();
+  if (tid < E) {
+    int run = 0;
+    for (int w = 0; w < pm::WARPS; ++w) {
+      const int v = whist[w][tid];
+      whist[w][tid] = run;
+      run += v;
+    }
+    scratch[c * E + tid] = run;
+  }
+  __syncthreads();
+  if (!grid_barrier(grid_counter, nchunks, err)) return;
+  int total = 0, before = 0;
+  if (tid < E) {
+    for (int cc = 0; cc < nchunks; ++cc) {
+      const int v = __ldcg(scratch + cc * E + tid);
+      total += v;
+      if (cc < c) before += v;
+    }
+  }
+  int incl = total;  // inclusive scan of the totals over the experts: within the warp, then across
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int pre = 0;
+  for (int w = 0; w < warp; ++w) pre += wsum[w];
+  const int excl = pre + incl - total;
+  if (tid < E) {
+    base[tid] = excl + before;
+    if (c == 0) {
+      counts[tid] = total;
+      offsets[tid] = excl;
+    }
+  }
+  if (tid == pm::THREADS - 1) routed_total = pre + incl;
+  __syncthreads();
+  const int routed = routed_total;
+  if (c == 0 && tid == 0) {
+    counts[E] = has_shared ? T : 0;
+    offsets[E] = routed;
+    offsets[E + 1] = routed + (has_shared ? T : 0);
+  }
+#pragma unroll
+  for (int j = 0; j < pm::FUSED_STEPS; ++j) {
+    const int e = e_reg[j];
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(same & lt_mask);
+    if (e >= 0) sorted[base[e] + whist[warp][e] + rank] = seg0 + j * 32 + lane;
+    __syncwarp();
+    if (e >= 0 && rank == 0) whist[warp][e] += __popc(same);
+    __syncwarp();
+  }
+  if (has_shared)
+    for (int t = c * pm::THREADS + tid; t < T; t += nchunks * pm::THREADS) sorted[routed + t] = n + t;
+}
+
 cudaError_t launch_permute(const int32_t *idx, int T, int E, int K, int has_shared, int32_t *counts,
                            int32_t *offsets, int32_t *sorted, int32_t *scratch, int *err,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, int *grid_counter, int num_sms) {
   const int n = T * K;
   if (n <= pm::SMALL_N) {
     permute_small_kernel<<<1, pm::SMALL_THREADS, 0, stream>>>(idx, n, E, T, has_shared, counts,
@@ -262,6 +379,13 @@ cudaError_t launch_permute(const int32_t *idx, int T, int E, int K, int has_shar
     return cudaGetLastError();
   }
   const int nchunks = permute_num_chunks(n);
+  if (grid_counter && nchunks <= num_sms) {
+    cudaError_t e = cudaMemsetAsync(grid_counter, 0, sizeof(int), stream);
+    if (e != cudaSuccess) return e;
+    permute_fused_kernel<<<nchunks, pm::THREADS, 0, stream>>>(idx, n, E, T, has_shared, scratch,
+                                                              grid_counter, counts, offsets, sorted, err);
+    return cudaGetLastError();
+  }
   permute_hist_kernel<<<nchunks, pm::THREADS, 0, stream>>>(idx, n, E, nchunks, scratch, err);
   permute_scan_kernel<<<1, pm::SCAN_THREADS, 0, stream>>>(scratch, E, nchunks, T, has_shared, counts,
                                                           offsets);

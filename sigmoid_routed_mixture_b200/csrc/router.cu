@@ -251,29 +251,6 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// Grid barrier of a launch whose CTAs are all resident together (the grid is
-// at most one CTA per SM): one arrival per CTA on a counter that is zero
-// before the launch, then a wait bounded by kWaitLimitNs.  Returns false (and
-// records MOE_ERR_TIMEOUT) if the wait ran out.
-__device__ __forceinline__ bool grid_barrier(int *counter, int n_ctas, int *err) {
-  __shared__ int ok;
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(counter, 1);
-    const uint64_t t0 = global_timer_ns();
-    int seen = 0;
-    while (true) {
-      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(seen) : "l"(counter) : "memory");
-      if (seen >= n_ctas) break;
-      if (global_timer_ns() - t0 > kWaitLimitNs) break;
-    }
-    ok = seen >= n_ctas;
-    if (!ok) record_error(err, MOE_ERR_TIMEOUT);
-  }
-  __syncthreads();
-  return ok != 0;
-}
-
 // Selection for a staged tile of z rows, one thread per (row, half of the
 // experts): the thread scans experts [hf*HALF, min(E, (hf+1)*HALF)) of its row
 // in index order (s = sigmoid(z), key = s + b) into a sorted top-LK list

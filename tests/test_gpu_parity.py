@@ -205,15 +205,51 @@ def test_zero_tokens():
     assert np.all(res["counts"] == 0) and np.all(res["offsets"] == 0)
 
 
-def test_out_of_range_expert_id_is_flagged():
-    w = W.WORKLOADS["tiny"]
+@pytest.mark.parametrize("T", [64, 4096, 65536])  # one-CTA, fused and three-kernel permutation
+def test_out_of_range_expert_id_is_flagged(T):
+    """An id past E and a negative one are flagged MOE_ERR_BAD_INDEX; the next
+    call with good ids on the same workspace is exact."""
+    w = W.WORKLOADS["tiny"].replace(T=T)
     cfg = moe.Config.of(w)
-    idx = torch.randint(0, w.E, (w.T, w.K), dtype=torch.int32, device="cuda")
-    idx[7, 2] = w.E + 3
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3300 + T)
+    idx = torch.randint(0, w.E, (w.T, w.K), dtype=torch.int32, device="cuda", generator=g)
+    bad = idx.clone()
+    bad[7, 2] = w.E + 3
+    bad[T - 1, 0] = -1
     ws = moe.workspace(cfg)
-    moe.permute(cfg, idx, ws)
+    moe.permute(cfg, bad, ws)
     assert moe.device_error(ws) == 5
     assert moe.device_error(ws) == 0  # read clears it
+    counts, offsets, srt = moe.permute(cfg, idx, ws)
+    want = O.permute(idx.cpu().numpy(), w.E, w.has_shared)
+    assert moe.device_error(ws) == 0
+    for got, ref in zip((counts, offsets, srt), want):
+        assert np.array_equal(got.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("T,K,E,has_shared", [
+    (1025, 4, 16, True),      # 5 chunks, the last one ragged: one fused launch
+    (4097, 1, 7, False),      # K = 1, no shared expert
+    (16384, 8, 256, True),    # the GLM-5 prefill shape: 128 chunks
+    (37888, 4, 16, True),     # 148 chunks: the most one fused launch takes
+    (38144, 4, 16, True),     # 149 chunks: histogram, scan and scatter kernels
+])
+def test_permutation_paths_match_the_oracle(T, K, E, has_shared):
+    """The permutation is index work: bit-exact against the oracle's counting
+    sort on either side of the fused path's chunk limit."""
+    w = W.WORKLOADS["tiny"].replace(T=T, K=K, E=E, has_shared=has_shared)
+    cfg = moe.Config.of(w)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3400 + T)
+    idx = torch.randint(0, E, (T, K), dtype=torch.int32, device="cuda", generator=g)
+    ws = moe.workspace(cfg)
+    for _ in range(2):  # the second call reuses the workspace and its grid counter
+        counts, offsets, srt = moe.permute(cfg, idx, ws)
+        assert moe.device_error(ws) == 0
+        want = O.permute(idx.cpu().numpy(), E, has_shared)
+        for got, ref in zip((counts, offsets, srt), want):
+            assert np.array_equal(got.cpu().numpy(), ref)
 
 
 @pytest.mark.parametrize("T", [64, 4096])  # single-CTA tiles, CTA-pair tiles

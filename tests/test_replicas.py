@@ -112,13 +112,16 @@ def test_tensor_peak_follows_the_timed_loop_length():
 
 def test_launches_per_step_match_the_kernel_structure():
     """The bench's gpu_launches claim: one router kernel (logits, selection and
-    gates; the router weights are split once at pack time), the one-CTA
-    permutation for small batches or histogram + scan + scatter, invert,
-    gather, up, down, combine: 7 kernels at decode, 9 at prefill."""
+    gates; the router weights are split once at pack time), the permutation
+    (one CTA for small batches, one fused launch while the 1024-assignment
+    chunks fit one per SM, else histogram + scan + scatter), invert, gather,
+    up, down, combine: 7 kernels at decode and at the 16384-token prefill, 9
+    at 65536 tokens."""
     sys.path.insert(0, ROOT)
     import bench
     from sigmoid_routed_mixture_b200 import workloads as W
 
     assert bench.kernels_per_step(W.WORKLOADS["glm5_decode"]) == 7
-    assert bench.kernels_per_step(W.WORKLOADS["glm5_prefill"]) == 9
+    assert bench.kernels_per_step(W.WORKLOADS["glm5_prefill"]) == 7
+    assert bench.kernels_per_step(W.WORKLOADS["glm5_prefill"].replace(T=65536)) == 9
     assert bench.DSA_KERNELS_PER_STEP == 3  # plan, scores, top-k

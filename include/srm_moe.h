@@ -180,7 +180,11 @@ moe_status_t moe_route_packed(const moe_cfg_t *cfg, const void *x, const void *w
  *             of the r-th row of group g in ascending token order; a routed
  *             row id is t*K + slot, a shared row id is T*K + t.
  *   ws, ws_bytes: workspace of at least moe_workspace_size(cfg) bytes.
- * An id outside [0, E) is skipped and flagged MOE_ERR_BAD_INDEX on the device. */
+ * An id outside [0, E) is skipped and flagged MOE_ERR_BAD_INDEX on the device.
+ * Up to 151552 assignments (at most one 1024-assignment chunk per SM) this is
+ * one launch whose CTAs meet at a grid barrier bounded in time: MOE_ERR_TIMEOUT
+ * on the device if they cannot all be resident at once (e.g. another stream's
+ * kernels hold the SMs), the outputs then undefined. */
 moe_status_t moe_permute(const moe_cfg_t *cfg, const int32_t *topk_idx, int32_t *counts,
                          int32_t *offsets, int32_t *sorted, void *ws, size_t ws_bytes, void *stream);
 

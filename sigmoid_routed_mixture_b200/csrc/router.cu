@@ -725,7 +725,7 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
 
   if (kSplit) {
     // Every CTA's partials are written; after the grid barrier CTA c takes the
-    // tokens t = c, c + C, c + 2C, ... (C CTAs in the grid), RB rows at a time.
+    // tokens t = c, c + C, c + 2C, ... (C CTAs in the grid), a batch of rows at a time.
     // All its threads sum the S partials of those rows: groups of eight splits
     // in a fixed tree ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7)) (a
     // shorter last group in split order), then the group sums in group order
@@ -751,8 +751,12 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
     const float4 *zp4 = reinterpret_cast<const float4 *>(zp);
     float4 *part = reinterpret_cast<float4 *>(zs + kRowBatch * ZS);  // [groups][kRowBatch][V]
     const int n_warps = blockDim.x >> 5;
-    for (int r0 = 0; r0 < n_rows; r0 += kRowBatch) {
-      const int nb = min(kRowBatch, n_rows - r0);
+    // rows per batch: all of the CTA's rows (up to 128) when the splits form one
+    // group, so one pass of loads and one round of warps cover them; kRowBatch
+    // when the group sums need the `part` buffer
+    const int rb = groups == 1 ? BM : kRowBatch;
+    for (int r0 = 0; r0 < n_rows; r0 += rb) {
+      const int nb = min(rb, n_rows - r0);
       // Up to three items per thread, all their loads issued before any sum, so
       // one round trip to L2 covers the thread's share of the splits.
       const int n_items = groups * nb * V;

@@ -763,8 +763,8 @@ cudaError_t launch_dsa_topk(const float *scores, int64_t B, int T, int S, int to
     dsa_topk_kernel<256, 16, SRM_TOPK_FIRST_BITS><<<grid, 256, 0, stream>>>(scores, T, S, n_sel, sel);
   else if (S <= 1024 * 16)
     dsa_topk_kernel<1024, 16, SRM_TOPK_FIRST_BITS><<<grid, 1024, 0, stream>>>(scores, T, S, n_sel, sel);
-  else if (S <= 512 * 64)
-    dsa_topk_kernel<512, 64, SRM_TOPK_FIRST_BITS><<<grid, 512, 0, stream>>>(scores, T, S, n_sel, sel);
+  else if (S <= 1024 * 32)  // (512 threads x 64 keys: 24.8 against 22.7 us for 64 rows of 32768 keys)
+    dsa_topk_kernel<1024, 32, SRM_TOPK_FIRST_BITS><<<grid, 1024, 0, stream>>>(scores, T, S, n_sel, sel);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

@@ -33,11 +33,10 @@
 //          together) meet at a bounded grid barrier, then every CTA takes
 //          some tokens, sums the S partials in a fixed order (deterministic)
 //          and selects: a CTA-wide ranking for a single token, otherwise K + 1
-//          rounds of a warp arg-max (key descending, index ascending) per token.
+//          rounds of a warp arg-max (key descending, index ascending) per token
+//          (two tokens' rounds interleaved per warp up to 64 experts).
 #include <cuda.h>
 #include <math.h>
-
-#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"

@@ -97,6 +97,19 @@ def test_visible_pairs_count():
         assert bench.dsa_visible_pairs(w) == brute
 
 
+def test_router_workloads_name_their_shapes():
+    """The router-only bench lines carry the block's shape in their metric."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from sigmoid_routed_mixture_b200 import workloads as W
+
+    for name, block in bench.ROUTER_WORKLOADS.items():
+        w = W.WORKLOADS[block]
+        m = bench.router_metric(w)
+        assert ("%d experts top-%d, H %d" % (w.E, w.K, w.H)) in m
+        assert ("GLM-5" in m) == block.startswith("glm5")
+
+
 def test_tensor_peak_follows_the_timed_loop_length():
     """A tensor-bound kernel timed inside a loop of at least 0.5 s is judged
     against the sustained (power-capped) bf16 figure, a short loop against the
